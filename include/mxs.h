@@ -1,0 +1,229 @@
+/*
+ * mxs.h -- C ABI of libmxs: mixed-width MXINT quantisation and GEMM for B200.
+ *
+ * The method is MXSens (Sensitivity-Aware Mixed-Precision Quantization for
+ * Efficient LLM Inference, arXiv 2607.17733).  Citations below name the page
+ * and section the operation comes from:
+ *   [TS]  gist.science technical summary ("Technische Samenvatting") §1-§5;
+ *   [ABS] the paper's abstract (insight.artgrammer.co.kr);
+ *   [RP]  researchpod.app summary.
+ * The pages publish no formula beyond H = X^T X, no bit layout and no API;
+ * the fixed readings used by this library are stated at each entry point.
+ *
+ * Conventions (all entry points):
+ *   - Pointers marked (device) are CUDA device pointers on the current device;
+ *     (host) are host pointers.  The caller allocates and owns every buffer,
+ *     including workspaces; the library never allocates device memory.
+ *   - Matrices are row-major with unit stride along K (the input dimension);
+ *     ld* arguments are row pitches in ELEMENTS.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default).
+ *     Device work is stream-ordered and asynchronous; arguments are checked
+ *     on the host before any launch and a non-MXS_OK status means nothing was
+ *     launched.  mxs_allocate is the one call that synchronises the stream
+ *     (it returns host-side counts).
+ *   - Device-side failures (a bounded wait that expired) are recorded in a
+ *     per-device status word and returned by mxs_sync.
+ *   - Calls are thread-safe apart from that shared status word.
+ */
+#ifndef MXS_H
+#define MXS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MXS_OK = 0,
+    MXS_ERR_ARG = 1,       /* NULL pointer, negative size, bad enum            */
+    MXS_ERR_SHAPE = 2,     /* inconsistent shapes / layouts                    */
+    MXS_ERR_ALIGN = 3,     /* pointer or pitch misaligned (16 bytes required)  */
+    MXS_ERR_DTYPE = 4,     /* unsupported element type                         */
+    MXS_ERR_BUDGET = 5,    /* the fixed 8-bit blocks alone exceed the budget   */
+    MXS_ERR_CUDA = 6,      /* a CUDA runtime call failed                       */
+    MXS_ERR_TIMEOUT = 7,   /* a device-side bounded wait expired               */
+    MXS_ERR_DEVICE = 8,    /* the current device is not sm_100                 */
+    MXS_ERR_WORKSPACE = 9  /* workspace NULL, misaligned or too small          */
+} mxs_status;
+
+typedef enum { MXS_F32 = 0, MXS_BF16 = 1 } mxs_dtype;
+
+/* One K-segment of the mixed-width layout.  Segments are stored in the order
+ * 8-bit, 6-bit, 4-bit; a segment holds k_real columns followed by zero
+ * padding up to k_pad = 32*ceil(k_real/32) positions and starts at padded
+ * position k_off.  [TS §2.2: three mantissa widths 4/6/8; TS §2.3 last
+ * paragraph: the mixed widths live inside MXINT's 32-value blocks.] */
+typedef struct {
+    int32_t bits;
+    int64_t k_real;
+    int64_t k_pad;
+    int64_t k_off;
+} mxs_segment;
+
+/* Column layout of one linear layer: perm (device, K entries, or NULL for
+ * the identity) lists the original column of each real position, segment by
+ * segment, ascending within a segment.  Build it with mxs_layout_make. */
+typedef struct {
+    int64_t K;
+    int64_t K_pad;
+    mxs_segment seg[3];
+    const int32_t *perm;
+} mxs_layout;
+
+/* A quantised matrix: `rows` rows in layout `lay`.  For segment g:
+ *   codes[g]  (device) rows x code_pitch[g] bytes; row r holds k_pad codes of
+ *             width bits, two's complement, packed: 4-bit two per byte (even
+ *             position in the low nibble), 6-bit four per three bytes (a
+ *             24-bit little-endian group, position 4j+i at bits 6i..6i+5),
+ *             8-bit one per byte;
+ *   scales[g] (device) rows x scale_pitch[g] bytes; one E8M0 byte per block
+ *             of 32 positions: byte = e + 127, the block's value is
+ *             code * 2^(e - bits + 2).
+ * Pitches are multiples of 16 bytes (mxs_mxtensor_bytes gives them); the
+ * bytes beyond each row's payload are left as the caller set them.
+ * Empty segments (k_pad == 0) may have NULL pointers. */
+typedef struct {
+    int64_t rows;
+    mxs_layout lay;
+    uint8_t *codes[3];
+    int64_t code_pitch[3];
+    uint8_t *scales[3];
+    int64_t scale_pitch[3];
+} mxs_mxtensor;
+
+enum { MXS_ALLOC_FRACTIONS = 0, MXS_ALLOC_BUDGET = 1 };
+
+/* Bit-allocation policy.
+ *   MXS_ALLOC_FRACTIONS: n8 = round(p8*K), n6 = round(p6*K) (half up, exact
+ *     rational arithmetic on p = num/den), the rest 4-bit.
+ *   MXS_ALLOC_BUDGET: n8 = min(fixed8, K) -- the most sensitive columns, one
+ *     MXINT block when fixed8 = 32 [TS §2.2 8-bit, §2.3 fixed high-precision
+ *     block]; then greedy 6-bit upgrades of 32-column groups under an average
+ *     mantissa-bit budget num/den over all weight elements, E8M0 scales not
+ *     counted [TS §2.3 dynamic 6-bit allocation; TS §4 hardware overhead:
+ *     4 + 4*32/4096 = 4.03 bits for the fixed block alone]. */
+typedef struct {
+    int32_t mode;
+    int64_t num, den;
+    int64_t p8_num, p8_den;
+    int64_t p6_num, p6_den;
+    int64_t fixed8;
+} mxs_budget;
+
+/* Human-readable name of a status code (static storage). */
+const char *mxs_status_str(mxs_status st);
+
+/* Number of kernels this library has launched in this process so far. */
+int64_t mxs_launch_count(void);
+
+/* Waits for `stream`, then returns and clears the device status word of the
+ * current device: MXS_ERR_TIMEOUT if a bounded device wait expired since the
+ * last call, MXS_ERR_CUDA if the stream reported an error, else MXS_OK. */
+mxs_status mxs_sync(void *stream);
+
+/* Fills *out for K columns with counts = {n8, n6, n4} (host, summing to K)
+ * and perm (device, K entries; NULL for the identity, e.g. the K/V cache
+ * layout {0, 0, K}).  No device access; perm is stored, not read. */
+mxs_status mxs_layout_make(int64_t K, const int64_t counts[3], const int32_t *perm,
+                           mxs_layout *out);
+
+/* Pitches and byte sizes of the code and scale buffers of a `rows`-row
+ * tensor in layout *lay (host outputs, 3 entries each, zero for empty
+ * segments; pitches are multiples of 16 bytes). */
+mxs_status mxs_mxtensor_bytes(int64_t rows, const mxs_layout *lay,
+                              int64_t code_pitch[3], int64_t code_bytes[3],
+                              int64_t scale_pitch[3], int64_t scale_bytes[3]);
+
+/* ---------------------------------------------------------------------------
+ * mxs_sensitivity -- column sensitivity of one linear layer.
+ * [TS §2.1: column-wise sensitivity from the diagonal of H = X^T X.]
+ *   H[j] = (2/T) * sum_t X[t][j]^2                 (fp64)
+ *   E[j] = sum_i (W[i][j] - Q4(W)[i][j])^2          (fp64)
+ *   s[j] = H[j] * E[j]
+ * Q4 is the 4-bit MXINT code of each W row in blocks of 32 ORIGINAL columns
+ * (a short last block is zero-padded).  Rounding order: rows are summed in
+ * chunks of 64 from zero, in row order, and chunk sums are added in chunk
+ * order; the result is bit-identical for any launch configuration.
+ *   X (device): T x K, dtype xt, pitch ldx (elements); W (device): N x K,
+ *   dtype wt, pitch ldw.  H, E, s (device): K doubles each (E may be NULL).
+ *   ws (device, 256-byte aligned): mxs_sensitivity_workspace_bytes(T, N, K).
+ * T, N >= 1, K >= 1. */
+mxs_status mxs_sensitivity_workspace_bytes(int64_t T, int64_t N, int64_t K, size_t *bytes);
+mxs_status mxs_sensitivity(const void *X, mxs_dtype xt, int64_t T, int64_t K, int64_t ldx,
+                           const void *W, mxs_dtype wt, int64_t N, int64_t ldw,
+                           double *H, double *E, double *s,
+                           void *ws, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * mxs_allocate -- 4/6/8-bit widths for n_layers layers and their column
+ * permutations.  [TS §2.3: sort columns by sensitivity; the top block gets 8
+ * bits; a sensitivity-driven number of 6-bit columns under a global budget;
+ * the rest 4 bits.]
+ *   Ranking: s descending, ties to the lower column index.
+ *   Budget greedy (MXS_ALLOC_BUDGET): candidates are the next 32 ranked
+ *   4-bit columns of each layer (fewer at the tail); gain = layer_w[l] * sum
+ *   of their s (fp64, rank order), cost = 2 * N[l] * count bits; repeatedly
+ *   take the highest gain/cost (compared as gain_a*cost_b > gain_b*cost_a in
+ *   fp64, ties to the lower layer) and stop at the first that does not fit
+ *   sum_l N_l (4 K_l + 4 n8_l + 2 n6_l) * den <= num * sum_l N_l K_l.
+ *   Inputs: K, N (host, n_layers each); s (host array of n_layers device
+ *   pointers, K[l] doubles each, finite and >= 0); layer_w (host, n_layers,
+ *   or NULL = all 1).
+ *   Outputs: perm (host array of device pointers, K[l] int32 each: the
+ *   8-bit columns, then 6-bit, then 4-bit, ascending within each);
+ *   counts (host, 3*n_layers: n8, n6, n4 per layer).
+ *   ws (device): mxs_allocate_workspace_bytes(n_layers, K).
+ * Synchronises `stream`.  MXS_ERR_BUDGET if infeasible. */
+mxs_status mxs_allocate_workspace_bytes(int32_t n_layers, const int64_t *K, size_t *bytes);
+mxs_status mxs_allocate(int32_t n_layers, const int64_t *K, const int64_t *N,
+                        const double *const *s, const double *layer_w,
+                        const mxs_budget *budget, int32_t *const *perm,
+                        int64_t *counts, void *ws, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * mxs_quantize_weight / mxs_quantize_act -- mixed-width MXINT quantisation of
+ * the rows of a matrix (weights offline, activations and the K/V cache per
+ * forward).  [TS §2.2 triplet widths; TS §2.3 last paragraph; RP: widths apply
+ * to weights and activations; TS §4 W4A4KV4.]
+ *   Row r, segment g, padded position p: x = src[r][perm[real_off_g + p]]
+ *   for p < k_real, else 0.  For each block of 32 positions:
+ *     e = floor(log2(max |x|)) clamped to [-127, 127], -127 for a zero block;
+ *     scale byte = e + 127;
+ *     q = clamp(round_half_even(x / 2^(e - m + 2)), -(2^(m-1)-1), 2^(m-1)-1).
+ *   src (device): rows x K, dtype, pitch ld (elements), with rows ==
+ *   out->rows and K == out->lay.K; out: caller-owned buffers sized by
+ *   mxs_mxtensor_bytes.  The two entry points compute the same function;
+ *   the K/V cache uses mxs_quantize_act with the identity layout {0, 0, K}. */
+mxs_status mxs_quantize_weight(const void *W, mxs_dtype dt, int64_t N, int64_t ldw,
+                               const mxs_mxtensor *out, void *stream);
+mxs_status mxs_quantize_act(const void *A, mxs_dtype dt, int64_t M, int64_t lda,
+                            const mxs_mxtensor *out, void *stream);
+
+/* Decodes a quantised tensor to fp32 in padded-position order:
+ * out (device) rows x K_pad, pitch ldo (elements).  A checking aid. */
+mxs_status mxs_dequantize(const mxs_mxtensor *in, float *out, int64_t ldo, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * mxs_gemm -- the mixed-width MXINT linear layer.
+ * [TS §2.3 last paragraph and §4: the layer runs on the mixed MXINT blocks
+ * directly, about 1% of the work at more than 4 bits for a 4.03-bit budget.]
+ *   Y[m][n] = sum over padded positions k of deq(A)[m][k] * deq(W)[n][k]
+ *   with fp32 accumulation, rounded to bf16 (round to nearest even).
+ *   A, W: quantised tensors with identical segment tables (and perm);
+ *   Y (device): A->rows x W->rows bf16, pitch ldy (elements).
+ *   ws (device, 256-byte aligned): mxs_gemm_workspace_bytes(A, W); it holds
+ *   the operands re-coded for the tensor cores (4-bit codes as E4M3 with
+ *   their E8M0 block scales, 6/8-bit codes as exact bf16 values).
+ * Products of decoded values are exact; only the fp32 accumulation and the
+ * final bf16 rounding round. */
+mxs_status mxs_gemm_workspace_bytes(const mxs_mxtensor *A, const mxs_mxtensor *W, size_t *bytes);
+mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, void *Y, int64_t ldy,
+                    void *ws, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXS_H */

@@ -1,0 +1,240 @@
+// mxs_allocate.cu -- 4/6/8-bit allocation and column permutation.
+//
+// MXSens (arXiv 2607.17733), technical summary §2.3 (sensitivity-guided
+// allocation): per linear layer the columns are sorted by sensitivity; the 32
+// most sensitive always get 8-bit mantissas (one MXINT block, §2.2); a
+// sensitivity-driven number of columns get 6 bits so that a global average
+// budget B is met; the rest get 4 bits.  §4: at ~4.03 bits about 1% of the
+// work is at higher precision (4 + 4*32/4096 = 4.03125 for K = 4096).
+//
+// Fixed readings: ranking by s descending with ties to the lower column;
+// budget = average mantissa bits over all weight elements (scales excluded);
+// the 6-bit count comes from a greedy over 32-column groups ordered by
+// gain/cost across layers (gain = layer weight x summed s, cost = 2 N count
+// bits), stopping at the first group that does not fit.
+//
+// Device work: an all-pairs rank count (each thread ranks one column against
+// every other, staged through shared memory -- exact and order-free), the
+// group gains (one thread sums one group in rank order), and a single-CTA
+// stable compaction that writes the permutation segment by segment in
+// ascending column order.  The integer budget arithmetic and the cross-layer
+// greedy are a few hundred scalar steps and run on the host side of the call.
+#include <algorithm>
+#include <vector>
+
+#include "mxs_internal.cuh"
+
+namespace mxs {
+
+constexpr int kRankThreads = 256;
+constexpr int kRankTile = 2048;
+
+__global__ void __launch_bounds__(kRankThreads) rank_kernel(const double *s, int64_t K, int32_t *rank,
+                                                            int32_t *order) {
+  __shared__ double tile[kRankTile];
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * kRankThreads + threadIdx.x;
+  const double sj = j < K ? s[j] : 0.0;
+  int64_t r = 0;
+  for (int64_t base = 0; base < K; base += kRankTile) {
+    const int64_t n = min(static_cast<int64_t>(kRankTile), K - base);
+    __syncthreads();
+    for (int64_t i = threadIdx.x; i < n; i += kRankThreads) tile[i] = s[base + i];
+    __syncthreads();
+    if (j < K) {
+      for (int64_t i = 0; i < n; ++i) {
+        const double si = tile[i];
+        const int64_t gi = base + i;
+        r += (si > sj) || (si == sj && gi < j);
+      }
+    }
+  }
+  if (j < K) {
+    rank[j] = static_cast<int32_t>(r);
+    order[r] = static_cast<int32_t>(j);
+  }
+}
+
+// gains[g] = sum of s over ranks [n8 + 32 g, min(n8 + 32 g + 32, K)), in rank order.
+__global__ void group_gain_kernel(const double *s, const int32_t *order, int64_t K, int64_t n8,
+                                  int64_t ngroups, double *gains) {
+  const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (g >= ngroups) return;
+  const int64_t r0 = n8 + 32 * g, r1 = min(r0 + 32, K);
+  double sum = 0.0;
+  for (int64_t r = r0; r < r1; ++r) sum = __dadd_rn(sum, s[order[r]]);
+  gains[g] = sum;
+}
+
+constexpr int kPermThreads = 1024;
+
+// One CTA: columns in ascending order, segment of column j from its rank;
+// block-wide ballot scans give each column its slot inside its segment.
+__global__ void __launch_bounds__(kPermThreads) perm_kernel(const int32_t *rank, int64_t K, int64_t n8,
+                                                            int64_t n6, int32_t *perm) {
+  __shared__ int warp_cnt[3][kPermThreads / 32];
+  __shared__ int64_t running[3];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x < 3) running[threadIdx.x] = 0;
+  const int64_t base_of[3] = {0, n8, n8 + n6};
+  for (int64_t t0 = 0; t0 < K; t0 += kPermThreads) {
+    const int64_t j = t0 + threadIdx.x;
+    int seg = -1;
+    if (j < K) {
+      const int64_t r = rank[j];
+      seg = r < n8 ? 0 : (r < n8 + n6 ? 1 : 2);
+    }
+    int within[3];
+#pragma unroll
+    for (int g = 0; g < 3; ++g) {
+      const unsigned m = __ballot_sync(0xffffffffu, seg == g);
+      within[g] = __popc(m & ((1u << lane) - 1u));
+      if (lane == 0) warp_cnt[g][warp] = __popc(m);
+    }
+    __syncthreads();
+    if (seg >= 0) {
+      int64_t before = running[seg] + within[seg];
+      for (int w = 0; w < warp; ++w) before += warp_cnt[seg][w];
+      perm[base_of[seg] + before] = static_cast<int32_t>(j);
+    }
+    __syncthreads();
+    if (threadIdx.x < 3) {
+      int64_t tot = 0;
+      for (int w = 0; w < kPermThreads / 32; ++w) tot += warp_cnt[threadIdx.x][w];
+      running[threadIdx.x] += tot;
+    }
+    __syncthreads();
+  }
+}
+
+struct LayerWs {
+  int32_t *rank;
+  int32_t *order;
+  double *gains;
+};
+
+static size_t layer_ws_bytes(int64_t K) {
+  const int64_t ng = K / 32 + 2;
+  return static_cast<size_t>(round_up(K * 4, 256) * 2 + round_up(ng * 8, 256));
+}
+
+static int64_t round_half_up_frac(int64_t num, int64_t den, int64_t K) {
+  return (2 * num * K + den) / (2 * den);
+}
+
+}  // namespace mxs
+
+using namespace mxs;
+
+extern "C" mxs_status mxs_allocate_workspace_bytes(int32_t n_layers, const int64_t *K, size_t *bytes) {
+  if (n_layers < 1 || !K || !bytes) return MXS_ERR_ARG;
+  size_t b = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    if (K[l] < 1) return MXS_ERR_ARG;
+    b += layer_ws_bytes(K[l]);
+  }
+  *bytes = b;
+  return MXS_OK;
+}
+
+extern "C" mxs_status mxs_allocate(int32_t n_layers, const int64_t *K, const int64_t *N,
+                                   const double *const *s, const double *layer_w,
+                                   const mxs_budget *budget, int32_t *const *perm,
+                                   int64_t *counts, void *ws, size_t ws_bytes, void *stream) {
+  if (n_layers < 1 || !K || !N || !s || !budget || !perm || !counts) return MXS_ERR_ARG;
+  for (int l = 0; l < n_layers; ++l) {
+    if (K[l] < 1 || N[l] < 1 || !s[l] || !perm[l]) return MXS_ERR_ARG;
+    if (K[l] > INT32_MAX) return MXS_ERR_SHAPE;
+  }
+  const mxs_budget &B = *budget;
+  if (B.mode == MXS_ALLOC_FRACTIONS) {
+    if (B.p8_den <= 0 || B.p6_den <= 0 || B.p8_num < 0 || B.p6_num < 0) return MXS_ERR_ARG;
+  } else if (B.mode == MXS_ALLOC_BUDGET) {
+    if (B.den <= 0 || B.num < 0 || B.fixed8 < 0) return MXS_ERR_ARG;
+  } else {
+    return MXS_ERR_ARG;
+  }
+  size_t need = 0;
+  mxs_allocate_workspace_bytes(n_layers, K, &need);
+  if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MXS_ERR_WORKSPACE;
+  mxs_status st = check_device();
+  if (st != MXS_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+  std::vector<LayerWs> L(n_layers);
+  uint8_t *p = reinterpret_cast<uint8_t *>(ws);
+  for (int l = 0; l < n_layers; ++l) {
+    L[l].rank = reinterpret_cast<int32_t *>(p);
+    L[l].order = reinterpret_cast<int32_t *>(p + round_up(K[l] * 4, 256));
+    L[l].gains = reinterpret_cast<double *>(p + 2 * round_up(K[l] * 4, 256));
+    p += layer_ws_bytes(K[l]);
+    rank_kernel<<<static_cast<unsigned>((K[l] + kRankThreads - 1) / kRankThreads), kRankThreads, 0, cs>>>(
+        s[l], K[l], L[l].rank, L[l].order);
+    count_launch();
+  }
+
+  std::vector<int64_t> n8(n_layers, 0), n6(n_layers, 0);
+  if (B.mode == MXS_ALLOC_FRACTIONS) {
+    for (int l = 0; l < n_layers; ++l) {
+      n8[l] = std::min(round_half_up_frac(B.p8_num, B.p8_den, K[l]), K[l]);
+      n6[l] = std::min(round_half_up_frac(B.p6_num, B.p6_den, K[l]), K[l] - n8[l]);
+    }
+  } else {
+    __int128 cap = 0, used = 0;
+    for (int l = 0; l < n_layers; ++l) {
+      n8[l] = std::min(B.fixed8, K[l]);
+      cap += static_cast<__int128>(B.num) * N[l] * K[l];
+      used += static_cast<__int128>(B.den) * N[l] * (4 * K[l] + 4 * n8[l]);
+    }
+    if (used > cap) return MXS_ERR_BUDGET;
+    std::vector<std::vector<double>> gains(n_layers);
+    if (n_layers > 1) {
+      for (int l = 0; l < n_layers; ++l) {
+        const int64_t ng = (K[l] - n8[l] + 31) / 32;
+        gains[l].assign(static_cast<size_t>(std::max<int64_t>(ng, 1)), 0.0);
+        if (ng > 0) {
+          group_gain_kernel<<<static_cast<unsigned>((ng + 127) / 128), 128, 0, cs>>>(s[l], L[l].order, K[l],
+                                                                                    n8[l], ng, L[l].gains);
+          count_launch();
+          if (cudaMemcpyAsync(gains[l].data(), L[l].gains, static_cast<size_t>(ng) * 8,
+                              cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+            return MXS_ERR_CUDA;
+        }
+      }
+      if (cudaStreamSynchronize(cs) != cudaSuccess) return MXS_ERR_CUDA;
+    }
+    for (;;) {
+      int best = -1;
+      double best_gain = 0.0, best_cost = 0.0;
+      for (int l = 0; l < n_layers; ++l) {
+        const int64_t r0 = n8[l] + n6[l];
+        if (r0 >= K[l]) continue;
+        const int64_t cnt = std::min<int64_t>(32, K[l] - r0);
+        const double w = layer_w ? layer_w[l] : 1.0;
+        const double gain = n_layers > 1 ? w * gains[l][static_cast<size_t>(n6[l] / 32)] : 0.0;
+        const double cost = static_cast<double>(2 * N[l] * cnt);
+        if (best < 0 || gain * best_cost > best_gain * cost) {
+          best = l;
+          best_gain = gain;
+          best_cost = cost;
+        }
+      }
+      if (best < 0) break;
+      const int64_t r0 = n8[best] + n6[best];
+      const int64_t cnt = std::min<int64_t>(32, K[best] - r0);
+      const __int128 add = static_cast<__int128>(B.den) * 2 * N[best] * cnt;
+      if (used + add > cap) break;
+      used += add;
+      n6[best] += cnt;
+    }
+  }
+
+  for (int l = 0; l < n_layers; ++l) {
+    perm_kernel<<<1, kPermThreads, 0, cs>>>(L[l].rank, K[l], n8[l], n6[l], perm[l]);
+    count_launch();
+    counts[3 * l + 0] = n8[l];
+    counts[3 * l + 1] = n6[l];
+    counts[3 * l + 2] = K[l] - n8[l] - n6[l];
+  }
+  if (cudaGetLastError() != cudaSuccess) return MXS_ERR_CUDA;
+  return cuda_status(cudaStreamSynchronize(cs));
+}

@@ -1,0 +1,113 @@
+"""Host-only checks of the C ABI: the library loads, exports every entry point
+declared in include/mxs.h, and rejects bad arguments before any launch.
+No call here touches a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mxs.h")
+
+
+@pytest.fixture(scope="module")
+def capi():
+    from mx_microscaling_mixed_b200 import build
+    build.build()
+    from mx_microscaling_mixed_b200 import capi as c
+    return c
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mxs_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_symbols_exported(capi):
+    names = _declared()
+    assert len(names) >= 14
+    lib = ctypes.CDLL(capi._LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(capi.EXPORTS)
+
+
+def test_status_strings(capi):
+    for st in range(10):
+        assert capi.mxs_status_str(st).startswith(capi.STATUS[st])
+
+
+def test_layout_make_and_sizes(capi):
+    lay = capi.mxs_layout_make(256, (13, 38, 205))
+    segs = [(s.bits, s.k_real, s.k_pad, s.k_off) for s in lay.c.seg]
+    assert segs == [(8, 13, 32, 0), (6, 38, 64, 32), (4, 205, 224, 96)]
+    assert lay.K_pad == 320
+    cp, cb, sp, sb = capi.mxs_mxtensor_bytes(256, lay)
+    assert cp == [32, 48, 112] and cb == [256 * 32, 256 * 48, 256 * 112]
+    assert sp == [16, 16, 16] and sb == [256 * 16] * 3
+    kv = capi.mxs_layout_make(128, (0, 0, 128))
+    cp, cb, sp, sb = capi.mxs_mxtensor_bytes(65536, kv)
+    assert cp == [0, 0, 64] and sp == [0, 0, 16]
+
+
+def test_layout_rejects_bad_counts(capi):
+    with pytest.raises(capi.MxsError) as e:
+        capi.mxs_layout_make(10, (3, 3, 3))
+    assert e.value.status == 2
+    with pytest.raises(capi.MxsError):
+        capi.mxs_layout_make(10, (-1, 5, 6))
+
+
+def test_workspace_queries(capi):
+    need = ctypes.c_size_t(0)
+    assert capi._lib.mxs_sensitivity_workspace_bytes(2048, 4096, 4096, ctypes.byref(need)) == 0
+    assert need.value == (32 + 64) * 4096 * 8
+    K = (ctypes.c_int64 * 1)(4096)
+    assert capi._lib.mxs_allocate_workspace_bytes(1, K, ctypes.byref(need)) == 0
+    assert need.value > 2 * 4096 * 4
+    assert capi._lib.mxs_sensitivity_workspace_bytes(0, 1, 1, ctypes.byref(need)) == 1
+
+
+def _fake_tensor(capi, rows, lay, base=1 << 20):
+    t = capi.MXTensorC()
+    t.rows = rows
+    t.lay = lay.c
+    cp, cb, sp, sb = capi.mxs_mxtensor_bytes(rows, lay)
+    for g in range(3):
+        t.codes[g] = base + 4096 * g if cb[g] else None
+        t.scales[g] = base + 65536 + 4096 * g if sb[g] else None
+        t.code_pitch[g] = cp[g]
+        t.scale_pitch[g] = sp[g]
+    return t
+
+
+def test_gemm_argument_checks(capi):
+    lay = capi.mxs_layout_make(256, (32, 64, 160))
+    A = _fake_tensor(capi, 100, lay)
+    W = _fake_tensor(capi, 300, lay)
+    need = ctypes.c_size_t(0)
+    assert capi._lib.mxs_gemm_workspace_bytes(ctypes.byref(A), ctypes.byref(W), ctypes.byref(need)) == 0
+    assert need.value >= 100 * 96 * 2 + 300 * 96 * 2 + 100 * 160 + 300 * 160
+    # different layouts -> MXS_ERR_SHAPE, no launch
+    lay2 = capi.mxs_layout_make(256, (32, 32, 192))
+    W2 = _fake_tensor(capi, 300, lay2)
+    assert capi._lib.mxs_gemm(ctypes.byref(A), ctypes.byref(W2), 1 << 24, 300, 1 << 26, 1 << 30, None) == 2
+    # misaligned code pointer -> MXS_ERR_ALIGN
+    A.codes[2] = (1 << 20) + 8
+    assert capi._lib.mxs_gemm(ctypes.byref(A), ctypes.byref(W), 1 << 24, 300, 1 << 26, 1 << 30, None) == 3
+    # ldy < N -> MXS_ERR_SHAPE
+    A.codes[2] = 1 << 21
+    assert capi._lib.mxs_gemm(ctypes.byref(A), ctypes.byref(W), 1 << 24, 299, 1 << 26, 1 << 30, None) == 2
+
+
+def test_quantize_argument_checks(capi):
+    lay = capi.mxs_layout_make(64, (0, 0, 64))
+    t = _fake_tensor(capi, 8, lay)
+    # rows mismatch
+    assert capi._lib.mxs_quantize_act(1 << 20, 1, 9, 64, ctypes.byref(t), None) == 2
+    # bad dtype
+    assert capi._lib.mxs_quantize_act(1 << 20, 7, 8, 64, ctypes.byref(t), None) == 4
+    # ld < K
+    assert capi._lib.mxs_quantize_weight(1 << 20, 0, 8, 32, ctypes.byref(t), None) == 2

@@ -130,3 +130,16 @@ def test_all_4bit_layout_equals_plain_blockwise_product():
                 out[r, 32 * b:32 * b + 32] = [float(brute.code_value(c, e, 4)) for c in q]
         return out
     assert np.allclose(Y, deq(A) @ deq(W).T, rtol=1e-14, atol=1e-14)
+
+
+def test_bf16_tolerance_metric():
+    # The bf16 half-ulp used by the GEMM check: 257 rounds to 256 (tie to
+    # even) -- a 1/257 relative error that is all output rounding.
+    from tests import parity
+    import torch
+    x = np.array([257.0, 1.0, 3.0, -1000.5, 1e-30])
+    hu = parity.half_ulp_bf16(x)
+    rounded = torch.tensor(x).to(torch.bfloat16).double().numpy()
+    assert np.all(np.abs(rounded - x) <= hu)
+    assert parity.gemm_rel_error(np.array([256.0]), np.array([257.0])) == 0.0
+    assert parity.gemm_rel_error(np.array([254.0]), np.array([257.0])) > 0.0

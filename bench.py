@@ -76,7 +76,7 @@ def gemm_roofline_s(M, N, counts, pk):
 class ClockSampler:
     """NVML samples of SM clock and throttle reasons while running."""
 
-    def __init__(self, index, period=0.02):
+    def __init__(self, index, period=0.005):
         self.index, self.period = index, period
         self.samples, self.reasons = [], set()
         self.max_mhz = None
@@ -426,7 +426,7 @@ def cpu_baseline():
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")

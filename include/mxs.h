@@ -19,8 +19,9 @@
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default).
  *     Device work is stream-ordered and asynchronous; arguments are checked
  *     on the host before any launch and a non-MXS_OK status means nothing was
- *     launched.  mxs_allocate is the one call that synchronises the stream
- *     (it returns host-side counts).
+ *     launched.  mxs_allocate synchronises the stream in one case only:
+ *     budget mode over more than one layer, where the greedy needs the
+ *     device-computed group gains on the host.
  *   - Device-side failures (a bounded wait that expired) are recorded in a
  *     per-device status word and returned by mxs_sync.
  *   - Calls are thread-safe apart from that shared status word.
@@ -175,7 +176,9 @@ mxs_status mxs_sensitivity(const void *X, mxs_dtype xt, int64_t T, int64_t K, in
  *   8-bit columns, then 6-bit, then 4-bit, ascending within each);
  *   counts (host, 3*n_layers: n8, n6, n4 per layer).
  *   ws (device): mxs_allocate_workspace_bytes(n_layers, K).
- * Synchronises `stream`.  MXS_ERR_BUDGET if infeasible. */
+ * The counts depend only on K, N and the policy except in multi-layer budget
+ * mode, which synchronises `stream` to read the group gains; otherwise the
+ * call is asynchronous.  MXS_ERR_BUDGET if infeasible. */
 mxs_status mxs_allocate_workspace_bytes(int32_t n_layers, const int64_t *K, size_t *bytes);
 mxs_status mxs_allocate(int32_t n_layers, const int64_t *K, const int64_t *N,
                         const double *const *s, const double *layer_w,

@@ -239,7 +239,7 @@ def mxs_allocate(s_list: Sequence[torch.Tensor], N_list: Sequence[int], *, mode:
                  p8=(5, 100), p6=(15, 100), fixed8: int = 32, layer_w=None, stream=None,
                  perms: Optional[List[torch.Tensor]] = None, workspace: Optional[torch.Tensor] = None):
     """Returns (perms: list of device int32 tensors, counts: list of (n8, n6, n4)).
-    Synchronises the stream (the counts come back to the host)."""
+    Synchronises the stream only in multi-layer budget mode."""
     L = len(s_list)
     dev = s_list[0].device
     K = (ctypes.c_int64 * L)(*[int(s.numel()) for s in s_list])

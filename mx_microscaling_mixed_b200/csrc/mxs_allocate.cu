@@ -13,12 +13,14 @@
 // gain/cost across layers (gain = layer weight x summed s, cost = 2 N count
 // bits), stopping at the first group that does not fit.
 //
-// Device work: an all-pairs rank count (each thread ranks one column against
-// every other, staged through shared memory -- exact and order-free), the
-// group gains (one thread sums one group in rank order), and a single-CTA
-// stable compaction that writes the permutation segment by segment in
-// ascending column order.  The integer budget arithmetic and the cross-layer
-// greedy are a few hundred scalar steps and run on the host side of the call.
+// Device work: an all-pairs rank count (a 2-D grid: each CTA ranks 256
+// columns against a tile of 1024 candidates staged in shared memory and adds
+// its counts atomically -- exact and order-free), the group gains (one thread
+// sums one group in rank order), and a single-CTA stable compaction that
+// writes the permutation segment by segment in ascending column order.  The
+// integer budget arithmetic and the cross-layer greedy are a few hundred
+// scalar steps and run on the host side of the call; only the multi-layer
+// greedy needs device data (the group gains) and so a stream synchronisation.
 #include <algorithm>
 #include <vector>
 
@@ -27,31 +29,31 @@
 namespace mxs {
 
 constexpr int kRankThreads = 256;
-constexpr int kRankTile = 2048;
+constexpr int kRankTile = 1024;
 
-__global__ void __launch_bounds__(kRankThreads) rank_kernel(const double *s, int64_t K, int32_t *rank,
-                                                            int32_t *order) {
+// rank[j] += #{i in this CTA's tile : s_i > s_j, or s_i == s_j and i < j}.
+// Grid: (column blocks of 256) x (tiles of 1024 candidates); rank starts at 0.
+__global__ void __launch_bounds__(kRankThreads) rank_kernel(const double *s, int64_t K, int32_t *rank) {
   __shared__ double tile[kRankTile];
   const int64_t j = static_cast<int64_t>(blockIdx.x) * kRankThreads + threadIdx.x;
-  const double sj = j < K ? s[j] : 0.0;
-  int64_t r = 0;
-  for (int64_t base = 0; base < K; base += kRankTile) {
-    const int64_t n = min(static_cast<int64_t>(kRankTile), K - base);
-    __syncthreads();
-    for (int64_t i = threadIdx.x; i < n; i += kRankThreads) tile[i] = s[base + i];
-    __syncthreads();
-    if (j < K) {
-      for (int64_t i = 0; i < n; ++i) {
-        const double si = tile[i];
-        const int64_t gi = base + i;
-        r += (si > sj) || (si == sj && gi < j);
-      }
-    }
+  const int64_t base = static_cast<int64_t>(blockIdx.y) * kRankTile;
+  const int n = static_cast<int>(min(static_cast<int64_t>(kRankTile), K - base));
+  for (int i = threadIdx.x; i < n; i += kRankThreads) tile[i] = s[base + i];
+  __syncthreads();
+  if (j >= K) return;
+  const double sj = s[j];
+  int r = 0;
+  const int64_t jl = j - base;     // ties count for candidates with local index < jl
+  for (int i = 0; i < n; ++i) {
+    const double si = tile[i];
+    r += (si > sj) | ((si == sj) & (i < jl));
   }
-  if (j < K) {
-    rank[j] = static_cast<int32_t>(r);
-    order[r] = static_cast<int32_t>(j);
-  }
+  if (r) atomicAdd(rank + j, r);
+}
+
+__global__ void order_kernel(const int32_t *rank, int64_t K, int32_t *order) {
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (j < K) order[rank[j]] = static_cast<int32_t>(j);
 }
 
 // gains[g] = sum of s over ranks [n8 + 32 g, min(n8 + 32 g + 32, K)), in rank order.
@@ -167,9 +169,11 @@ extern "C" mxs_status mxs_allocate(int32_t n_layers, const int64_t *K, const int
     L[l].order = reinterpret_cast<int32_t *>(p + round_up(K[l] * 4, 256));
     L[l].gains = reinterpret_cast<double *>(p + 2 * round_up(K[l] * 4, 256));
     p += layer_ws_bytes(K[l]);
-    rank_kernel<<<static_cast<unsigned>((K[l] + kRankThreads - 1) / kRankThreads), kRankThreads, 0, cs>>>(
-        s[l], K[l], L[l].rank, L[l].order);
-    count_launch();
+    if (cudaMemsetAsync(L[l].rank, 0, static_cast<size_t>(K[l]) * 4, cs) != cudaSuccess) return MXS_ERR_CUDA;
+    const dim3 rgrid(static_cast<unsigned>((K[l] + kRankThreads - 1) / kRankThreads),
+                     static_cast<unsigned>((K[l] + kRankTile - 1) / kRankTile));
+    rank_kernel<<<rgrid, kRankThreads, 0, cs>>>(s[l], K[l], L[l].rank);
+    count_launch(2);
   }
 
   std::vector<int64_t> n8(n_layers, 0), n6(n_layers, 0);
@@ -192,6 +196,8 @@ extern "C" mxs_status mxs_allocate(int32_t n_layers, const int64_t *K, const int
         const int64_t ng = (K[l] - n8[l] + 31) / 32;
         gains[l].assign(static_cast<size_t>(std::max<int64_t>(ng, 1)), 0.0);
         if (ng > 0) {
+          order_kernel<<<static_cast<unsigned>((K[l] + 255) / 256), 256, 0, cs>>>(L[l].rank, K[l], L[l].order);
+          count_launch();
           group_gain_kernel<<<static_cast<unsigned>((ng + 127) / 128), 128, 0, cs>>>(s[l], L[l].order, K[l],
                                                                                     n8[l], ng, L[l].gains);
           count_launch();
@@ -235,6 +241,5 @@ extern "C" mxs_status mxs_allocate(int32_t n_layers, const int64_t *K, const int
     counts[3 * l + 1] = n6[l];
     counts[3 * l + 2] = K[l] - n8[l] - n6[l];
   }
-  if (cudaGetLastError() != cudaSuccess) return MXS_ERR_CUDA;
-  return cuda_status(cudaStreamSynchronize(cs));
+  return cuda_status(cudaGetLastError());
 }

@@ -272,7 +272,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int it = 0; it < n_iters; ++it) {
         const int s = it % kStages;
         if (!wait_bounded(&full[s], (it / kStages) & 1, abort_flag)) break;
-        ptx::tc_fence_after();
         const uint32_t a_base = ptx::smem_addr(smem + GemmSmem::a_off + s * kABytes);
         const uint32_t b_base = ptx::smem_addr(smem + GemmSmem::b_off + s * kBBytes);
         if (it < g.n16_stages) {
@@ -339,6 +338,297 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ------------------------------------------------- 2-CTA persistent kernel
+//
+// A cluster of two CTAs computes 256 x 256 output tiles with cta_group::2
+// MMAs: each CTA stages its own 128 rows of A and its own 128 rows (half of
+// N) of B, the leader issues M=256, N=256 MMAs that read both CTAs' shared
+// memory and write each CTA's 128-row half of the accumulator into that
+// CTA's tensor memory.  Per pair this halves the B tile traffic of the
+// 1-CTA kernel.  Both CTAs' TMA copies complete on the leader's "full"
+// barriers; the MMA commits arrive on both CTAs' "empty" barriers.  The
+// 4-bit segment's scales: each CTA holds its own 128 A-row chunk and the
+// full 256 N-row pair of chunks (the MMA needs all N scales in each CTA).
+// CTAs are persistent: pair p takes tiles p, p + pairs, ...; eight epilogue
+// warps per CTA drain the accumulator into registers, release it to the
+// leader (one arrival per warp per CTA) and store bf16 while the next tile's
+// MMAs already run.
+
+namespace ptx {
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map, uint32_t leader_bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc2(uint32_t *slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot)), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish2() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void mma2_bf16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma2_mxf8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc,
+                                          uint32_t sfa, uint32_t sfb) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+__device__ __forceinline__ void mma2_commit_both(uint64_t *bar) {
+  asm volatile(
+      "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
+          smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void copy_sf_to_tmem2(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+}  // namespace ptx
+
+constexpr int kP2Stages = 6;
+constexpr int kP2Rows = 128;                       // rows of A and of B per CTA per stage
+constexpr int kP2TileBytes = kP2Rows * kSliceBytes;
+constexpr int kP2SfaBytes = kSfChunk;              // own 128 A rows x 4 blocks
+constexpr int kP2SfbBytes = 2 * kSfChunk;          // the pair's 256 N rows x 4 blocks
+constexpr int kP2EpiWarps = 8;
+constexpr int kP2Threads = (2 + kP2EpiWarps) * 32;
+// cta_group::2, M = 256, N = 256
+constexpr uint32_t kIdesc2Bf16 = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(256 >> 3) << 17) |
+                                 (static_cast<uint32_t>(256 >> 4) << 24);
+constexpr uint32_t kIdesc2Mxf8 = (static_cast<uint32_t>(256 >> 3) << 17) | (1u << 23) |
+                                 (static_cast<uint32_t>(256 >> 4) << 24);
+
+struct P2Smem {
+  static constexpr int a_off = 0;
+  static constexpr int b_off = a_off + kP2Stages * kP2TileBytes;
+  static constexpr int sfa_off = b_off + kP2Stages * kP2TileBytes;
+  static constexpr int sfb_off = sfa_off + kP2Stages * kP2SfaBytes;
+  static constexpr int bar_off = sfb_off + kP2Stages * kP2SfbBytes;
+  // full[S], empty[S], acc_full, acc_empty, tmem slot, abort flag
+  static constexpr int bytes = bar_off + (2 * kP2Stages + 2) * 8 + 16;
+};
+constexpr int kP2SmemBytes = P2Smem::bytes + 1024;
+
+struct P2Args {
+  int32_t M, N;
+  int32_t n16_stages, n8_stages;
+  int32_t m_tiles, n_tiles;
+  int32_t nrg_a, nrg_b;
+  __nv_bfloat16 *Y;
+  int64_t ldy;
+  int32_t y_vec;
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA16, const __grid_constant__ CUtensorMap tmB16,
+                    const __grid_constant__ CUtensorMap tmA8, const __grid_constant__ CUtensorMap tmB8,
+                    const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB, P2Args g) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + P2Smem::bar_off);
+  uint64_t *empty = full + kP2Stages;
+  uint64_t *acc_full = empty + kP2Stages;
+  uint64_t *acc_empty = acc_full + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int n_iters = g.n16_stages + g.n8_stages;
+  const int n_tiles_total = g.m_tiles * g.n_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kP2Stages; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    ptx::mbar_init(acc_full, 1);
+    ptx::mbar_init(acc_empty, 2 * kP2EpiWarps);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc2(tmem_slot, kTmemCols);
+    ptx::tmem_relinquish2();
+  }
+  ptx::tc_fence_before();
+  ptx::cluster_sync();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint32_t bytes16 = 2 * (2 * kP2TileBytes);
+      const uint32_t bytes8 = 2 * (2 * kP2TileBytes + kP2SfaBytes + kP2SfbBytes);
+      int it = 0;
+      for (int t = pair; t < n_tiles_total && !*abort_flag; t += npairs) {
+        const int mt = t / g.n_tiles, nt = t - mt * g.n_tiles;
+        const int am = mt * 256 + static_cast<int>(rank) * kP2Rows;      // this CTA's A rows
+        const int bn = nt * 256 + static_cast<int>(rank) * kP2Rows;      // this CTA's B rows
+        for (int k = 0; k < n_iters; ++k, ++it) {
+          const int s = it % kP2Stages;
+          if (it >= kP2Stages && !wait_bounded(&empty[s], ((it / kP2Stages) - 1) & 1, abort_flag)) break;
+          const uint32_t lbar = ptx::map_to_rank(ptx::smem_addr(&full[s]), 0);
+          uint8_t *sa = smem + P2Smem::a_off + s * kP2TileBytes;
+          uint8_t *sb = smem + P2Smem::b_off + s * kP2TileBytes;
+          if (k < g.n16_stages) {
+            if (leader) ptx::mbar_arrive_expect_tx(&full[s], bytes16);
+            ptx::tma_load_2d_pair(sa, &tmA16, lbar, k * 64, am);
+            ptx::tma_load_2d_pair(sb, &tmB16, lbar, k * 64, bn);
+          } else {
+            const int j = k - g.n16_stages;
+            if (leader) ptx::mbar_arrive_expect_tx(&full[s], bytes8);
+            ptx::tma_load_2d_pair(sa, &tmA8, lbar, j * 128, am);
+            ptx::tma_load_2d_pair(sb, &tmB8, lbar, j * 128, bn);
+            ptx::tma_load_2d_pair(smem + P2Smem::sfa_off + s * kP2SfaBytes, &tmSFA, lbar, 0,
+                                  4 * (j * g.nrg_a + am / 128));
+            ptx::tma_load_2d_pair(smem + P2Smem::sfb_off + s * kP2SfbBytes, &tmSFB, lbar, 0,
+                                  4 * (j * g.nrg_b + nt * 2));
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (leader && lane == 0) {
+      const uint32_t tsfa = tmem + kSfaCol, tsfb = tmem + kSfbCol;
+      int it = 0, tl = 0;
+      for (int t = pair; t < n_tiles_total && !*abort_flag; t += npairs, ++tl) {
+        if (tl > 0 && !wait_bounded(acc_empty, (tl - 1) & 1, abort_flag)) break;
+        ptx::tc_fence_after();
+        bool ok = true;
+        for (int k = 0; k < n_iters; ++k, ++it) {
+          const int s = it % kP2Stages;
+          if (!wait_bounded(&full[s], (it / kP2Stages) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t a_base = ptx::smem_addr(smem + P2Smem::a_off + s * kP2TileBytes);
+          const uint32_t b_base = ptx::smem_addr(smem + P2Smem::b_off + s * kP2TileBytes);
+          if (k < g.n16_stages) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              ptx::mma2_bf16(tmem, ptx::desc_sw128(a_base + 32 * q), ptx::desc_sw128(b_base + 32 * q), kIdesc2Bf16,
+                             (k > 0 || q > 0) ? 1u : 0u);
+          } else {
+            const uint32_t sfa_s = ptx::smem_addr(smem + P2Smem::sfa_off + s * kP2SfaBytes);
+            const uint32_t sfb_s = ptx::smem_addr(smem + P2Smem::sfb_off + s * kP2SfbBytes);
+            ptx::copy_sf_to_tmem2(tsfa, ptx::desc_sf(sfa_s));
+            ptx::copy_sf_to_tmem2(tsfb, ptx::desc_sf(sfb_s));
+            ptx::copy_sf_to_tmem2(tsfb + 4, ptx::desc_sf(sfb_s + kSfChunk));
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t idesc = kIdesc2Mxf8 | (static_cast<uint32_t>(q) << 4) | (static_cast<uint32_t>(q) << 29);
+              ptx::mma2_mxf8(tmem, ptx::desc_sw128(a_base + 32 * q), ptx::desc_sw128(b_base + 32 * q), idesc,
+                             (k > 0 || q > 0) ? 1u : 0u, tsfa | (static_cast<uint32_t>(q) << 30),
+                             tsfb | (static_cast<uint32_t>(q) << 30));
+            }
+          }
+          ptx::mma2_commit_both(&empty[s]);
+        }
+        if (!ok) break;
+        ptx::mma2_commit_both(acc_full);
+      }
+    }
+  } else {
+    // epilogue: warp w reads lanes 32*(w%4)..+31, columns 128*h..128*h+127
+    const int q = warp & 3, h = (warp - 2) >> 2;
+    const uint32_t acc_empty_leader = ptx::map_to_rank(ptx::smem_addr(acc_empty), 0);
+    int tl = 0;
+    for (int t = pair; t < n_tiles_total; t += npairs, ++tl) {
+      if (!wait_bounded(acc_full, tl & 1, abort_flag)) break;
+      ptx::tc_fence_after();
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        ptx::tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + 128 * h + 32 * c, r[c]);
+      ptx::tmem_wait_ld();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_cluster(acc_empty_leader);
+      const int mt = t / g.n_tiles, nt = t - mt * g.n_tiles;
+      const int row = mt * 256 + static_cast<int>(rank) * kP2Rows + q * 32 + lane;
+      if (row < g.M) {
+        __nv_bfloat16 *yrow = g.Y + static_cast<int64_t>(row) * g.ldy;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int n = nt * 256 + 128 * h + 32 * c + 8 * v;
+            if (g.y_vec && n + 8 <= g.N) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[c][8 * v + 2 * i]),
+                                                          __uint_as_float(r[c][8 * v + 2 * i + 1]));
+                pk[i] = *reinterpret_cast<uint32_t *>(&b2);
+              }
+              *reinterpret_cast<uint4 *>(yrow + n) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                if (n + i < g.N) yrow[n + i] = __float2bfloat16_rn(__uint_as_float(r[c][8 * v + i]));
+            }
+          }
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc2(tmem, kTmemCols);
+  }
+}
+
 // ---------------------------------------------------------------- staging
 
 struct StageOperand {
@@ -360,79 +650,433 @@ struct StageArgs {
   int64_t k16, k4;
   int64_t k6_off16;     // start of the 6-bit segment inside x16 rows
   int32_t nkg;          // k-groups of 4 blocks in the 4-bit segment
-  int64_t n_decode[2];  // rows * nb_total per operand
-  int64_t n_pad[2];     // scale-chunk entries per operand (all, incl. padding)
 };
 
 __device__ __forceinline__ int64_t sf_index(int64_t r, int64_t b, int32_t nrg) {
   return ((b >> 2) * nrg + (r >> 7)) * kSfChunk + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (b & 3);
 }
 
-__device__ __forceinline__ int unpack_code(const uint8_t *c, int t, int m) {
-  if (m == 8) return static_cast<int8_t>(c[t]);
-  if (m == 4) {
-    const int v = (c[t >> 1] >> (4 * (t & 1))) & 0xF;
-    return v >= 8 ? v - 16 : v;
-  }
-  const int grp = t >> 2, sub = t & 3;
-  const uint32_t w = c[3 * grp] | (c[3 * grp + 1] << 8) | (c[3 * grp + 2] << 16);
-  const int v = (w >> (6 * sub)) & 0x3F;
-  return v >= 32 ? v - 64 : v;
+// Code value of an m-bit two's complement field, as an exact float:
+// the integer rides in the mantissa of 1.5*2^23 and is taken back out by a
+// subtraction.
+__device__ __forceinline__ float code_to_float(int q) {
+  return __uint_as_float(static_cast<uint32_t>(0x4B400000 + q)) - 12582912.0f;
 }
 
-__global__ void __launch_bounds__(256) gemm_stage_kernel(StageArgs a) {
-  const int64_t total = a.n_decode[0] + a.n_decode[1] + a.n_pad[0] + a.n_pad[1];
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    int64_t w = i;
-    if (w < a.n_decode[0] + a.n_decode[1]) {
-      const int o = w < a.n_decode[0] ? 0 : 1;
-      if (o) w -= a.n_decode[0];
-      const StageOperand &op = a.op[o];
-      const int64_t row = w / a.nb_total;
-      int blk = static_cast<int>(w - row * a.nb_total);
-      int g = 0;
-      while (blk >= a.nb[g]) { blk -= a.nb[g]; ++g; }
-      const int m = seg_bits(g);
-      const uint8_t *c = op.codes[g] + row * op.cpitch[g] + static_cast<int64_t>(blk) * kBlock * m / 8;
-      const uint8_t sbyte = op.scales[g][row * op.spitch[g] + blk];
-      if (g == 2) {
-        __align__(16) uint8_t out[kBlock];
+// 6/8-bit block -> 32 exact bf16 values q * 2^(e-m+2), four 16-byte stores.
+template <int M>
+__device__ __forceinline__ void stage_wide_block(const uint8_t *c, uint8_t sbyte, __nv_bfloat16 *dst) {
+  const float step = pow2f(static_cast<int>(sbyte) - 127 - M + 2);
+  int q[kBlock];
+  if constexpr (M == 8) {
+    const uint4 a = *reinterpret_cast<const uint4 *>(c), b = *reinterpret_cast<const uint4 *>(c + 16);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int t = 0; t < kBlock; t += 2) {
-          const float2 f = make_float2(0.25f * static_cast<float>(unpack_code(c, t, 4)),
-                                       0.25f * static_cast<float>(unpack_code(c, t + 1, 4)));
-          const __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
-          out[t] = static_cast<uint8_t>(p & 0xFF);
-          out[t + 1] = static_cast<uint8_t>(p >> 8);
+    for (int t = 0; t < kBlock; ++t) q[t] = static_cast<int>(static_cast<int8_t>((w[t >> 2] >> (8 * (t & 3))) & 0xFF));
+  } else {
+    const uint2 a = *reinterpret_cast<const uint2 *>(c), b = *reinterpret_cast<const uint2 *>(c + 8),
+                d = *reinterpret_cast<const uint2 *>(c + 16);
+    const uint32_t w[6] = {a.x, a.y, b.x, b.y, d.x, d.y};
+#pragma unroll
+    for (int t = 0; t < kBlock; ++t) {
+      const int pos = 6 * t, word = pos >> 5, off = pos & 31;
+      uint32_t f = w[word] >> off;
+      if (off > 26) f |= w[word + 1] << (32 - off);
+      q[t] = static_cast<int>(f << 26) >> 26;    // sign-extend the 6-bit field
+    }
+  }
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(code_to_float(q[2 * i]) * step, code_to_float(q[2 * i + 1]) * step);
+    pk[i] = *reinterpret_cast<uint32_t *>(&h);
+  }
+  uint4 *o = reinterpret_cast<uint4 *>(dst);
+  o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  o[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+  o[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+}
+
+// Tiles of 128 rows x 32 blocks of one segment of one operand; a CTA takes
+// tiles in a grid-stride loop.  Each warp walks 16 rows of the tile with its
+// lanes on 32 consecutive blocks, so code loads (16/24/32 bytes per lane) and
+// the converted stores (32 or 64 bytes per lane) are contiguous across the
+// warp.  For the 4-bit segment the tile's E8M0 bytes are placed in shared
+// memory in the tensor core's 512-byte chunk layout (128 rows x 4 blocks per
+// chunk; 2^0 where the tile runs past the real rows or blocks) and written
+// out as whole chunks.
+constexpr int kStageRows = 128;
+constexpr int kStageBlocks = 32;
+
+__global__ void __launch_bounds__(256) gemm_stage_kernel(StageArgs a) {
+  __shared__ uint16_t lut[256];                        // byte of two 4-bit codes -> their E4M3 pair (q/4)
+  __shared__ __align__(16) uint8_t sf_tile[kStageBlocks / 4][kSfChunk];
+  {
+    const int b = threadIdx.x;
+    const int lo = (b & 0xF) >= 8 ? (b & 0xF) - 16 : (b & 0xF);
+    const int hi = (b >> 4) >= 8 ? (b >> 4) - 16 : (b >> 4);
+    lut[b] = static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(make_float2(0.25f * lo, 0.25f * hi), __NV_SATFINITE, __NV_E4M3));
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // tile counts per (operand, segment)
+  int ntile[2][3];
+  int total = 0;
+  for (int o = 0; o < 2; ++o)
+    for (int g = 0; g < 3; ++g) {
+      const int rt = static_cast<int>((a.op[o].rows + kStageRows - 1) / kStageRows);
+      const int bt = (a.nb[g] + kStageBlocks - 1) / kStageBlocks;
+      ntile[o][g] = g == 2 ? static_cast<int>(a.op[o].nrg) * ((a.nkg * 4 + kStageBlocks - 1) / kStageBlocks) : rt * bt;
+      if (a.nb[g] == 0) ntile[o][g] = 0;
+      total += ntile[o][g];
+    }
+  __syncthreads();
+  for (int t = blockIdx.x; t < total; t += gridDim.x) {
+    int o = 0, g = 0, w = t;
+    while (w >= ntile[o][g]) {
+      w -= ntile[o][g];
+      if (++g == 3) { g = 0; ++o; }
+    }
+    const StageOperand &op = a.op[o];
+    const int m = seg_bits(g);
+    if (g == 2) {
+      // 4-bit: tiles cover the chunk grid (row groups x groups of 8 k-groups)
+      const int kg_tiles = (a.nkg * 4 + kStageBlocks - 1) / kStageBlocks;
+      const int rt = w / kg_tiles, bt = w - rt * kg_tiles;
+      const int r0 = rt * kStageRows, b0 = bt * kStageBlocks;
+      for (int i = threadIdx.x; i < (kStageBlocks / 4) * kSfChunk / 16; i += blockDim.x)
+        reinterpret_cast<uint4 *>(&sf_tile[0][0])[i] = make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+      __syncthreads();
+      const int blk = b0 + lane;
+      for (int rr = warp; rr < kStageRows; rr += 8) {
+        const int64_t row = r0 + rr;
+        if (row >= op.rows || blk >= a.nb[2]) continue;
+        const uint4 v = *reinterpret_cast<const uint4 *>(op.codes[2] + row * op.cpitch[2] + static_cast<int64_t>(blk) * 16);
+        const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+        uint32_t out[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t x = in[j];
+          out[2 * j] = static_cast<uint32_t>(lut[x & 0xFF]) | (static_cast<uint32_t>(lut[(x >> 8) & 0xFF]) << 16);
+          out[2 * j + 1] = static_cast<uint32_t>(lut[(x >> 16) & 0xFF]) | (static_cast<uint32_t>(lut[x >> 24]) << 16);
         }
         uint4 *dst = reinterpret_cast<uint4 *>(op.x8 + row * a.k4 + static_cast<int64_t>(blk) * kBlock);
-        dst[0] = *reinterpret_cast<uint4 *>(out);
-        dst[1] = *reinterpret_cast<uint4 *>(out + 16);
-        op.sf[sf_index(row, blk, op.nrg)] = sbyte;
-      } else {
-        const float step = pow2f(static_cast<int>(sbyte) - 127 - m + 2);
-        __align__(16) __nv_bfloat16 out[kBlock];
-#pragma unroll
-        for (int t = 0; t < kBlock; ++t) out[t] = __float2bfloat16_rn(static_cast<float>(unpack_code(c, t, m)) * step);
-        const int64_t col = (g == 0 ? 0 : a.k6_off16) + static_cast<int64_t>(blk) * kBlock;
-        uint4 *dst = reinterpret_cast<uint4 *>(op.x16 + row * a.k16 + col);
-        const uint4 *src = reinterpret_cast<const uint4 *>(out);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) dst[v] = src[v];
+        dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+        dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+        sf_tile[lane >> 2][(rr & 31) * 16 + ((rr >> 5) & 3) * 4 + (lane & 3)] = op.scales[2][row * op.spitch[2] + blk];
       }
+      __syncthreads();
+      // whole chunks out: chunk (k-group b0/4 + c, row group rt)
+      const int nchunks = min(kStageBlocks / 4, a.nkg - b0 / 4);
+      for (int i = threadIdx.x; i < nchunks * kSfChunk / 16; i += blockDim.x) {
+        const int c = i / (kSfChunk / 16), e = i - c * (kSfChunk / 16);
+        uint4 *dst = reinterpret_cast<uint4 *>(op.sf + (static_cast<int64_t>(b0 / 4 + c) * op.nrg + rt) * kSfChunk);
+        dst[e] = reinterpret_cast<const uint4 *>(&sf_tile[c][0])[e];
+      }
+      __syncthreads();
     } else {
-      // neutral scale (2^0) for chunk entries outside the real rows / blocks
-      w -= a.n_decode[0] + a.n_decode[1];
-      const int o = w < a.n_pad[0] ? 0 : 1;
-      if (o) w -= a.n_pad[0];
-      const StageOperand &op = a.op[o];
-      const int64_t nbp = static_cast<int64_t>(a.nkg) * 4;
-      const int64_t row = w / nbp, blk = w - row * nbp;
-      if (row >= op.rows || blk >= a.nb[2]) op.sf[sf_index(row, blk, op.nrg)] = 127;
+      const int bt_n = (a.nb[g] + kStageBlocks - 1) / kStageBlocks;
+      const int rt = w / bt_n, bt = w - rt * bt_n;
+      const int blk = bt * kStageBlocks + lane;
+      if (blk >= a.nb[g]) continue;
+      const int64_t col = (g == 0 ? 0 : a.k6_off16) + static_cast<int64_t>(blk) * kBlock;
+      for (int rr = warp; rr < kStageRows; rr += 8) {
+        const int64_t row = static_cast<int64_t>(rt) * kStageRows + rr;
+        if (row >= op.rows) break;
+        const uint8_t *c = op.codes[g] + row * op.cpitch[g] + static_cast<int64_t>(blk) * kBlock * m / 8;
+        const uint8_t sbyte = op.scales[g][row * op.spitch[g] + blk];
+        if (g == 0) stage_wide_block<8>(c, sbyte, op.x16 + row * a.k16 + col);
+        else stage_wide_block<6>(c, sbyte, op.x16 + row * a.k16 + col);
+      }
     }
   }
 }
+
+// ------------------------------------------------------ small-M decode path
+//
+// For a handful of activation rows the GEMM is bound by the bytes of W, so
+// W is read packed, straight from HBM, and never staged.  Within one
+// 32-position block both operands share one E8M0 scale each, so the block's
+// contribution is an integer dot product times an exact power of two:
+//   sum_t qa_t qw_t * 2^(ea - m + 2) * 2^(ew - m + 2).
+// The integer part runs on dp4a (4 byte products per instruction) with the W
+// codes in offset binary (qw + 2^(m-1), one XOR per word), the offset taken
+// back out with the A block's code sum; |sum| < 2^22, so the integer converts
+// exactly and the scaling is exact; only the fp32 accumulation over blocks
+// (and the final bf16 rounding) rounds.
+// Each CTA stages the activations of one K chunk in shared memory as signed
+// bytes in the order that matches the W unpacking, then each warp runs a
+// group of R W rows: lane l takes blocks l, l+32, ... (U of them with their
+// loads in flight together) and a butterfly
+// over the warp sums the lanes.
+
+struct SmallArgs {
+  int32_t M, N;
+  int32_t nb[3];
+  int32_t nb_total;
+  int32_t chunk_blocks;              // blocks staged per K chunk
+  const uint8_t *a_codes[3];
+  int64_t a_cpitch[3];
+  const uint8_t *a_scales[3];
+  int64_t a_spitch[3];
+  const uint8_t *w_codes[3];
+  int64_t w_cpitch[3];
+  const uint8_t *w_scales[3];
+  int64_t w_spitch[3];
+  __nv_bfloat16 *Y;
+  int64_t ldy;
+};
+
+__device__ __forceinline__ int dp4a_us(uint32_t u, uint32_t s, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(u), "r"(s), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ void small_locate(const SmallArgs &a, int gb, int &g, int &b) {
+  if (gb < a.nb[0]) { g = 0; b = gb; }
+  else if (gb < a.nb[0] + a.nb[1]) { g = 1; b = gb - a.nb[0]; }
+  else { g = 2; b = gb - a.nb[0] - a.nb[1]; }
+}
+
+// Raw packed words of one W block (4-bit: 4 words, 6-bit: 6, 8-bit: 8).
+__device__ __forceinline__ void load_w_raw(const uint8_t *c, int g, uint32_t (&w)[8]) {
+  if (g == 2) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(c));
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else if (g == 1) {
+    const uint2 x0 = __ldg(reinterpret_cast<const uint2 *>(c)), x1 = __ldg(reinterpret_cast<const uint2 *>(c + 8)),
+                x2 = __ldg(reinterpret_cast<const uint2 *>(c + 16));
+    w[0] = x0.x; w[1] = x0.y; w[2] = x1.x; w[3] = x1.y; w[4] = x2.x; w[5] = x2.y;
+  } else {
+    const uint4 v0 = __ldg(reinterpret_cast<const uint4 *>(c)), v1 = __ldg(reinterpret_cast<const uint4 *>(c + 16));
+    w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w; w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+  }
+}
+
+// 32 codes of one block as the 8 words the dp4a loop consumes, W side in
+// offset binary (code + 2^(m-1), unsigned bytes):
+// 4-bit: word 2j = codes 8j, 8j+2, 8j+4, 8j+6, word 2j+1 = the odd ones;
+// 6-bit and 8-bit: word j = codes 4j..4j+3.
+__device__ __forceinline__ void unpack_w(const uint32_t (&w)[8], int g, uint32_t (&u)[8]) {
+  if (g == 2) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      u[2 * j] = (w[j] & 0x0F0F0F0Fu) ^ 0x08080808u;
+      u[2 * j + 1] = ((w[j] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+    }
+  } else if (g == 1) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int pos = 24 * j, word = pos >> 5, off = pos & 31;
+      uint32_t v = w[word] >> off;
+      if (off > 8) v |= w[word + 1] << (32 - off);
+      const uint32_t spread = (v & 0x3Fu) | ((v << 2) & 0x3F00u) | ((v << 4) & 0x3F0000u) | ((v << 6) & 0x3F000000u);
+      u[j] = spread ^ 0x20202020u;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) u[j] = w[j] ^ 0x80808080u;
+  }
+}
+
+// Activation side: signed bytes in the same word order, the code sum (to
+// remove the W offset) and the block's scale 2^(e-m+2).
+__device__ __forceinline__ void stage_a_block(const uint8_t *c, int g, uint32_t (&wd)[8], int &sum) {
+  sum = 0;
+  if (g == 2) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t ev = 0, od = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int qe = static_cast<int>(w[j] << (28 - 8 * i)) >> 28;       // nibble 2i
+        const int qo = static_cast<int>(w[j] << (24 - 8 * i)) >> 28;       // nibble 2i+1
+        sum += qe + qo;
+        ev |= (static_cast<uint32_t>(qe) & 0xFFu) << (8 * i);
+        od |= (static_cast<uint32_t>(qo) & 0xFFu) << (8 * i);
+      }
+      wd[2 * j] = ev;
+      wd[2 * j + 1] = od;
+    }
+  } else if (g == 1) {
+    const uint2 x0 = *reinterpret_cast<const uint2 *>(c), x1 = *reinterpret_cast<const uint2 *>(c + 8),
+                x2 = *reinterpret_cast<const uint2 *>(c + 16);
+    const uint32_t w[6] = {x0.x, x0.y, x1.x, x1.y, x2.x, x2.y};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      uint32_t o = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int pos = 6 * (4 * j + i), word = pos >> 5, off = pos & 31;
+        uint32_t f = w[word] >> off;
+        if (off > 26) f |= w[word + 1] << (32 - off);
+        const int q = static_cast<int>(f << 26) >> 26;
+        sum += q;
+        o |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * i);
+      }
+      wd[j] = o;
+    }
+  } else {
+    const uint4 v0 = *reinterpret_cast<const uint4 *>(c), v1 = *reinterpret_cast<const uint4 *>(c + 16);
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      wd[j] = w[j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sum += static_cast<int>(w[j] << (24 - 8 * i)) >> 24;
+    }
+  }
+}
+
+// MT: activation rows handled (>= M), R: W rows per warp, U: blocks per lane
+// whose loads are issued together, WPC: warps per CTA.
+template <int MT, int R, int U, int WPC>
+__global__ void __launch_bounds__(WPC * 32) gemm_small_kernel(SmallArgs a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int CB = a.chunk_blocks;
+  uint8_t *sa = smem;                                               // [MT][2][CB][16 B]
+  int32_t *scorr = reinterpret_cast<int32_t *>(smem + static_cast<int64_t>(MT) * CB * 32);   // [MT][CB]
+  float *sfa = reinterpret_cast<float *>(scorr + MT * CB);                                     // [MT][CB]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = (blockIdx.x * WPC + warp) * R;
+  float acc[R][MT];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int m = 0; m < MT; ++m) acc[r][m] = 0.f;
+
+  for (int c0 = 0; c0 < a.nb_total; c0 += CB) {
+    const int cb = min(CB, a.nb_total - c0);
+    __syncthreads();
+    for (int it = threadIdx.x; it < a.M * cb; it += blockDim.x) {
+      const int m = it / cb, b = it - m * cb;
+      int g, bb;
+      small_locate(a, c0 + b, g, bb);
+      const int mb = seg_bits(g);
+      uint32_t wd[8];
+      int sum;
+      stage_a_block(a.a_codes[g] + m * a.a_cpitch[g] + static_cast<int64_t>(bb) * kBlock * mb / 8, g, wd, sum);
+      const int e = static_cast<int>(a.a_scales[g][m * a.a_spitch[g] + bb]) - 127;
+      *reinterpret_cast<uint4 *>(sa + ((m * 2 + 0) * CB + b) * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+      *reinterpret_cast<uint4 *>(sa + ((m * 2 + 1) * CB + b) * 16) = make_uint4(wd[4], wd[5], wd[6], wd[7]);
+      scorr[m * CB + b] = -(1 << (mb - 1)) * sum;                  // removes the W offset
+      sfa[m * CB + b] = pow2f(e - mb + 2);
+    }
+    __syncthreads();
+    for (int b0 = lane; b0 < cb; b0 += 32 * U) {
+      uint32_t raw[U][R][8];
+      float fw[U][R];
+      int gs[U];
+      // issue every load of this round before using any of them
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int b = b0 + 32 * u;
+        gs[u] = -1;
+        if (b < cb) {
+          int g, bb;
+          small_locate(a, c0 + b, g, bb);
+          gs[u] = g;
+          const int mb = seg_bits(g);
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            const int n = min(n0 + r, a.N - 1);     // rows past N load row N-1 and are never stored
+            load_w_raw(a.w_codes[g] + static_cast<int64_t>(n) * a.w_cpitch[g] + static_cast<int64_t>(bb) * kBlock * mb / 8,
+                       g, raw[u][r]);
+            fw[u][r] = pow2f(static_cast<int>(__ldg(a.w_scales[g] + static_cast<int64_t>(n) * a.w_spitch[g] + bb)) - 127 - mb + 2);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int g = gs[u];
+        if (g < 0) continue;
+        const int b = b0 + 32 * u;
+        uint32_t uw[R][8];
+#pragma unroll
+        for (int r = 0; r < R; ++r) unpack_w(raw[u][r], g, uw[r]);
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          if (m < a.M) {
+            const uint4 x0 = *reinterpret_cast<const uint4 *>(sa + ((m * 2 + 0) * CB + b) * 16);
+            const uint4 x1 = *reinterpret_cast<const uint4 *>(sa + ((m * 2 + 1) * CB + b) * 16);
+            const uint32_t av[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            const int corr = scorr[m * CB + b];
+            const float fa = sfa[m * CB + b];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+              int d = corr;
+#pragma unroll
+              for (int j = 0; j < 8; ++j) d = dp4a_us(uw[r][j], av[j], d);
+              acc[r][m] = fmaf(code_to_float(d), fw[u][r] * fa, acc[r][m]);
+            }
+          }
+        }
+      }
+    }
+  }
+  // butterfly over the warp, then one lane per (row, activation) stores
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      float v = acc[r][m];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      acc[r][m] = v;
+    }
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+      if (lane == ((r * MT + m) & 31) && m < a.M && n0 + r < a.N)
+        a.Y[static_cast<int64_t>(m) * a.ldy + n0 + r] = __float2bfloat16_rn(acc[r][m]);
+}
+
+template <int MT, int R, int U, int WPC>
+static mxs_status launch_small(const SmallArgs &base, cudaStream_t cs) {
+  SmallArgs a = base;
+  const int per_block_bytes = MT * (32 + 8);
+  // about 40 KB of staged activations per CTA, several CTAs per SM
+  a.chunk_blocks = std::max(32, std::min(a.nb_total, (40 * 1024) / per_block_bytes));
+  const int smem = a.chunk_blocks * per_block_bytes;
+  if (!ensure_smem(gemm_small_kernel<MT, R, U, WPC>, 48 * 1024)) return MXS_ERR_CUDA;
+  const int rows_per_cta = WPC * R;
+  gemm_small_kernel<MT, R, U, WPC><<<(a.N + rows_per_cta - 1) / rows_per_cta, WPC * 32, smem, cs>>>(a);
+  count_launch();
+  return cuda_status(cudaGetLastError());
+}
+
+static mxs_status gemm_small(const mxs_mxtensor *A, const mxs_mxtensor *W, void *Y, int64_t ldy, cudaStream_t cs) {
+  SmallArgs a{};
+  a.M = static_cast<int32_t>(A->rows);
+  a.N = static_cast<int32_t>(W->rows);
+  a.nb_total = 0;
+  for (int g = 0; g < 3; ++g) {
+    a.nb[g] = static_cast<int32_t>(A->lay.seg[g].k_pad / kBlock);
+    a.nb_total += a.nb[g];
+    a.a_codes[g] = A->codes[g];
+    a.a_cpitch[g] = A->code_pitch[g];
+    a.a_scales[g] = A->scales[g];
+    a.a_spitch[g] = A->scale_pitch[g];
+    a.w_codes[g] = W->codes[g];
+    a.w_cpitch[g] = W->code_pitch[g];
+    a.w_scales[g] = W->scales[g];
+    a.w_spitch[g] = W->scale_pitch[g];
+  }
+  a.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
+  a.ldy = ldy;
+  if (a.M <= 1) return launch_small<1, 1, 4, 8>(a, cs);
+  if (a.M <= 2) return launch_small<2, 1, 4, 8>(a, cs);
+  if (a.M <= 4) return launch_small<4, 2, 2, 8>(a, cs);
+  if (a.M <= 8) return launch_small<8, 4, 2, 4>(a, cs);
+  return launch_small<16, 4, 1, 4>(a, cs);
+}
+
+constexpr int64_t kSmallMaxM = 16;
+constexpr int64_t kPairMinM = 512;   // from here the 2-CTA pair kernel
 
 // ---------------------------------------------------------------- host side
 
@@ -497,6 +1141,20 @@ static bool make_map(CUtensorMap *m, CUtensorMapDataType dt, int esize, void *ba
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D byte map with 128-byte rows, no swizzle: the scale-chunk arrays seen as
+// rows of 128 bytes (a 512-byte chunk is 4 rows).
+static bool make_rows_map(CUtensorMap *m, void *base, int64_t total_bytes, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(total_bytes / 128)};
+  const cuuint64_t strides[1] = {128};
+  const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 static bool same_layout(const mxs_layout &a, const mxs_layout &b) {
   if (a.K != b.K || a.K_pad != b.K_pad || a.perm != b.perm) return false;
   for (int g = 0; g < 3; ++g)
@@ -553,6 +1211,7 @@ extern "C" mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, voi
     return cuda_status(cudaMemset2DAsync(Y, static_cast<size_t>(ldy) * 2, 0, static_cast<size_t>(N) * 2,
                                          static_cast<size_t>(M), cs));
   }
+  if (M <= kSmallMaxM) return gemm_small(A, W, Y, ldy, cs);
   const WsPlan p = plan_workspace(A, W);
   if (!ws || ws_bytes < p.total || (reinterpret_cast<uintptr_t>(ws) & 1023u)) return MXS_ERR_WORKSPACE;
   uint8_t *base = reinterpret_cast<uint8_t *>(ws);
@@ -582,15 +1241,16 @@ extern "C" mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, voi
   sa.k4 = p.k4;
   sa.k6_off16 = A->lay.seg[0].k_pad;
   sa.nkg = p.nkg;
-  sa.n_decode[0] = M * sa.nb_total;
-  sa.n_decode[1] = N * sa.nb_total;
-  sa.n_pad[0] = static_cast<int64_t>(p.nrg_a) * 128 * p.nkg * 4;
-  sa.n_pad[1] = static_cast<int64_t>(p.nrg_b) * 128 * p.nkg * 4;
   int dev = 0, nsm = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t total = sa.n_decode[0] + sa.n_decode[1] + sa.n_pad[0] + sa.n_pad[1];
-  const int sgrid = static_cast<int>(std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(nsm) * 16));
+  int64_t stage_tiles = 0;
+  for (int g = 0; g < 3; ++g) {
+    if (sa.nb[g] == 0) continue;
+    const int64_t bt = g == 2 ? (p.nkg * 4 + kStageBlocks - 1) / kStageBlocks : (sa.nb[g] + kStageBlocks - 1) / kStageBlocks;
+    stage_tiles += (g == 2 ? (p.nrg_a + p.nrg_b) : ((M + kStageRows - 1) / kStageRows + (N + kStageRows - 1) / kStageRows)) * bt;
+  }
+  const int sgrid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(stage_tiles, static_cast<int64_t>(nsm) * 8)));
   gemm_stage_kernel<<<sgrid, 256, 0, cs>>>(sa);
   count_launch();
 
@@ -605,25 +1265,54 @@ extern "C" mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, voi
         !make_map(&mB8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + p.off_b8, p.k4, N, kBN))
       return MXS_ERR_CUDA;
   }
+  const int32_t n16_stages = static_cast<int32_t>((p.k16 + 63) / 64);
+  const int32_t n8_stages = static_cast<int32_t>((p.k4 + 127) / 128);
+  const int32_t y_vec = aligned16(Y) && (ldy * 2) % 16 == 0;
+  if (M >= kPairMinM) {
+    CUtensorMap mSFA{}, mSFB{};
+    if (p.k4 > 0) {
+      if (!make_rows_map(&mSFA, base + p.off_sfa, static_cast<int64_t>(p.nkg) * p.nrg_a * kSfChunk, 4) ||
+          !make_rows_map(&mSFB, base + p.off_sfb, static_cast<int64_t>(p.nkg) * p.nrg_b * kSfChunk, 8))
+        return MXS_ERR_CUDA;
+    }
+    if (p.k16 > 0) {   // the pair kernel loads 128-row boxes of B
+      if (!make_map(&mB16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base + p.off_b16, p.k16, N, kP2Rows)) return MXS_ERR_CUDA;
+    }
+    if (p.k4 > 0) {
+      if (!make_map(&mB8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + p.off_b8, p.k4, N, kP2Rows)) return MXS_ERR_CUDA;
+    }
+    P2Args pa{};
+    pa.M = static_cast<int32_t>(M);
+    pa.N = static_cast<int32_t>(N);
+    pa.n16_stages = n16_stages;
+    pa.n8_stages = n8_stages;
+    pa.m_tiles = static_cast<int32_t>((M + 255) / 256);
+    pa.n_tiles = static_cast<int32_t>((N + 255) / 256);
+    pa.nrg_a = p.nrg_a;
+    pa.nrg_b = p.nrg_b;
+    pa.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
+    pa.ldy = ldy;
+    pa.y_vec = y_vec;
+    if (!ensure_smem(gemm_tc2_kernel, kP2SmemBytes)) return MXS_ERR_CUDA;
+    const int tiles = pa.m_tiles * pa.n_tiles;
+    const int pairs = std::max(1, std::min(tiles, nsm / 2));
+    gemm_tc2_kernel<<<2 * pairs, kP2Threads, kP2SmemBytes, cs>>>(mA16, mB16, mA8, mB8, mSFA, mSFB, pa);
+    count_launch();
+    return cuda_status(cudaGetLastError());
+  }
   GemmArgs ga{};
   ga.M = static_cast<int32_t>(M);
   ga.N = static_cast<int32_t>(N);
-  ga.n16_stages = static_cast<int32_t>((p.k16 + 63) / 64);
-  ga.n8_stages = static_cast<int32_t>((p.k4 + 127) / 128);
+  ga.n16_stages = n16_stages;
+  ga.n8_stages = n8_stages;
   ga.nrg_a = p.nrg_a;
   ga.nrg_b = p.nrg_b;
   ga.sfa = base + p.off_sfa;
   ga.sfb = base + p.off_sfb;
   ga.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
   ga.ldy = ldy;
-  ga.y_vec = aligned16(Y) && (ldy * 2) % 16 == 0;
-  static bool attr_set[64] = {};
-  if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) !=
-        cudaSuccess)
-      return MXS_ERR_CUDA;
-    attr_set[dev] = true;
-  }
+  ga.y_vec = y_vec;
+  if (!ensure_smem(gemm_tc_kernel, kGemmSmemBytes)) return MXS_ERR_CUDA;
   dim3 grid(static_cast<unsigned>((N + kBN - 1) / kBN), static_cast<unsigned>((M + kBM - 1) / kBM));
   gemm_tc_kernel<<<grid, kGemmThreads, kGemmSmemBytes, cs>>>(mA16, mB16, mA8, mB8, ga);
   count_launch();

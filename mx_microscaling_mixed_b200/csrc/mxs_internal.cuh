@@ -39,6 +39,15 @@ mxs_status check_mxtensor(const mxs_mxtensor *t);
 
 inline mxs_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MXS_OK : MXS_ERR_CUDA; }
 
+// Raises a kernel's dynamic shared memory limit to at least `bytes`, once
+// per (kernel, device): the attribute belongs to the kernel on the current
+// device.
+bool ensure_smem_impl(const void *kernel, int bytes);
+template <typename Kernel>
+inline bool ensure_smem(Kernel k, int bytes) {
+  return ensure_smem_impl(reinterpret_cast<const void *>(k), bytes);
+}
+
 // ---------------------------------------------------------------- device side
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);

@@ -37,6 +37,30 @@ void count_launch(int n) {
   g_launches += n;
 }
 
+bool ensure_smem_impl(const void *kernel, int bytes) {
+  struct Entry {
+    const void *fn;
+    int dev;
+    int bytes;
+  };
+  static Entry table[256];
+  static int used = 0;
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lk(mu);
+  for (int i = 0; i < used; ++i)
+    if (table[i].fn == kernel && table[i].dev == dev && table[i].bytes >= bytes) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  for (int i = 0; i < used; ++i)
+    if (table[i].fn == kernel && table[i].dev == dev) {
+      table[i].bytes = bytes;
+      return true;
+    }
+  if (used < 256) table[used++] = Entry{kernel, dev, bytes};
+  return true;
+}
+
 mxs_status check_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MXS_ERR_CUDA;
@@ -87,33 +111,49 @@ mxs_status check_mxtensor(const mxs_mxtensor *t) {
 
 struct QuantArgs {
   const void *src;
-  int64_t ld;          // elements
-  int64_t rows, K;
-  const int32_t *perm; // NULL: identity
-  int64_t k_real[3];
-  int64_t real_off[3]; // first real position of each segment in perm order
-  int32_t nb[3];       // blocks per row per segment
+  int64_t ld;            // elements
+  int64_t rows;
+  int32_t K;
+  const int32_t *perm;   // NULL: identity
+  int32_t k_real[3];
+  int32_t real_off[3];   // first real position of each segment in perm order
+  int32_t nb[3];         // blocks per row per segment
   int32_t nb_total;
   uint8_t *codes[3];
   int64_t cpitch[3];
   uint8_t *scales[3];
   int64_t spitch[3];
+  int32_t rows_per_batch;  // rows staged per CTA iteration
+  int32_t row_stride;      // staged row length in elements (>= K + 1, multiple of 8)
+  int32_t vec_rows;        // rows are 16-byte aligned with K*esize % 16 == 0
 };
 
+constexpr uint32_t kMagic = 0x4B400000u;   // bits of 1.5 * 2^23: x + it rounds x to an integer, ties to even
+
+// Codes one block: v[] holds the 32 values of the block in position order.
+// The rounding uses the float unit: fma(v, 2^k, 1.5*2^23) rounds v*2^k (an
+// exact product) to the nearest integer with ties to even, and the integer
+// sits in the low mantissa bits of the result; clamping compares those bit
+// patterns as unsigned integers.
 template <int M>
-__device__ __forceinline__ void encode_store(const float (&v)[kBlock], uint8_t *cdst, uint8_t *sdst) {
-  uint32_t amax = 0;
+__device__ __forceinline__ void encode_store(float (&v)[kBlock], uint8_t *cdst, uint8_t *sdst) {
+  float amax = 0.f;
 #pragma unroll
-  for (int t = 0; t < kBlock; ++t) amax = max(amax, __float_as_uint(v[t]) & 0x7fffffffu);
-  const int ef = static_cast<int>(amax >> 23);   // E8M0 byte of the block
-  const int e = ef == 0 ? -127 : ef - 127;
-  const int k = M - 2 - e;
-  constexpr int L = (1 << (M - 1)) - 1;
-  int q[kBlock];
+  for (int t = 0; t < kBlock; ++t) amax = fmaxf(amax, fabsf(v[t]));
+  const int ef = static_cast<int>(__float_as_uint(amax) >> 23);   // E8M0 byte of the block
+  int k = M - 2 - (ef == 0 ? -127 : ef - 127);
+  if (k > 127) {                     // blocks below 2^-121: pre-scale by 2^64 (exact)
+#pragma unroll
+    for (int t = 0; t < kBlock; ++t) v[t] *= 18446744073709551616.0f;
+    k -= 64;
+  }
+  const float sc = __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
+  constexpr uint32_t L = (1u << (M - 1)) - 1u;
+  uint32_t b[kBlock];
 #pragma unroll
   for (int t = 0; t < kBlock; ++t) {
-    int c = __float2int_rn(scale_pow2(v[t], k));
-    q[t] = min(max(c, -L), L);
+    uint32_t x = __float_as_uint(fmaf(v[t], sc, 12582912.0f));
+    b[t] = min(max(x, kMagic - L), kMagic + L);
   }
   *sdst = static_cast<uint8_t>(ef);
   if constexpr (M == 4) {
@@ -122,46 +162,37 @@ __device__ __forceinline__ void encode_store(const float (&v)[kBlock], uint8_t *
     for (int j = 0; j < 4; ++j) {
       uint32_t x = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) x |= (static_cast<uint32_t>(q[8 * j + i]) & 0xFu) << (4 * i);
+      for (int i = 0; i < 8; ++i) x |= (b[8 * j + i] & 0xFu) << (4 * i);
       w[j] = x;
     }
     *reinterpret_cast<uint4 *>(cdst) = make_uint4(w[0], w[1], w[2], w[3]);
   } else if constexpr (M == 6) {
-    unsigned long long d[3] = {0ull, 0ull, 0ull};
+    uint32_t w[6] = {0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
     for (int t = 0; t < kBlock; ++t) {
-      const unsigned long long f = static_cast<unsigned long long>(q[t] & 0x3F);
-      const int pos = 6 * t, word = pos >> 6, off = pos & 63;
-      d[word] |= f << off;
-      if (off > 58) d[word + 1] |= f >> (64 - off);
+      const uint32_t f = b[t] & 0x3Fu;
+      const int pos = 6 * t, word = pos >> 5, off = pos & 31;
+      w[word] |= f << off;
+      if (off > 26) w[word + 1] |= f >> (32 - off);
     }
-    unsigned long long *p = reinterpret_cast<unsigned long long *>(cdst);
-    p[0] = d[0];
-    p[1] = d[1];
-    p[2] = d[2];
+    uint2 *q = reinterpret_cast<uint2 *>(cdst);
+    q[0] = make_uint2(w[0], w[1]);
+    q[1] = make_uint2(w[2], w[3]);
+    q[2] = make_uint2(w[4], w[5]);
   } else {
     uint32_t w[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      uint32_t x = 0;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) x |= (static_cast<uint32_t>(q[4 * j + i]) & 0xFFu) << (8 * i);
-      w[j] = x;
-    }
-    uint4 *p = reinterpret_cast<uint4 *>(cdst);
-    p[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    p[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    for (int j = 0; j < 8; ++j)
+      w[j] = __byte_perm(__byte_perm(b[4 * j], b[4 * j + 1], 0x0040), __byte_perm(b[4 * j + 2], b[4 * j + 3], 0x0040),
+                         0x5410);
+    uint4 *q = reinterpret_cast<uint4 *>(cdst);
+    q[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    q[1] = make_uint4(w[4], w[5], w[6], w[7]);
   }
 }
 
 template <bool F32>
-__device__ __forceinline__ float load_elem(const void *base, int64_t idx) {
-  if constexpr (F32) return __ldg(reinterpret_cast<const float *>(base) + idx);
-  else return bf16_bits_to_float(__ldg(reinterpret_cast<const unsigned short *>(base) + idx));
-}
-
-template <bool F32>
-__device__ __forceinline__ float smem_elem(const uint8_t *row, int64_t idx) {
+__device__ __forceinline__ float staged_elem(const uint8_t *row, uint32_t idx) {
   if constexpr (F32) return reinterpret_cast<const float *>(row)[idx];
   else return bf16_bits_to_float(reinterpret_cast<const unsigned short *>(row)[idx]);
 }
@@ -172,9 +203,7 @@ __device__ __forceinline__ void locate_block(const QuantArgs &a, int blk, int &g
   else { g = 2; b = blk - a.nb[0] - a.nb[1]; }
 }
 
-template <bool F32>
-__device__ __forceinline__ void code_block(const QuantArgs &a, int64_t row, int g, int b,
-                                           const float (&v)[kBlock]) {
+__device__ __forceinline__ void code_block(const QuantArgs &a, int64_t row, int g, int b, float (&v)[kBlock]) {
   uint8_t *cdst = a.codes[g] + row * a.cpitch[g] + static_cast<int64_t>(b) * kBlock * seg_bits(g) / 8;
   uint8_t *sdst = a.scales[g] + row * a.spitch[g] + b;
   if (g == 0) encode_store<8>(v, cdst, sdst);
@@ -182,11 +211,134 @@ __device__ __forceinline__ void code_block(const QuantArgs &a, int64_t row, int 
   else encode_store<4>(v, cdst, sdst);
 }
 
-// Flat grid over (row, block): positions read straight from global memory.
-// Used for the identity layout (K/V cache) and when the staged path does not
-// fit in shared memory.
+constexpr int kQuantThreads = 256;
+constexpr int kTabWordsPerBlock = 17;   // 32 uint16 source indices + 1 pad word: conflict-free pair reads
+
+__host__ __device__ inline int64_t quant_table_bytes(int64_t nb_total) {
+  return round_up(nb_total * kTabWordsPerBlock * 4, 16);
+}
+
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Issues the copies of one batch of rows into a staging buffer (cp.async
+// when rows are 16-byte aligned, plain loads otherwise).
 template <bool F32>
-__global__ void __launch_bounds__(256) quant_direct_kernel(QuantArgs a) {
+__device__ __forceinline__ void stage_rows(const QuantArgs &a, int64_t r0, int nr, uint8_t *buf, int64_t srow_bytes) {
+  constexpr int ES = F32 ? 4 : 2;
+  if (a.vec_rows) {
+    const int nvec = a.K * ES / 16;
+    for (int i = threadIdx.x; i < nr * nvec; i += blockDim.x) {
+      const int rr = i / nvec, v = i - rr * nvec;
+      cp_async16(buf + rr * srow_bytes + v * 16,
+                 reinterpret_cast<const uint8_t *>(a.src) + ((r0 + rr) * a.ld) * ES + v * 16);
+    }
+  } else {
+    for (int i = threadIdx.x; i < nr * a.K; i += blockDim.x) {
+      const int rr = i / a.K, c = i - rr * a.K;
+      const int64_t gi = (r0 + rr) * a.ld + c;
+      if constexpr (F32)
+        reinterpret_cast<float *>(buf + rr * srow_bytes)[c] = __ldg(reinterpret_cast<const float *>(a.src) + gi);
+      else
+        reinterpret_cast<unsigned short *>(buf + rr * srow_bytes)[c] =
+            __ldg(reinterpret_cast<const unsigned short *>(a.src) + gi);
+    }
+  }
+}
+
+// Persistent CTAs.  Prologue: the permutation is copied into shared memory
+// (cp.async, all requests in flight) and turned into a gather table that maps
+// every padded position of the layout to its source column (or to a zero
+// slot past the row end), 32 uint16 entries per block in 17 words.  Loop:
+// batches of rows stream through two staging buffers -- the copies of batch
+// i+1 are in flight while one thread per block of batch i gathers its 32
+// values through the table, codes and stores them.
+template <bool F32>
+__global__ void __launch_bounds__(kQuantThreads) quant_staged_kernel(QuantArgs a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint32_t *tab = reinterpret_cast<uint32_t *>(smem);
+  uint8_t *bufs = smem + quant_table_bytes(a.nb_total);
+  constexpr int ES = F32 ? 4 : 2;
+  const int RB = a.rows_per_batch;
+  const int64_t srow_bytes = static_cast<int64_t>(a.row_stride) * ES;
+  const int64_t buf_bytes = RB * srow_bytes;
+
+  // prologue: permutation -> shared memory (the staging buffers are free yet)
+  int32_t *sperm = reinterpret_cast<int32_t *>(bufs);
+  if (a.perm) {
+    if ((a.K & 3) == 0 && (reinterpret_cast<uintptr_t>(a.perm) & 15u) == 0) {
+      for (int i = threadIdx.x; i < a.K / 4; i += blockDim.x) cp_async16(sperm + 4 * i, a.perm + 4 * i);
+      cp_async_commit();
+      cp_async_wait<0>();
+    } else {
+      for (int i = threadIdx.x; i < a.K; i += blockDim.x) sperm[i] = __ldg(a.perm + i);
+    }
+  }
+  __syncthreads();
+  unsigned short *tab16 = reinterpret_cast<unsigned short *>(tab);
+  for (int i = threadIdx.x; i < a.nb_total * kBlock; i += blockDim.x) {
+    const int blk = i >> 5, t = i & 31;
+    int g, b;
+    locate_block(a, blk, g, b);
+    const int p = b * kBlock + t;
+    int col = a.K;                                   // zero slot
+    if (p < a.k_real[g]) col = a.perm ? sperm[a.real_off[g] + p] : a.real_off[g] + p;
+    tab16[blk * (2 * kTabWordsPerBlock) + t] = static_cast<unsigned short>(col);
+  }
+  __syncthreads();
+  for (int rr = threadIdx.x; rr < 2 * RB; rr += blockDim.x) {     // zero slots of both buffers
+    if constexpr (F32) reinterpret_cast<float *>(bufs + rr * srow_bytes)[a.K] = 0.f;
+    else reinterpret_cast<unsigned short *>(bufs + rr * srow_bytes)[a.K] = 0;
+  }
+
+  const int64_t nbatches = (a.rows + RB - 1) / RB;
+  int64_t batch = blockIdx.x;
+  if (batch < nbatches) stage_rows<F32>(a, batch * RB, static_cast<int>(min(static_cast<int64_t>(RB), a.rows - batch * RB)), bufs, srow_bytes);
+  cp_async_commit();
+  for (int it = 0; batch < nbatches; batch += gridDim.x, ++it) {
+    const int64_t next = batch + gridDim.x;
+    uint8_t *cur = bufs + (it & 1) * buf_bytes;
+    if (next < nbatches)
+      stage_rows<F32>(a, next * RB, static_cast<int>(min(static_cast<int64_t>(RB), a.rows - next * RB)),
+                      bufs + ((it + 1) & 1) * buf_bytes, srow_bytes);
+    cp_async_commit();
+    cp_async_wait<1>();                              // the current batch has landed
+    __syncthreads();
+    const int64_t r0 = batch * RB;
+    const int nr = static_cast<int>(min(static_cast<int64_t>(RB), a.rows - r0));
+    const int items = nr * a.nb_total;
+    for (int item = threadIdx.x; item < items; item += blockDim.x) {
+      const int rr = item / a.nb_total, blk = item - rr * a.nb_total;
+      int g, b;
+      locate_block(a, blk, g, b);
+      const uint32_t *tw = tab + blk * kTabWordsPerBlock;
+      const uint8_t *srow = cur + rr * srow_bytes;
+      float v[kBlock];
+#pragma unroll
+      for (int j = 0; j < kBlock / 2; ++j) {
+        const uint32_t w = tw[j];
+        v[2 * j] = staged_elem<F32>(srow, w & 0xFFFFu);
+        v[2 * j + 1] = staged_elem<F32>(srow, w >> 16);
+      }
+      code_block(a, r0 + rr, g, b, v);
+    }
+    __syncthreads();                                 // buffer free for the copy issued next iteration
+  }
+  cp_async_wait<0>();
+}
+
+// Fallback when a staged row does not fit in shared memory (or K >= 65535):
+// flat grid over (row, block), values read straight from global memory.
+template <bool F32>
+__global__ void __launch_bounds__(128) quant_direct_kernel(QuantArgs a) {
   const int64_t total = a.rows * a.nb_total;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -194,71 +346,21 @@ __global__ void __launch_bounds__(256) quant_direct_kernel(QuantArgs a) {
     const int blk = static_cast<int>(i - row * a.nb_total);
     int g, b;
     locate_block(a, blk, g, b);
-    const int64_t p0 = static_cast<int64_t>(b) * kBlock;
+    const int p0 = b * kBlock;
     const int64_t rbase = row * a.ld;
     float v[kBlock];
 #pragma unroll
     for (int t = 0; t < kBlock; ++t) {
-      const int64_t p = p0 + t;
+      const int p = p0 + t;
       float x = 0.f;
       if (p < a.k_real[g]) {
         const int64_t col = a.perm ? __ldg(a.perm + a.real_off[g] + p) : a.real_off[g] + p;
-        x = load_elem<F32>(a.src, rbase + col);
+        if constexpr (F32) x = __ldg(reinterpret_cast<const float *>(a.src) + rbase + col);
+        else x = bf16_bits_to_float(__ldg(reinterpret_cast<const unsigned short *>(a.src) + rbase + col));
       }
       v[t] = x;
     }
-    code_block<F32>(a, row, g, b, v);
-  }
-}
-
-constexpr int kQuantThreads = 128;
-
-__host__ __device__ inline int64_t perm_smem_words(int64_t K) { return (K / 32 + 1) * 33; }
-
-// CTA per row (grid-stride): stage the permutation once and each row once in
-// shared memory, then one thread per block gathers, codes and stores.
-template <bool F32>
-__global__ void __launch_bounds__(kQuantThreads) quant_staged_kernel(QuantArgs a) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  int32_t *sperm = reinterpret_cast<int32_t *>(smem);
-  uint8_t *srow = smem + round_up(perm_smem_words(a.K) * 4, 16);
-  constexpr int ES = F32 ? 4 : 2;
-  for (int64_t i = threadIdx.x; i < a.K; i += blockDim.x)
-    sperm[(i >> 5) * 33 + (i & 31)] = __ldg(a.perm + i);
-  const int64_t row_bytes = a.K * ES;
-  for (int64_t row = blockIdx.x; row < a.rows; row += gridDim.x) {
-    __syncthreads();
-    const uint8_t *gsrc = reinterpret_cast<const uint8_t *>(a.src) + row * a.ld * ES;
-    int64_t done = 0;
-    if ((reinterpret_cast<uintptr_t>(gsrc) & 15u) == 0) {
-      const int64_t n16 = row_bytes / 16;
-      const uint4 *s16 = reinterpret_cast<const uint4 *>(gsrc);
-      uint4 *d16 = reinterpret_cast<uint4 *>(srow);
-      for (int64_t i = threadIdx.x; i < n16; i += blockDim.x) d16[i] = __ldg(s16 + i);
-      done = n16 * 16;
-    }
-    for (int64_t i = done + threadIdx.x * ES; i < row_bytes; i += blockDim.x * ES) {
-      if constexpr (F32) *reinterpret_cast<float *>(srow + i) = __ldg(reinterpret_cast<const float *>(gsrc + i));
-      else *reinterpret_cast<unsigned short *>(srow + i) = __ldg(reinterpret_cast<const unsigned short *>(gsrc + i));
-    }
-    __syncthreads();
-    for (int blk = threadIdx.x; blk < a.nb_total; blk += blockDim.x) {
-      int g, b;
-      locate_block(a, blk, g, b);
-      const int64_t p0 = static_cast<int64_t>(b) * kBlock;
-      float v[kBlock];
-#pragma unroll
-      for (int t = 0; t < kBlock; ++t) {
-        const int64_t p = p0 + t;
-        float x = 0.f;
-        if (p < a.k_real[g]) {
-          const int64_t r = a.real_off[g] + p;
-          x = smem_elem<F32>(srow, sperm[(r >> 5) * 33 + (r & 31)]);
-        }
-        v[t] = x;
-      }
-      code_block<F32>(a, row, g, b, v);
-    }
+    code_block(a, row, g, b, v);
   }
 }
 
@@ -378,7 +480,7 @@ static mxs_status quantize_impl(const void *src, mxs_dtype dt, int64_t rows, int
   if (!out || !dtype_ok(dt)) return !out ? MXS_ERR_ARG : MXS_ERR_DTYPE;
   mxs_status st = check_mxtensor(out);
   if (st != MXS_OK) return st;
-  if (rows != out->rows || ld < out->lay.K) return MXS_ERR_SHAPE;
+  if (rows != out->rows || ld < out->lay.K || out->lay.K > INT32_MAX / 2) return MXS_ERR_SHAPE;
   if (rows == 0 || out->lay.K_pad == 0) return MXS_OK;
   if (!src) return MXS_ERR_ARG;
   if ((st = check_device()) != MXS_OK) return st;
@@ -387,16 +489,16 @@ static mxs_status quantize_impl(const void *src, mxs_dtype dt, int64_t rows, int
   a.src = src;
   a.ld = ld;
   a.rows = rows;
-  a.K = out->lay.K;
+  a.K = static_cast<int32_t>(out->lay.K);
   a.perm = out->lay.perm;
-  int64_t real = 0;
+  int32_t real = 0;
   a.nb_total = 0;
   for (int g = 0; g < 3; ++g) {
-    const mxs_segment &s = out->lay.seg[g];
-    a.k_real[g] = s.k_real;
+    const mxs_segment &sg = out->lay.seg[g];
+    a.k_real[g] = static_cast<int32_t>(sg.k_real);
     a.real_off[g] = real;
-    real += s.k_real;
-    a.nb[g] = static_cast<int32_t>(s.k_pad / kBlock);
+    real += static_cast<int32_t>(sg.k_real);
+    a.nb[g] = static_cast<int32_t>(sg.k_pad / kBlock);
     a.nb_total += a.nb[g];
     a.codes[g] = out->codes[g];
     a.cpitch[g] = out->code_pitch[g];
@@ -406,23 +508,37 @@ static mxs_status quantize_impl(const void *src, mxs_dtype dt, int64_t rows, int
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool f32 = dt == MXS_F32;
   const int64_t es = static_cast<int64_t>(dtype_size(dt));
-  const int64_t smem = round_up(perm_smem_words(a.K) * 4, 16) + round_up(a.K * es, 16);
+  a.row_stride = static_cast<int32_t>(round_up(a.K + 1, 8));
+  a.vec_rows = aligned16(src) && (ld * es) % 16 == 0 && (a.K * es) % 16 == 0;
+  const int64_t tab_bytes = quant_table_bytes(a.nb_total);
+  const int64_t srow_bytes = a.row_stride * es;
+  // rows per batch: about 16 KB of staged rows (two buffers), at least enough
+  // blocks to occupy the CTA
+  int64_t rb = std::max<int64_t>(1, (16 * 1024) / srow_bytes);
+  rb = std::max<int64_t>(rb, (kQuantThreads + a.nb_total - 1) / a.nb_total);
+  rb = std::min<int64_t>(rb, std::min<int64_t>(rows, 256));
+  auto smem_of = [&](int64_t r) { return tab_bytes + std::max<int64_t>(2 * r * srow_bytes, round_up(a.K * 4, 16)); };
+  int64_t smem = smem_of(rb);
+  while (rb > 1 && smem > 160 * 1024) smem = smem_of(--rb);
+  a.rows_per_batch = static_cast<int32_t>(rb);
   const int nsm = sm_count();
-  if (a.perm && smem <= 200 * 1024) {
-    const int per_sm = std::max<int>(1, std::min<int>(16, static_cast<int>((220 * 1024) / (smem + 1024))));
-    const int grid = static_cast<int>(std::min<int64_t>(rows, static_cast<int64_t>(nsm) * per_sm));
+  const int64_t nbatch = (rows + rb - 1) / rb;
+  const bool small = rows * a.nb_total <= 8192;       // prologue would dominate: read straight from global
+  if (!small && a.K < 65535 && smem <= 200 * 1024) {
+    const int per_sm = std::max<int>(1, std::min<int>(4, static_cast<int>((220 * 1024) / (smem + 1024))));
+    const int grid = static_cast<int>(std::min<int64_t>(nbatch, static_cast<int64_t>(nsm) * per_sm));
     if (f32) {
-      cudaFuncSetAttribute(quant_staged_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (!ensure_smem(quant_staged_kernel<true>, 200 * 1024)) return MXS_ERR_CUDA;
       quant_staged_kernel<true><<<grid, kQuantThreads, smem, s>>>(a);
     } else {
-      cudaFuncSetAttribute(quant_staged_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (!ensure_smem(quant_staged_kernel<false>, 200 * 1024)) return MXS_ERR_CUDA;
       quant_staged_kernel<false><<<grid, kQuantThreads, smem, s>>>(a);
     }
   } else {
     const int64_t total = rows * a.nb_total;
-    const int grid = static_cast<int>(std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(nsm) * 8));
-    if (f32) quant_direct_kernel<true><<<grid, 256, 0, s>>>(a);
-    else quant_direct_kernel<false><<<grid, 256, 0, s>>>(a);
+    const int grid = static_cast<int>(std::min<int64_t>((total + 127) / 128, static_cast<int64_t>(nsm) * 16));
+    if (f32) quant_direct_kernel<true><<<grid, 128, 0, s>>>(a);
+    else quant_direct_kernel<false><<<grid, 128, 0, s>>>(a);
   }
   count_launch();
   return cuda_status(cudaGetLastError());

@@ -14,9 +14,9 @@
 // intrinsics so that no fused multiply-add can change the result.
 //
 // Two launches: (1) partial sums, one CTA row per 64-row chunk of X or of W,
-// each thread owning 8 consecutive columns (16-byte bf16 / 32-byte fp32
-// loads, coalesced across the warp); for W the 4 lanes that own one 32-column
-// block share its maximum through two xor-shuffles; (2) a per-column pass that
+// each thread owning 4 consecutive columns (8-byte bf16 / 16-byte fp32 loads,
+// coalesced across the warp, 8 rows in flight); for W the 8 lanes that own
+// one 32-column block share its maximum through three xor-shuffles; (2) a per-column pass that
 // adds the chunk sums in order and forms H, E and s.
 #include <algorithm>
 
@@ -26,7 +26,7 @@ namespace mxs {
 
 constexpr int kSumChunk = 64;
 constexpr int kSensThreads = 256;
-constexpr int kColsPerThread = 8;
+constexpr int kColsPerThread = 4;
 
 struct SensArgs {
   const void *X;
@@ -37,22 +37,18 @@ struct SensArgs {
 };
 
 template <bool F32, bool VEC>
-__device__ __forceinline__ void load8(const void *base, int64_t row_off, int64_t c0, int64_t K,
+__device__ __forceinline__ void load4(const void *base, int64_t row_off, int64_t c0, int64_t K,
                                       float (&v)[kColsPerThread]) {
   if (VEC && c0 + kColsPerThread <= K) {
     if constexpr (F32) {
-      const float4 *p = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(base) + row_off + c0);
-      float4 a = __ldg(p), b = __ldg(p + 1);
+      const float4 a = __ldg(reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(base) + row_off + c0));
       v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-      v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
     } else {
-      uint4 a = __ldg(reinterpret_cast<const uint4 *>(reinterpret_cast<const unsigned short *>(base) + row_off + c0));
-      const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        v[2 * i] = __uint_as_float(w[i] << 16);
-        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-      }
+      const uint2 a = __ldg(reinterpret_cast<const uint2 *>(reinterpret_cast<const unsigned short *>(base) + row_off + c0));
+      v[0] = __uint_as_float(a.x << 16);
+      v[1] = __uint_as_float(a.x & 0xFFFF0000u);
+      v[2] = __uint_as_float(a.y << 16);
+      v[3] = __uint_as_float(a.y & 0xFFFF0000u);
     }
   } else {
 #pragma unroll
@@ -72,6 +68,44 @@ __device__ __forceinline__ double pow2d(int k) {
   return __longlong_as_double(static_cast<long long>(k + 1023) << 52);
 }
 
+constexpr int kRowBatch = 8;   // rows loaded ahead per thread
+
+// Square of x as an fp64 term (one fp64 product; exact for fp32 or bf16 x).
+__device__ __forceinline__ double square_term(float x) {
+  const double d = static_cast<double>(x);
+  return __dmul_rn(d, d);
+}
+
+// (w - Q4(w))^2 as an fp64 term, Q4 the 4-bit code under the block exponent:
+// sc = 2^(2-e) (a normal float), step = 2^(e-2).  The code comes from
+// fma(w, sc, 1.5*2^23) (round half to even), clamped on its bit pattern; the
+// same pattern minus 1.5*2^23 is the code as a float.  For bf16 w the
+// difference w - q*step has <= 9 significant bits on the bf16 grid and is
+// exact in fp32; for fp32 w it is formed in fp64.  The square is one fp64
+// product.
+template <bool F32>
+__device__ __forceinline__ double q4_err_term(float w, float sc, float step) {
+  uint32_t x = __float_as_uint(fmaf(w, sc, 12582912.0f));
+  x = min(max(x, 0x4B400000u - 7u), 0x4B400000u + 7u);
+  const float qv = __fmul_rn(__uint_as_float(x) - 12582912.0f, step);     // exact
+  double d;
+  if constexpr (F32) d = __dsub_rn(static_cast<double>(w), static_cast<double>(qv));
+  else d = static_cast<double>(__fsub_rn(w, qv));
+  return __dmul_rn(d, d);
+}
+
+// The same term for a block whose maximum is below 2^-125, where 2^(2-e)
+// is not a normal float: the code is found on the input pre-scaled by 2^64
+// and the difference is formed in fp64.
+__device__ __forceinline__ double q4_err_term_tiny(float w, int e) {
+  const float sc = __uint_as_float(static_cast<uint32_t>(2 - e - 64 + 127) << 23);
+  uint32_t x = __float_as_uint(fmaf(w * 18446744073709551616.0f, sc, 12582912.0f));
+  x = min(max(x, 0x4B400000u - 7u), 0x4B400000u + 7u);
+  const double q = static_cast<double>(__uint_as_float(x) - 12582912.0f);
+  const double d = __dsub_rn(static_cast<double>(w), __dmul_rn(q, pow2d(e - 2)));
+  return __dmul_rn(d, d);
+}
+
 template <bool XF32, bool WF32, bool XVEC, bool WVEC>
 __global__ void __launch_bounds__(kSensThreads) sens_partial_kernel(SensArgs a) {
   const int64_t gtid = static_cast<int64_t>(blockIdx.x) * kSensThreads + threadIdx.x;
@@ -84,37 +118,53 @@ __global__ void __launch_bounds__(kSensThreads) sens_partial_kernel(SensArgs a) 
     if (c0 >= a.K) return;                      // no cross-lane work on this side
     const int64_t r0 = static_cast<int64_t>(chunk) * kSumChunk;
     const int64_t r1 = min(r0 + kSumChunk, a.T);
-    for (int64_t t = r0; t < r1; ++t) {
-      float v[kColsPerThread];
-      load8<XF32, XVEC>(a.X, t * a.ldx, c0, a.K, v);
+    for (int64_t t = r0; t < r1; t += kRowBatch) {
+      float v[kRowBatch][kColsPerThread];
 #pragma unroll
-      for (int i = 0; i < kColsPerThread; ++i) {
-        const double x = static_cast<double>(v[i]);
-        acc[i] = __dadd_rn(acc[i], __dmul_rn(x, x));
+      for (int u = 0; u < kRowBatch; ++u) {
+        if (t + u < r1) load4<XF32, XVEC>(a.X, (t + u) * a.ldx, c0, a.K, v[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < kRowBatch; ++u) {
+        if (t + u < r1) {
+#pragma unroll
+          for (int i = 0; i < kColsPerThread; ++i) acc[i] = __dadd_rn(acc[i], square_term(v[u][i]));
+        }
       }
     }
   } else {
-    // All lanes stay to the end: the block maximum needs the 4 owner lanes.
+    // All lanes stay to the end: the block maximum needs the 8 owner lanes.
     const int wchunk = chunk - a.nchunk_x;
     const int64_t r0 = static_cast<int64_t>(wchunk) * kSumChunk;
     const int64_t r1 = min(r0 + kSumChunk, a.N);
-    for (int64_t i = r0; i < r1; ++i) {
-      float v[kColsPerThread];
-      load8<WF32, WVEC>(a.W, i * a.ldw, c0, a.K, v);
-      uint32_t amax = 0;
+    for (int64_t t = r0; t < r1; t += kRowBatch) {
+      float v[kRowBatch][kColsPerThread];
 #pragma unroll
-      for (int t = 0; t < kColsPerThread; ++t) amax = max(amax, __float_as_uint(v[t]) & 0x7fffffffu);
-      amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-      amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-      const int ef = static_cast<int>(amax >> 23);
-      const int e = ef == 0 ? -127 : ef - 127;
-      const double step = pow2d(e - 2);
+      for (int u = 0; u < kRowBatch; ++u) {
+        if (t + u < r1) load4<WF32, WVEC>(a.W, (t + u) * a.ldw, c0, a.K, v[u]);
+      }
 #pragma unroll
-      for (int t = 0; t < kColsPerThread; ++t) {
-        int q = __float2int_rn(scale_pow2(v[t], 2 - e));
-        q = min(max(q, -7), 7);
-        const double d = __dsub_rn(static_cast<double>(v[t]), __dmul_rn(static_cast<double>(q), step));
-        acc[t] = __dadd_rn(acc[t], __dmul_rn(d, d));
+      for (int u = 0; u < kRowBatch; ++u) {
+        if (t + u < r1) {                       // uniform across the warp
+          float amax = 0.f;
+#pragma unroll
+          for (int i = 0; i < kColsPerThread; ++i) amax = fmaxf(amax, fabsf(v[u][i]));
+          uint32_t ab = __float_as_uint(amax);
+          ab = max(ab, __shfl_xor_sync(0xffffffffu, ab, 1));   // 8 lanes own one 32-column block
+          ab = max(ab, __shfl_xor_sync(0xffffffffu, ab, 2));
+          ab = max(ab, __shfl_xor_sync(0xffffffffu, ab, 4));
+          const int ef = static_cast<int>(ab >> 23);
+          const int e = ef == 0 ? -127 : ef - 127;
+          if (e >= -125) {
+            const float sc = __uint_as_float(static_cast<uint32_t>(2 - e + 127) << 23);
+            const float step = pow2f(e - 2);
+#pragma unroll
+            for (int i = 0; i < kColsPerThread; ++i) acc[i] = __dadd_rn(acc[i], q4_err_term<WF32>(v[u][i], sc, step));
+          } else {
+#pragma unroll
+            for (int i = 0; i < kColsPerThread; ++i) acc[i] = __dadd_rn(acc[i], q4_err_term_tiny(v[u][i], e));
+          }
+        }
       }
     }
     if (c0 >= a.K) return;
@@ -125,14 +175,27 @@ __global__ void __launch_bounds__(kSensThreads) sens_partial_kernel(SensArgs a) 
     if (c0 + i < a.K) out[i] = acc[i];
 }
 
+// Sum of n chunk partials of column j in chunk order; loads are issued 8 at a
+// time ahead of the (sequential) additions.
+__device__ __forceinline__ double sum_chunks(const double *p, int n, int64_t stride) {
+  double acc = 0.0;
+  int c = 0;
+  for (; c + 8 <= n; c += 8) {
+    double v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = p[static_cast<int64_t>(c + u) * stride];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc = __dadd_rn(acc, v[u]);
+  }
+  for (; c < n; ++c) acc = __dadd_rn(acc, p[static_cast<int64_t>(c) * stride]);
+  return acc;
+}
+
 __global__ void sens_finalize_kernel(SensArgs a, double *H, double *E, double *s) {
   const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (j >= a.K) return;
-  double sx = 0.0;
-  for (int c = 0; c < a.nchunk_x; ++c) sx = __dadd_rn(sx, a.part[static_cast<int64_t>(c) * a.K + j]);
-  double se = 0.0;
-  for (int c = 0; c < a.nchunk_w; ++c)
-    se = __dadd_rn(se, a.part[static_cast<int64_t>(a.nchunk_x + c) * a.K + j]);
+  const double sx = sum_chunks(a.part + j, a.nchunk_x, a.K);
+  const double se = sum_chunks(a.part + static_cast<int64_t>(a.nchunk_x) * a.K + j, a.nchunk_w, a.K);
   const double h = __ddiv_rn(__dmul_rn(2.0, sx), static_cast<double>(a.T));
   H[j] = h;
   if (E) E[j] = se;
@@ -184,6 +247,7 @@ extern "C" mxs_status mxs_sensitivity(const void *X, mxs_dtype xt, int64_t T, in
   a.nchunk_w = static_cast<int32_t>(chunks(N));
   a.part = reinterpret_cast<double *>(ws);
   // 16-byte vector loads need aligned rows: base and pitch multiples of 16 bytes.
+  // vector loads (4 columns: 8 bytes bf16, 16 bytes fp32) need aligned rows
   const bool xvec = aligned16(X) && (ldx * static_cast<int64_t>(dtype_size(xt))) % 16 == 0;
   const bool wvec = aligned16(W) && (ldw * static_cast<int64_t>(dtype_size(wt))) % 16 == 0;
   const int64_t col_threads = (K + kColsPerThread - 1) / kColsPerThread;
@@ -195,7 +259,7 @@ extern "C" mxs_status mxs_sensitivity(const void *X, mxs_dtype xt, int64_t T, in
   else if (xf) launch_partials<true, false>(a, xvec, wvec, grid, cs);
   else if (wf) launch_partials<false, true>(a, xvec, wvec, grid, cs);
   else launch_partials<false, false>(a, xvec, wvec, grid, cs);
-  sens_finalize_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, cs>>>(a, H, E, s);
+  sens_finalize_kernel<<<static_cast<unsigned>((K + 127) / 128), 128, 0, cs>>>(a, H, E, s);
   count_launch(2);
   return cuda_status(cudaGetLastError());
 }

@@ -122,3 +122,55 @@ def test_zero_k_segments_and_strided_output(c):
     wc, ws = oracle.quantize_rows(parity.host64(W), perm, (0, 0, K))
     Yref = oracle.gemm(ac, as_, wc, ws, (0, 0, K))
     assert parity.gemm_rel_error(Ybig[:, :90].float().cpu().numpy().astype(np.float64), Yref) <= parity.GEMM_TOL
+
+
+SMALL_M = [
+    # M, N, K, counts -- every activation-row template (1, 2, 4, 8, 16), K chunking
+    # (K = 14336 at M = 16 spans several staged chunks), ragged N, and M = 17
+    # just past the decode path.
+    (2, 100, 200, (32, 64, 104)),
+    (3, 37, 96, (0, 32, 64)),
+    (5, 260, 512, (32, 96, 384)),
+    (8, 130, 1000, (40, 200, 760)),
+    (11, 64, 14336, (32, 3520, 10784)),
+    (16, 96, 14336, (32, 3520, 10784)),
+    (17, 300, 640, (32, 96, 512)),
+]
+
+
+@pytest.mark.parametrize("M,N,K,counts", SMALL_M)
+def test_gemm_small_m_matches_oracle(c, M, N, K, counts):
+    A = inputs.random_matrix(M, K, device="cuda", seed=3 * M + K, dtype=torch.bfloat16)
+    W = inputs.random_matrix(N, K, device="cuda", seed=N + K, dtype=torch.bfloat16, std=0.02)
+    Y, Yref = _run(c, A, W, counts, seed=M)
+    err = parity.gemm_rel_error(Y, Yref)
+    assert err <= parity.GEMM_TOL, f"max rel err {err:.3e}"
+
+
+def test_gemm_small_m_extreme_codes(c):
+    # blocks at the clamp (all codes +-(2^(m-1)-1)) in every segment
+    K = 256
+    A = torch.full((4, K), 1.96875, dtype=torch.bfloat16, device="cuda")
+    A[:, 1::2] = -1.96875
+    W = torch.full((40, K), -1.96875, dtype=torch.bfloat16, device="cuda")
+    Y, Yref = _run(c, A, W, (64, 64, 128), seed=9)
+    assert parity.gemm_rel_error(Y, Yref) <= parity.GEMM_TOL
+
+
+PAIR_SHAPES = [
+    # M >= 512 runs the 2-CTA pair kernel (256 x 256 tiles, persistent)
+    (512, 256, 4096, (32, 960, 3104)),
+    (600, 700, 640, (32, 96, 512)),          # ragged M and N tiles
+    (512, 512, 256, (256, 0, 0)),            # 8-bit only: bf16 MMAs only
+    (520, 300, 320, (0, 0, 320)),            # 4-bit only: block-scaled MMAs only
+    (2560, 2048, 256, (32, 64, 160)),        # 80 tiles > 74 pairs: persistent loop
+]
+
+
+@pytest.mark.parametrize("M,N,K,counts", PAIR_SHAPES)
+def test_gemm_pair_kernel_matches_oracle(c, M, N, K, counts):
+    A = inputs.random_matrix(M, K, device="cuda", seed=M + 5 * K, dtype=torch.bfloat16)
+    W = inputs.random_matrix(N, K, device="cuda", seed=N + 7 * K, dtype=torch.bfloat16, std=0.02)
+    Y, Yref = _run(c, A, W, counts, seed=M + N)
+    err = parity.gemm_rel_error(Y, Yref)
+    assert err <= parity.GEMM_TOL, f"max rel err {err:.3e}"

@@ -35,121 +35,11 @@
 #include <mutex>
 
 #include "mxs_internal.cuh"
+#include "mxs_ptx.cuh"
 
 namespace mxs {
 
-__device__ int g_gemm_status = 0;
-
-namespace ptx {
-
-__device__ __forceinline__ uint32_t smem_addr(const void *p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(b)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(b)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_addr(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
-}
-__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot)),
-               "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void mma_bf16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
-__device__ __forceinline__ void mma_mxf8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc,
-                                         uint32_t sfa, uint32_t sfb) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
-      : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint64_t *bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_addr(bar))
-               : "memory");
-}
-__device__ __forceinline__ void copy_sf_to_tmem(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-        "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-// Shared-memory matrix descriptor, K-major, 128-byte swizzle: 8-row groups
-// 1024 bytes apart; the start address may move by 32-byte K steps inside the
-// 128-byte swizzle atom (tiles are 1024-byte aligned).
-__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
-  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
-         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
-         (static_cast<uint64_t>(2) << 61);
-}
-// Descriptor of one 512-byte scale chunk for tcgen05.cp 32x128b: 32 rows of
-// 16 bytes, no swizzle, 8-row core matrices 128 bytes apart.
-__device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
-  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(128 >> 4) << 32) |
-         (static_cast<uint64_t>(1) << 46);
-}
-
-}  // namespace ptx
+__device__ int g_status = 0;
 
 constexpr int kBM = 128;           // output rows per CTA (A rows)
 constexpr int kBN = 256;           // output columns per CTA (W rows)
@@ -203,7 +93,7 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, vol
     if (*abort_flag) return false;
     if (clock64() - t0 > kWaitLimit) {
       *abort_flag = 1;
-      atomicExch(&g_gemm_status, static_cast<int>(MXS_ERR_TIMEOUT));
+      atomicExch(&g_status, static_cast<int>(MXS_ERR_TIMEOUT));
       return false;
     }
   }
@@ -748,22 +638,39 @@ __global__ void __launch_bounds__(256) gemm_stage_kernel(StageArgs a) {
         reinterpret_cast<uint4 *>(&sf_tile[0][0])[i] = make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
       __syncthreads();
       const int blk = b0 + lane;
-      for (int rr = warp; rr < kStageRows; rr += 8) {
-        const int64_t row = r0 + rr;
-        if (row >= op.rows || blk >= a.nb[2]) continue;
-        const uint4 v = *reinterpret_cast<const uint4 *>(op.codes[2] + row * op.cpitch[2] + static_cast<int64_t>(blk) * 16);
-        const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-        uint32_t out[8];
+      const bool blk_ok = blk < a.nb[2];
+      // 8 rows of loads in flight per warp, then convert and store them
+#pragma unroll 1
+      for (int r8 = 0; r8 < kStageRows / 8; r8 += 8) {
+        uint4 v[8];
+        uint8_t sb[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t x = in[j];
-          out[2 * j] = static_cast<uint32_t>(lut[x & 0xFF]) | (static_cast<uint32_t>(lut[(x >> 8) & 0xFF]) << 16);
-          out[2 * j + 1] = static_cast<uint32_t>(lut[(x >> 16) & 0xFF]) | (static_cast<uint32_t>(lut[x >> 24]) << 16);
+        for (int u = 0; u < 8; ++u) {
+          const int rr = warp + 8 * (r8 + u);
+          const int64_t row = r0 + rr;
+          if (blk_ok && row < op.rows) {
+            v[u] = *reinterpret_cast<const uint4 *>(op.codes[2] + row * op.cpitch[2] + static_cast<int64_t>(blk) * 16);
+            sb[u] = op.scales[2][row * op.spitch[2] + blk];
+          }
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(op.x8 + row * a.k4 + static_cast<int64_t>(blk) * kBlock);
-        dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-        dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-        sf_tile[lane >> 2][(rr & 31) * 16 + ((rr >> 5) & 3) * 4 + (lane & 3)] = op.scales[2][row * op.spitch[2] + blk];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int rr = warp + 8 * (r8 + u);
+          const int64_t row = r0 + rr;
+          if (!blk_ok || row >= op.rows) continue;
+          const uint32_t in[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+          uint32_t out[8];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t x = in[j];
+            out[2 * j] = static_cast<uint32_t>(lut[x & 0xFF]) | (static_cast<uint32_t>(lut[(x >> 8) & 0xFF]) << 16);
+            out[2 * j + 1] = static_cast<uint32_t>(lut[(x >> 16) & 0xFF]) | (static_cast<uint32_t>(lut[x >> 24]) << 16);
+          }
+          uint4 *dst = reinterpret_cast<uint4 *>(op.x8 + row * a.k4 + static_cast<int64_t>(blk) * kBlock);
+          dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+          dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+          sf_tile[lane >> 2][(rr & 31) * 16 + ((rr >> 5) & 3) * 4 + (lane & 3)] = sb[u];
+        }
       }
       __syncthreads();
       // whole chunks out: chunk (k-group b0/4 + c, row group rt)
@@ -780,6 +687,7 @@ __global__ void __launch_bounds__(256) gemm_stage_kernel(StageArgs a) {
       const int blk = bt * kStageBlocks + lane;
       if (blk >= a.nb[g]) continue;
       const int64_t col = (g == 0 ? 0 : a.k6_off16) + static_cast<int64_t>(blk) * kBlock;
+#pragma unroll 4
       for (int rr = warp; rr < kStageRows; rr += 8) {
         const int64_t row = static_cast<int64_t>(rt) * kStageRows + rr;
         if (row >= op.rows) break;
@@ -799,11 +707,11 @@ __global__ void __launch_bounds__(256) gemm_stage_kernel(StageArgs a) {
 // 32-position block both operands share one E8M0 scale each, so the block's
 // contribution is an integer dot product times an exact power of two:
 //   sum_t qa_t qw_t * 2^(ea - m + 2) * 2^(ew - m + 2).
-// The integer part runs on dp4a (4 byte products per instruction) with the W
-// codes in offset binary (qw + 2^(m-1), one XOR per word), the offset taken
-// back out with the A block's code sum; |sum| < 2^22, so the integer converts
-// exactly and the scaling is exact; only the fp32 accumulation over blocks
-// (and the final bf16 rounding) rounds.
+// The integer part runs on signed dp4a (4 byte products per instruction)
+// with each W code in the top bits of its byte (code * 2^(8-m), one mask per
+// word) and the activation codes sign-extended; |sum| < 2^22, so the integer
+// converts exactly and the scaling is exact; only the fp32 accumulation over
+// blocks (and the final bf16 rounding) rounds.
 // Each CTA stages the activations of one K chunk in shared memory as signed
 // bytes in the order that matches the W unpacking, then each warp runs a
 // group of R W rows: lane l takes blocks l, l+32, ... (U of them with their
@@ -827,10 +735,8 @@ struct SmallArgs {
   int64_t ldy;
 };
 
-__device__ __forceinline__ int dp4a_us(uint32_t u, uint32_t s, int c) {
-  int d;
-  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(u), "r"(s), "r"(c));
-  return d;
+__device__ __forceinline__ int dp4a_ss(uint32_t a, uint32_t b, int c) {
+  return __dp4a(static_cast<int>(a), static_cast<int>(b), c);
 }
 
 __device__ __forceinline__ void small_locate(const SmallArgs &a, int gb, int &g, int &b) {
@@ -854,16 +760,18 @@ __device__ __forceinline__ void load_w_raw(const uint8_t *c, int g, uint32_t (&w
   }
 }
 
-// 32 codes of one block as the 8 words the dp4a loop consumes, W side in
-// offset binary (code + 2^(m-1), unsigned bytes):
-// 4-bit: word 2j = codes 8j, 8j+2, 8j+4, 8j+6, word 2j+1 = the odd ones;
-// 6-bit and 8-bit: word j = codes 4j..4j+3.
+// 32 codes of one block as the 8 signed-byte words the dp4a loop consumes,
+// W side: each code sits in the top bits of its byte, i.e. the byte is
+// code * 2^(8-m) (4-bit: 16q, 6-bit: 4q, 8-bit: q) -- exact in int8 and free
+// to form (a mask, no sign extension); the 2^(8-m) goes into the exact block
+// scale.  Word order: 4-bit word 2j = codes 8j, 8j+2, 8j+4, 8j+6 and word
+// 2j+1 the odd ones; 6-bit and 8-bit word j = codes 4j..4j+3.
 __device__ __forceinline__ void unpack_w(const uint32_t (&w)[8], int g, uint32_t (&u)[8]) {
   if (g == 2) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      u[2 * j] = (w[j] & 0x0F0F0F0Fu) ^ 0x08080808u;
-      u[2 * j + 1] = ((w[j] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+      u[2 * j] = (w[j] << 4) & 0xF0F0F0F0u;
+      u[2 * j + 1] = w[j] & 0xF0F0F0F0u;
     }
   } else if (g == 1) {
 #pragma unroll
@@ -871,19 +779,16 @@ __device__ __forceinline__ void unpack_w(const uint32_t (&w)[8], int g, uint32_t
       const int pos = 24 * j, word = pos >> 5, off = pos & 31;
       uint32_t v = w[word] >> off;
       if (off > 8) v |= w[word + 1] << (32 - off);
-      const uint32_t spread = (v & 0x3Fu) | ((v << 2) & 0x3F00u) | ((v << 4) & 0x3F0000u) | ((v << 6) & 0x3F000000u);
-      u[j] = spread ^ 0x20202020u;
+      u[j] = ((v << 2) & 0xFCu) | ((v << 4) & 0xFC00u) | ((v << 6) & 0xFC0000u) | ((v << 8) & 0xFC000000u);
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) u[j] = w[j] ^ 0x80808080u;
+    for (int j = 0; j < 8; ++j) u[j] = w[j];
   }
 }
 
-// Activation side: signed bytes in the same word order, the code sum (to
-// remove the W offset) and the block's scale 2^(e-m+2).
-__device__ __forceinline__ void stage_a_block(const uint8_t *c, int g, uint32_t (&wd)[8], int &sum) {
-  sum = 0;
+// Activation side: sign-extended bytes in the same word order.
+__device__ __forceinline__ void stage_a_block(const uint8_t *c, int g, uint32_t (&wd)[8]) {
   if (g == 2) {
     const uint4 v = *reinterpret_cast<const uint4 *>(c);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -894,7 +799,6 @@ __device__ __forceinline__ void stage_a_block(const uint8_t *c, int g, uint32_t 
       for (int i = 0; i < 4; ++i) {
         const int qe = static_cast<int>(w[j] << (28 - 8 * i)) >> 28;       // nibble 2i
         const int qo = static_cast<int>(w[j] << (24 - 8 * i)) >> 28;       // nibble 2i+1
-        sum += qe + qo;
         ev |= (static_cast<uint32_t>(qe) & 0xFFu) << (8 * i);
         od |= (static_cast<uint32_t>(qo) & 0xFFu) << (8 * i);
       }
@@ -914,7 +818,6 @@ __device__ __forceinline__ void stage_a_block(const uint8_t *c, int g, uint32_t 
         uint32_t f = w[word] >> off;
         if (off > 26) f |= w[word + 1] << (32 - off);
         const int q = static_cast<int>(f << 26) >> 26;
-        sum += q;
         o |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * i);
       }
       wd[j] = o;
@@ -923,23 +826,46 @@ __device__ __forceinline__ void stage_a_block(const uint8_t *c, int g, uint32_t 
     const uint4 v0 = *reinterpret_cast<const uint4 *>(c), v1 = *reinterpret_cast<const uint4 *>(c + 16);
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      wd[j] = w[j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) sum += static_cast<int>(w[j] << (24 - 8 * i)) >> 24;
-    }
+    for (int j = 0; j < 8; ++j) wd[j] = w[j];
   }
+}
+
+// Activations in the dp4a word order, once per call, into the workspace:
+// codes [M][2][nb_total][16 B], then the block scales 2^(e-m+2) [M][NBP]
+// (float), NBP = nb_total rounded up to a multiple of 4 so every row starts
+// 16-byte aligned.  One thread per (activation row, block).
+__global__ void __launch_bounds__(128) gemm_small_prep_kernel(SmallArgs a, uint8_t *ws) {
+  const int NB = a.nb_total, NBP = (NB + 3) & ~3;
+  uint8_t *codes = ws;
+  float *fa = reinterpret_cast<float *>(ws + static_cast<int64_t>(a.M) * NB * 32);
+  const int it = blockIdx.x * blockDim.x + threadIdx.x;
+  if (it >= a.M * NB) return;
+  const int m = it / NB, b = it - m * NB;
+  int g, bb;
+  small_locate(a, b, g, bb);
+  const int mb = seg_bits(g);
+  uint32_t wd[8];
+  stage_a_block(a.a_codes[g] + m * a.a_cpitch[g] + static_cast<int64_t>(bb) * kBlock * mb / 8, g, wd);
+  const int e = static_cast<int>(a.a_scales[g][m * a.a_spitch[g] + bb]) - 127;
+  *reinterpret_cast<uint4 *>(codes + ((m * 2 + 0) * NB + b) * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+  *reinterpret_cast<uint4 *>(codes + ((m * 2 + 1) * NB + b) * 16) = make_uint4(wd[4], wd[5], wd[6], wd[7]);
+  fa[m * NBP + b] = pow2f(e - mb + 2);
+}
+
+__device__ __forceinline__ void cp_async16_g(void *smem_dst, const void *gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(gsrc)
+               : "memory");
 }
 
 // MT: activation rows handled (>= M), R: W rows per warp, U: blocks per lane
 // whose loads are issued together, WPC: warps per CTA.
 template <int MT, int R, int U, int WPC>
-__global__ void __launch_bounds__(WPC * 32) gemm_small_kernel(SmallArgs a) {
+__global__ void __launch_bounds__(WPC * 32) gemm_small_kernel(SmallArgs a, const uint8_t *__restrict__ ws) {
   extern __shared__ __align__(16) uint8_t smem[];
-  const int CB = a.chunk_blocks;
+  const int CB = a.chunk_blocks, CBP = (CB + 3) & ~3;
   uint8_t *sa = smem;                                               // [MT][2][CB][16 B]
-  int32_t *scorr = reinterpret_cast<int32_t *>(smem + static_cast<int64_t>(MT) * CB * 32);   // [MT][CB]
-  float *sfa = reinterpret_cast<float *>(scorr + MT * CB);                                     // [MT][CB]
+  float *sfa = reinterpret_cast<float *>(smem + static_cast<int64_t>(MT) * CB * 32);   // [MT][CBP]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = (blockIdx.x * WPC + warp) * R;
   float acc[R][MT];
@@ -951,19 +877,22 @@ __global__ void __launch_bounds__(WPC * 32) gemm_small_kernel(SmallArgs a) {
   for (int c0 = 0; c0 < a.nb_total; c0 += CB) {
     const int cb = min(CB, a.nb_total - c0);
     __syncthreads();
-    for (int it = threadIdx.x; it < a.M * cb; it += blockDim.x) {
-      const int m = it / cb, b = it - m * cb;
-      int g, bb;
-      small_locate(a, c0 + b, g, bb);
-      const int mb = seg_bits(g);
-      uint32_t wd[8];
-      int sum;
-      stage_a_block(a.a_codes[g] + m * a.a_cpitch[g] + static_cast<int64_t>(bb) * kBlock * mb / 8, g, wd, sum);
-      const int e = static_cast<int>(a.a_scales[g][m * a.a_spitch[g] + bb]) - 127;
-      *reinterpret_cast<uint4 *>(sa + ((m * 2 + 0) * CB + b) * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-      *reinterpret_cast<uint4 *>(sa + ((m * 2 + 1) * CB + b) * 16) = make_uint4(wd[4], wd[5], wd[6], wd[7]);
-      scorr[m * CB + b] = -(1 << (mb - 1)) * sum;                  // removes the W offset
-      sfa[m * CB + b] = pow2f(e - mb + 2);
+    {
+      // the chunk's activations, prepared once per call, copied in with every request in flight
+      const int NB = a.nb_total, NBP = (NB + 3) & ~3;
+      const float *gfa = reinterpret_cast<const float *>(ws + static_cast<int64_t>(a.M) * NB * 32);
+      for (int i = threadIdx.x; i < a.M * 2 * cb; i += blockDim.x) {
+        const int mh = i / cb, b = i - mh * cb;
+        cp_async16_g(sa + (mh * CB + b) * 16, ws + (static_cast<int64_t>(mh) * NB + c0 + b) * 16);
+      }
+      // 16-byte units of the scale rows (c0 is a multiple of 4; the last unit
+      // may carry padding entries, never read)
+      const int cbu = (cb + 3) / 4;
+      for (int i = threadIdx.x; i < a.M * cbu; i += blockDim.x) {
+        const int m = i / cbu, b = 4 * (i - m * cbu);
+        cp_async16_g(sfa + m * CBP + b, gfa + m * NBP + c0 + b);
+      }
+      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
     }
     __syncthreads();
     for (int b0 = lane; b0 < cb; b0 += 32 * U) {
@@ -985,7 +914,8 @@ __global__ void __launch_bounds__(WPC * 32) gemm_small_kernel(SmallArgs a) {
             const int n = min(n0 + r, a.N - 1);     // rows past N load row N-1 and are never stored
             load_w_raw(a.w_codes[g] + static_cast<int64_t>(n) * a.w_cpitch[g] + static_cast<int64_t>(bb) * kBlock * mb / 8,
                        g, raw[u][r]);
-            fw[u][r] = pow2f(static_cast<int>(__ldg(a.w_scales[g] + static_cast<int64_t>(n) * a.w_spitch[g] + bb)) - 127 - mb + 2);
+            // W bytes hold code * 2^(8-m): scale by 2^(e-m+2) * 2^(m-8) = 2^(e-6)
+            fw[u][r] = pow2f(static_cast<int>(__ldg(a.w_scales[g] + static_cast<int64_t>(n) * a.w_spitch[g] + bb)) - 127 - 6);
           }
         }
       }
@@ -1003,13 +933,12 @@ __global__ void __launch_bounds__(WPC * 32) gemm_small_kernel(SmallArgs a) {
             const uint4 x0 = *reinterpret_cast<const uint4 *>(sa + ((m * 2 + 0) * CB + b) * 16);
             const uint4 x1 = *reinterpret_cast<const uint4 *>(sa + ((m * 2 + 1) * CB + b) * 16);
             const uint32_t av[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-            const int corr = scorr[m * CB + b];
-            const float fa = sfa[m * CB + b];
+            const float fa = sfa[m * CBP + b];
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-              int d = corr;
+              int d = 0;
 #pragma unroll
-              for (int j = 0; j < 8; ++j) d = dp4a_us(uw[r][j], av[j], d);
+              for (int j = 0; j < 8; ++j) d = dp4a_ss(uw[r][j], av[j], d);
               acc[r][m] = fmaf(code_to_float(d), fw[u][r] * fa, acc[r][m]);
             }
           }
@@ -1036,20 +965,28 @@ __global__ void __launch_bounds__(WPC * 32) gemm_small_kernel(SmallArgs a) {
 }
 
 template <int MT, int R, int U, int WPC>
-static mxs_status launch_small(const SmallArgs &base, cudaStream_t cs) {
+static mxs_status launch_small(const SmallArgs &base, uint8_t *ws, cudaStream_t cs) {
   SmallArgs a = base;
-  const int per_block_bytes = MT * (32 + 8);
-  // about 40 KB of staged activations per CTA, several CTAs per SM
-  a.chunk_blocks = std::max(32, std::min(a.nb_total, (40 * 1024) / per_block_bytes));
-  const int smem = a.chunk_blocks * per_block_bytes;
+  const int per_block_bytes = MT * (32 + 4);
+  // about 40 KB of staged activations per CTA (several CTAs per SM); chunks
+  // are multiples of 4 blocks so the int32/float slices copy in 16-byte units
+  a.chunk_blocks = std::max(32, std::min(a.nb_total, (40 * 1024) / per_block_bytes)) & ~3;
+  if (a.chunk_blocks > a.nb_total) a.chunk_blocks = a.nb_total;
+  const int smem = MT * (a.chunk_blocks * 32 + 4 * ((a.chunk_blocks + 3) & ~3));
   if (!ensure_smem(gemm_small_kernel<MT, R, U, WPC>, 48 * 1024)) return MXS_ERR_CUDA;
+  gemm_small_prep_kernel<<<(a.M * a.nb_total + 127) / 128, 128, 0, cs>>>(a, ws);
   const int rows_per_cta = WPC * R;
-  gemm_small_kernel<MT, R, U, WPC><<<(a.N + rows_per_cta - 1) / rows_per_cta, WPC * 32, smem, cs>>>(a);
-  count_launch();
+  gemm_small_kernel<MT, R, U, WPC><<<(a.N + rows_per_cta - 1) / rows_per_cta, WPC * 32, smem, cs>>>(a, ws);
+  count_launch(2);
   return cuda_status(cudaGetLastError());
 }
 
-static mxs_status gemm_small(const mxs_mxtensor *A, const mxs_mxtensor *W, void *Y, int64_t ldy, cudaStream_t cs) {
+static size_t small_ws_bytes(int64_t M, int64_t nb_total) {
+  return static_cast<size_t>(M * nb_total * 32 + M * round_up(nb_total, 4) * 4 + 1024);
+}
+
+static mxs_status gemm_small(const mxs_mxtensor *A, const mxs_mxtensor *W, void *Y, int64_t ldy, uint8_t *ws,
+                             cudaStream_t cs) {
   SmallArgs a{};
   a.M = static_cast<int32_t>(A->rows);
   a.N = static_cast<int32_t>(W->rows);
@@ -1068,11 +1005,11 @@ static mxs_status gemm_small(const mxs_mxtensor *A, const mxs_mxtensor *W, void 
   }
   a.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
   a.ldy = ldy;
-  if (a.M <= 1) return launch_small<1, 1, 4, 8>(a, cs);
-  if (a.M <= 2) return launch_small<2, 1, 4, 8>(a, cs);
-  if (a.M <= 4) return launch_small<4, 2, 2, 8>(a, cs);
-  if (a.M <= 8) return launch_small<8, 4, 2, 4>(a, cs);
-  return launch_small<16, 4, 1, 4>(a, cs);
+  if (a.M <= 1) return launch_small<1, 1, 4, 8>(a, ws, cs);
+  if (a.M <= 2) return launch_small<2, 1, 4, 8>(a, ws, cs);
+  if (a.M <= 4) return launch_small<4, 2, 2, 8>(a, ws, cs);
+  if (a.M <= 8) return launch_small<8, 4, 2, 4>(a, ws, cs);
+  return launch_small<16, 4, 1, 4>(a, ws, cs);
 }
 
 constexpr int64_t kSmallMaxM = 16;
@@ -1141,6 +1078,33 @@ static bool make_map(CUtensorMap *m, CUtensorMapDataType dt, int esize, void *ba
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_plain_map(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, int64_t cols,
+                    int64_t rows, int64_t ld, int box_cols, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * esize)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+int *device_status_word() {
+  static int *addr[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int *>(p);
+  }
+  return addr[dev];
+}
+
 // 2-D byte map with 128-byte rows, no swizzle: the scale-chunk arrays seen as
 // rows of 128 bytes (a 512-byte chunk is 4 rows).
 static bool make_rows_map(CUtensorMap *m, void *base, int64_t total_bytes, int box_rows) {
@@ -1179,10 +1143,10 @@ using namespace mxs;
 extern "C" mxs_status mxs_sync(void *stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MXS_ERR_CUDA;
   int st = 0;
-  if (cudaMemcpyFromSymbol(&st, g_gemm_status, sizeof(int)) != cudaSuccess) return MXS_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&st, g_status, sizeof(int)) != cudaSuccess) return MXS_ERR_CUDA;
   if (st != 0) {
     const int zero = 0;
-    cudaMemcpyToSymbol(g_gemm_status, &zero, sizeof(int));
+    cudaMemcpyToSymbol(g_status, &zero, sizeof(int));
     return static_cast<mxs_status>(st);
   }
   return MXS_OK;
@@ -1192,7 +1156,7 @@ extern "C" mxs_status mxs_gemm_workspace_bytes(const mxs_mxtensor *A, const mxs_
   if (!bytes) return MXS_ERR_ARG;
   mxs_status st = gemm_check(A, W);
   if (st != MXS_OK) return st;
-  *bytes = plan_workspace(A, W).total;
+  *bytes = A->rows <= kSmallMaxM ? small_ws_bytes(A->rows, A->lay.K_pad / kBlock) : plan_workspace(A, W).total;
   return MXS_OK;
 }
 
@@ -1211,7 +1175,11 @@ extern "C" mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, voi
     return cuda_status(cudaMemset2DAsync(Y, static_cast<size_t>(ldy) * 2, 0, static_cast<size_t>(N) * 2,
                                          static_cast<size_t>(M), cs));
   }
-  if (M <= kSmallMaxM) return gemm_small(A, W, Y, ldy, cs);
+  if (M <= kSmallMaxM) {
+    const size_t need = small_ws_bytes(M, A->lay.K_pad / kBlock);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 1023u)) return MXS_ERR_WORKSPACE;
+    return gemm_small(A, W, Y, ldy, reinterpret_cast<uint8_t *>(ws), cs);
+  }
   const WsPlan p = plan_workspace(A, W);
   if (!ws || ws_bytes < p.total || (reinterpret_cast<uintptr_t>(ws) & 1023u)) return MXS_ERR_WORKSPACE;
   uint8_t *base = reinterpret_cast<uint8_t *>(ws);

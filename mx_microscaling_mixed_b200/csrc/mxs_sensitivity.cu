@@ -13,14 +13,21 @@
 // difference W - Q4(W)), formed and added with explicit round-to-nearest
 // intrinsics so that no fused multiply-add can change the result.
 //
-// Two launches: (1) partial sums, one CTA row per 64-row chunk of X or of W,
-// each thread owning 4 consecutive columns (8-byte bf16 / 16-byte fp32 loads,
-// coalesced across the warp, 8 rows in flight); for W the 8 lanes that own
-// one 32-column block share its maximum through three xor-shuffles; (2) a per-column pass that
-// adds the chunk sums in order and forms H, E and s.
+// Two launches.  (1) Chunk partials: one CTA per 64-row chunk x 256-column
+// tile of X or of W; one thread issues a single TMA tile load (zero fill past
+// the matrix edge, which adds exact zeros and leaves block maxima alone) and
+// the 64 threads each own 4 consecutive columns, walking the chunk's rows in
+// order out of shared memory; on the W side the 8 lanes that own one
+// 32-column block share its maximum through three xor-shuffles.  Several
+// CTAs per SM keep their tile loads in flight while others compute.  Rows or
+// pitches that a TMA map cannot describe (unaligned base or pitch) take a
+// register-streaming variant with the same arithmetic.  (2) A per-column pass
+// that stages the chunk partials of 32 columns in shared memory, adds them in
+// chunk order and forms H, E and s.
 #include <algorithm>
 
 #include "mxs_internal.cuh"
+#include "mxs_ptx.cuh"
 
 namespace mxs {
 
@@ -175,27 +182,132 @@ __global__ void __launch_bounds__(kSensThreads) sens_partial_kernel(SensArgs a) 
     if (c0 + i < a.K) out[i] = acc[i];
 }
 
-// Sum of n chunk partials of column j in chunk order; loads are issued 8 at a
-// time ahead of the (sequential) additions.
-__device__ __forceinline__ double sum_chunks(const double *p, int n, int64_t stride) {
-  double acc = 0.0;
-  int c = 0;
-  for (; c + 8 <= n; c += 8) {
-    double v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = p[static_cast<int64_t>(c + u) * stride];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) acc = __dadd_rn(acc, v[u]);
+constexpr int kTileCols = 256;                        // columns per tile
+constexpr int kTileThreads = kTileCols / kColsPerThread;
+constexpr long long kTileWaitLimit = 2000000000LL;    // cycles (~1 s)
+
+template <bool F32>
+__device__ __forceinline__ void lds4(const uint8_t *tile, int r, int cl, float (&v)[kColsPerThread]) {
+  if constexpr (F32) {
+    const float4 a = *reinterpret_cast<const float4 *>(tile + (static_cast<int64_t>(r) * kTileCols + cl) * 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  } else {
+    const uint2 a = *reinterpret_cast<const uint2 *>(tile + (static_cast<int64_t>(r) * kTileCols + cl) * 2);
+    v[0] = __uint_as_float(a.x << 16);
+    v[1] = __uint_as_float(a.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(a.y << 16);
+    v[3] = __uint_as_float(a.y & 0xFFFF0000u);
   }
-  for (; c < n; ++c) acc = __dadd_rn(acc, p[static_cast<int64_t>(c) * stride]);
-  return acc;
 }
 
-__global__ void sens_finalize_kernel(SensArgs a, double *H, double *E, double *s) {
-  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (j >= a.K) return;
-  const double sx = sum_chunks(a.part + j, a.nchunk_x, a.K);
-  const double se = sum_chunks(a.part + static_cast<int64_t>(a.nchunk_x) * a.K + j, a.nchunk_w, a.K);
+// One row of 4 W values: adds (w - Q4(w))^2 to acc under the 32-column
+// block's maximum (shared by the 8 lanes of the block).
+template <bool F32>
+__device__ __forceinline__ void w_row_terms(const float (&v)[kColsPerThread], double (&acc)[kColsPerThread]) {
+  uint32_t ab = 0;
+#pragma unroll
+  for (int i = 0; i < kColsPerThread; ++i) ab = max(ab, __float_as_uint(v[i]) & 0x7FFFFFFFu);
+  ab = max(ab, __shfl_xor_sync(0xffffffffu, ab, 1));
+  ab = max(ab, __shfl_xor_sync(0xffffffffu, ab, 2));
+  ab = max(ab, __shfl_xor_sync(0xffffffffu, ab, 4));
+  const int ef = static_cast<int>(ab >> 23);
+  const int e = ef == 0 ? -127 : ef - 127;
+  if (e >= -125) {
+    const float sc = __uint_as_float(static_cast<uint32_t>(2 - e + 127) << 23);
+    const float step = pow2f(e - 2);
+#pragma unroll
+    for (int i = 0; i < kColsPerThread; ++i) acc[i] = __dadd_rn(acc[i], q4_err_term<F32>(v[i], sc, step));
+  } else {
+#pragma unroll
+    for (int i = 0; i < kColsPerThread; ++i) acc[i] = __dadd_rn(acc[i], q4_err_term_tiny(v[i], e));
+  }
+}
+
+// Tiles in launch order: all X tiles (chunk-major), then all W tiles.
+template <bool XF32, bool WF32>
+__global__ void __launch_bounds__(kTileThreads)
+    sens_tile_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapW, SensArgs a,
+                     int32_t ctiles, int *status) {
+  extern __shared__ __align__(128) uint8_t tile[];
+  __shared__ __align__(8) uint64_t bar;
+  const int nx = a.nchunk_x * ctiles;
+  const bool is_x = static_cast<int>(blockIdx.x) < nx;
+  const int t = is_x ? blockIdx.x : blockIdx.x - nx;
+  const int chunk = t / ctiles, ct = t - chunk * ctiles;
+  const bool f32 = is_x ? XF32 : WF32;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    ptx::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(kSumChunk * kTileCols * (f32 ? 4 : 2)));
+    ptx::tma_load_2d(tile, is_x ? &mapX : &mapW, &bar, ct * kTileCols, chunk * kSumChunk);
+  }
+  if (!ptx::mbar_wait_cycles(&bar, 0, kTileWaitLimit)) {
+    atomicExch(status, static_cast<int>(MXS_ERR_TIMEOUT));
+    return;
+  }
+  const int cl = threadIdx.x * kColsPerThread;
+  const int64_t c0 = static_cast<int64_t>(ct) * kTileCols + cl;
+  const int64_t r0 = static_cast<int64_t>(chunk) * kSumChunk;
+  const int rows = static_cast<int>(min(static_cast<int64_t>(kSumChunk), (is_x ? a.T : a.N) - r0));
+  double acc[kColsPerThread];
+#pragma unroll
+  for (int i = 0; i < kColsPerThread; ++i) acc[i] = 0.0;
+  if (is_x) {
+#pragma unroll 8
+    for (int r = 0; r < rows; ++r) {
+      float v[kColsPerThread];
+      lds4<XF32>(tile, r, cl, v);
+#pragma unroll
+      for (int i = 0; i < kColsPerThread; ++i) acc[i] = __dadd_rn(acc[i], square_term(v[i]));
+    }
+  } else {
+#pragma unroll 4
+    for (int r = 0; r < rows; ++r) {     // rows is uniform over the CTA
+      float v[kColsPerThread];
+      lds4<WF32>(tile, r, cl, v);
+      w_row_terms<WF32>(v, acc);
+    }
+  }
+  double *out = a.part + static_cast<int64_t>(is_x ? chunk : a.nchunk_x + chunk) * a.K + c0;
+#pragma unroll
+  for (int i = 0; i < kColsPerThread; ++i)
+    if (c0 + i < a.K) out[i] = acc[i];
+}
+
+constexpr int kFinCols = 32;       // columns per CTA
+constexpr int kFinThreads = 256;
+constexpr int kFinSlab = 128;      // chunk partials staged per pass (32 KB)
+
+// Stages the partials of 32 columns, kFinSlab chunks at a time, with every
+// thread's loads in flight; one warp then adds them in chunk order.
+__global__ void __launch_bounds__(kFinThreads) sens_finalize_kernel(SensArgs a, double *H, double *E, double *s) {
+  __shared__ double sp[kFinSlab][kFinCols];
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kFinCols;
+  const int nch = a.nchunk_x + a.nchunk_w;
+  double sx = 0.0, se = 0.0;
+  for (int s0 = 0; s0 < nch; s0 += kFinSlab) {
+    const int ns = min(kFinSlab, nch - s0);
+    __syncthreads();
+#pragma unroll 4
+    for (int i = threadIdx.x; i < ns * kFinCols; i += kFinThreads) {
+      const int ch = i / kFinCols, col = i % kFinCols;
+      const int64_t c = c0 + col;
+      sp[ch][col] = c < a.K ? a.part[static_cast<int64_t>(s0 + ch) * a.K + c] : 0.0;
+    }
+    __syncthreads();
+    if (threadIdx.x < kFinCols) {
+      for (int ch = 0; ch < ns; ++ch) {
+        const double v = sp[ch][threadIdx.x];
+        if (s0 + ch < a.nchunk_x) sx = __dadd_rn(sx, v);
+        else se = __dadd_rn(se, v);
+      }
+    }
+  }
+  const int64_t j = c0 + threadIdx.x;
+  if (threadIdx.x >= kFinCols || j >= a.K) return;
   const double h = __ddiv_rn(__dmul_rn(2.0, sx), static_cast<double>(a.T));
   H[j] = h;
   if (E) E[j] = se;
@@ -246,8 +358,7 @@ extern "C" mxs_status mxs_sensitivity(const void *X, mxs_dtype xt, int64_t T, in
   a.nchunk_x = static_cast<int32_t>(chunks(T));
   a.nchunk_w = static_cast<int32_t>(chunks(N));
   a.part = reinterpret_cast<double *>(ws);
-  // 16-byte vector loads need aligned rows: base and pitch multiples of 16 bytes.
-  // vector loads (4 columns: 8 bytes bf16, 16 bytes fp32) need aligned rows
+  // vector loads and TMA tiles (4 columns: 8 bytes bf16, 16 bytes fp32) need aligned rows
   const bool xvec = aligned16(X) && (ldx * static_cast<int64_t>(dtype_size(xt))) % 16 == 0;
   const bool wvec = aligned16(W) && (ldw * static_cast<int64_t>(dtype_size(wt))) % 16 == 0;
   const int64_t col_threads = (K + kColsPerThread - 1) / kColsPerThread;
@@ -255,11 +366,43 @@ extern "C" mxs_status mxs_sensitivity(const void *X, mxs_dtype xt, int64_t T, in
             static_cast<unsigned>(a.nchunk_x + a.nchunk_w));
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const bool xf = xt == MXS_F32, wf = wt == MXS_F32;
-  if (xf && wf) launch_partials<true, true>(a, xvec, wvec, grid, cs);
-  else if (xf) launch_partials<true, false>(a, xvec, wvec, grid, cs);
-  else if (wf) launch_partials<false, true>(a, xvec, wvec, grid, cs);
-  else launch_partials<false, false>(a, xvec, wvec, grid, cs);
-  sens_finalize_kernel<<<static_cast<unsigned>((K + 127) / 128), 128, 0, cs>>>(a, H, E, s);
+  bool tiled = false;
+  if (xvec && wvec) {
+    // TMA tiles: 64 rows x 256 columns per CTA
+    CUtensorMap mx{}, mw{};
+    int *status = device_status_word();
+    const int64_t ctiles = (K + kTileCols - 1) / kTileCols;
+    const int64_t ntiles = (a.nchunk_x + a.nchunk_w) * ctiles;
+    if (status && ntiles < (1ll << 31) &&
+        make_plain_map(&mx, xf ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                       static_cast<int>(dtype_size(xt)), X, K, T, ldx, kTileCols, kSumChunk) &&
+        make_plain_map(&mw, wf ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                       static_cast<int>(dtype_size(wt)), W, K, N, ldw, kTileCols, kSumChunk)) {
+      const int smem = kSumChunk * kTileCols * ((xf || wf) ? 4 : 2);
+      const unsigned g = static_cast<unsigned>(ntiles);
+      const int32_t ct = static_cast<int32_t>(ctiles);
+      if (xf && wf) {
+        if (!ensure_smem(sens_tile_kernel<true, true>, smem)) return MXS_ERR_CUDA;
+        sens_tile_kernel<true, true><<<g, kTileThreads, smem, cs>>>(mx, mw, a, ct, status);
+      } else if (xf) {
+        if (!ensure_smem(sens_tile_kernel<true, false>, smem)) return MXS_ERR_CUDA;
+        sens_tile_kernel<true, false><<<g, kTileThreads, smem, cs>>>(mx, mw, a, ct, status);
+      } else if (wf) {
+        if (!ensure_smem(sens_tile_kernel<false, true>, smem)) return MXS_ERR_CUDA;
+        sens_tile_kernel<false, true><<<g, kTileThreads, smem, cs>>>(mx, mw, a, ct, status);
+      } else {
+        sens_tile_kernel<false, false><<<g, kTileThreads, smem, cs>>>(mx, mw, a, ct, status);
+      }
+      tiled = true;
+    }
+  }
+  if (!tiled) {
+    if (xf && wf) launch_partials<true, true>(a, xvec, wvec, grid, cs);
+    else if (xf) launch_partials<true, false>(a, xvec, wvec, grid, cs);
+    else if (wf) launch_partials<false, true>(a, xvec, wvec, grid, cs);
+    else launch_partials<false, false>(a, xvec, wvec, grid, cs);
+  }
+  sens_finalize_kernel<<<static_cast<unsigned>((K + kFinCols - 1) / kFinCols), kFinThreads, 0, cs>>>(a, H, E, s);
   count_launch(2);
   return cuda_status(cudaGetLastError());
 }

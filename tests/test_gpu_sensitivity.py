@@ -38,6 +38,11 @@ def test_parity_layer(c):
     (65, 129, 264, torch.bfloat16, torch.bfloat16),
     (1, 1, 1, torch.float32, torch.bfloat16),
     (300, 40, 1000, torch.float32, torch.bfloat16),
+    # TMA-tiled path: 16-byte aligned pitches, ragged chunk and column tile
+    (130, 200, 1000, torch.bfloat16, torch.float32),
+    (64, 64, 256, torch.float32, torch.float32),
+    (257, 65, 4104, torch.bfloat16, torch.bfloat16),
+    (3, 2, 8, torch.bfloat16, torch.bfloat16),
 ])
 def test_ragged_shapes(c, T, N, K, xd, wd):
     X = inputs.random_matrix(T, K, device="cuda", seed=T, dtype=xd)
@@ -49,6 +54,24 @@ def test_strided_inputs(c):
     Xw = inputs.random_matrix(100, 203, device="cuda", seed=1, dtype=torch.bfloat16)
     Ww = inputs.random_matrix(77, 203, device="cuda", seed=2, dtype=torch.bfloat16)
     _check(c, Xw[:, :200], Ww[:, :200])    # pitch 203: not 16-byte aligned rows
+
+
+def test_strided_aligned_inputs(c):
+    Xw = inputs.random_matrix(100, 1032, device="cuda", seed=3, dtype=torch.bfloat16)
+    Ww = inputs.random_matrix(90, 1040, device="cuda", seed=4, dtype=torch.float32)
+    _check(c, Xw[:, :1000], Ww[:, :1000])    # 16-byte aligned pitches, ragged width
+
+
+def test_tiny_and_zero_blocks(c):
+    """Blocks whose maximum is below 2^-125 (the pre-scaled code path) and
+    all-zero blocks, on the tiled and the streaming path."""
+    for K in (512, 509):
+        W = inputs.random_matrix(70, K, device="cuda", seed=5, dtype=torch.float32)
+        W[:, 32:64] *= 2.0 ** -140
+        W[3:9, 64:96] = 0.0
+        W[10, :] *= 2.0 ** -128
+        X = inputs.random_matrix(66, K, device="cuda", seed=6, dtype=torch.float32)
+        _check(c, X, W)
 
 
 def test_full_attention_layer(c):

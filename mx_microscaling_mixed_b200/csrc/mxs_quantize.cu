@@ -15,17 +15,28 @@
 //   q = clamp(rint_half_even(x * 2^(m-2-e)), -(2^(m-1)-1), 2^(m-1)-1),
 //       the scaling by a power of two being exact.
 //
-// Kernel shape: one thread codes one 32-position block (a 32-lane warp covers
-// 32 consecutive blocks), so the max is a register reduction and each thread
-// emits its packed block with 16/8-byte stores that are contiguous across
-// the warp.  With a permutation, a CTA stages the permutation once (padded to
-// 33 words per 32 so that the per-thread strided reads are bank-conflict
-// free) and each source row once, then gathers from shared memory.
+// Kernel shapes.  (1) The tiled quantiser (a permuted layout): persistent
+// CTAs, one per SM.  Batches of source rows stream into shared memory by
+// bulk copies (TMA, three buffers in flight); each block's 32 values are
+// gathered through a table built once per CTA from the permutation and coded
+// by one thread.  A warp's unit of work is G rows x 32/G blocks of one
+// segment (G = 8 when eight rows fit a buffer): lanes on different rows read
+// the same table words (broadcast) and, with a row pitch of 16 bytes mod 128,
+// mostly different banks for their gathers.  Warps take units from a shared
+// counter with no CTA-wide barrier; the warp that finishes a batch's last
+// unit refills its buffer.  (2) The identity layout (no permutation, e.g. the
+// K/V cache): one thread per block, 16-byte loads straight from global
+// memory.  (3) The lane quantiser, for a few rows or rows the bulk copies
+// cannot take (unaligned pitch, rows too long to stage): one warp per block, one lane per
+// position, the block maximum by a warp reduction and the packing by
+// shuffles; its loads are all independent, so a tiny batch (a decode step)
+// costs two memory latencies.
 #include <algorithm>
 #include <cstdio>
 #include <mutex>
 
 #include "mxs_internal.cuh"
+#include "mxs_ptx.cuh"
 
 namespace mxs {
 
@@ -123,9 +134,13 @@ struct QuantArgs {
   int64_t cpitch[3];
   uint8_t *scales[3];
   int64_t spitch[3];
-  int32_t rows_per_batch;  // rows staged per CTA iteration
-  int32_t row_stride;      // staged row length in elements (>= K + 1, multiple of 8)
-  int32_t vec_rows;        // rows are 16-byte aligned with K*esize % 16 == 0
+  int32_t boff[3];       // first block of each segment within a row
+  uint32_t nb_magic[3];   // floor(2^32 / nb[g]) + 1: i / nb[g] == umulhi(i, magic) while i * nb[g] < 2^32
+  int32_t rows_per_batch;  // rows staged per batch (a multiple of G)
+  int32_t row_stride;      // staged row pitch in elements (> K, 16 bytes mod 128)
+  int32_t lg;              // G = 1 << lg rows per work unit
+  int32_t quads[3];        // units per G-row group in each segment (ceil(nb * G / 32))
+  int32_t units_per_batch; // (rows_per_batch / G) * (quads[0] + quads[1] + quads[2])
 };
 
 constexpr uint32_t kMagic = 0x4B400000u;   // bits of 1.5 * 2^23: x + it rounds x to an integer, ties to even
@@ -191,10 +206,11 @@ __device__ __forceinline__ void encode_store(float (&v)[kBlock], uint8_t *cdst, 
   }
 }
 
+// Value at byte offset `off` of a staged row.
 template <bool F32>
-__device__ __forceinline__ float staged_elem(const uint8_t *row, uint32_t idx) {
-  if constexpr (F32) return reinterpret_cast<const float *>(row)[idx];
-  else return bf16_bits_to_float(reinterpret_cast<const unsigned short *>(row)[idx]);
+__device__ __forceinline__ float staged_elem(const uint8_t *row, uint32_t off) {
+  if constexpr (F32) return *reinterpret_cast<const float *>(row + off);
+  else return bf16_bits_to_float(*reinterpret_cast<const unsigned short *>(row + off));
 }
 
 __device__ __forceinline__ void locate_block(const QuantArgs &a, int blk, int &g, int &b) {
@@ -203,142 +219,208 @@ __device__ __forceinline__ void locate_block(const QuantArgs &a, int blk, int &g
   else { g = 2; b = blk - a.nb[0] - a.nb[1]; }
 }
 
-__device__ __forceinline__ void code_block(const QuantArgs &a, int64_t row, int g, int b, float (&v)[kBlock]) {
-  uint8_t *cdst = a.codes[g] + row * a.cpitch[g] + static_cast<int64_t>(b) * kBlock * seg_bits(g) / 8;
-  uint8_t *sdst = a.scales[g] + row * a.spitch[g] + b;
-  if (g == 0) encode_store<8>(v, cdst, sdst);
-  else if (g == 1) encode_store<6>(v, cdst, sdst);
-  else encode_store<4>(v, cdst, sdst);
-}
-
-constexpr int kQuantThreads = 256;
-constexpr int kTabWordsPerBlock = 17;   // 32 uint16 source indices + 1 pad word: conflict-free pair reads
+constexpr int kQuantThreads = 512;
+constexpr int kQuantSmemBudget = 224 * 1024;   // per CTA (one CTA per SM)
+constexpr int kQStages = 3;
+// 32 byte offsets per block + 4 pad words: 16-byte reads of up to 8
+// different blocks by one warp fall in different banks
+constexpr int kTabWordsPerBlock = 36;
+constexpr long long kQuantWaitLimit = 2000000000LL;   // cycles (~1 s)
 
 __host__ __device__ inline int64_t quant_table_bytes(int64_t nb_total) {
-  return round_up(nb_total * kTabWordsPerBlock * 4, 16);
+  return round_up(nb_total * kTabWordsPerBlock * 4, 128);
 }
 
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
-               "l"(gsrc)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-// Issues the copies of one batch of rows into a staging buffer (cp.async
-// when rows are 16-byte aligned, plain loads otherwise).
+// Warp-wide: issues the bulk copies of batch `batch` (one per row, rows
+// spread over the lanes) into buffer `buf`, completing on `bar`.
 template <bool F32>
-__device__ __forceinline__ void stage_rows(const QuantArgs &a, int64_t r0, int nr, uint8_t *buf, int64_t srow_bytes) {
+__device__ __forceinline__ void issue_batch(const QuantArgs &a, int64_t batch, uint8_t *buf, int64_t srow_bytes,
+                                            uint64_t *bar) {
   constexpr int ES = F32 ? 4 : 2;
-  if (a.vec_rows) {
-    const int nvec = a.K * ES / 16;
-    for (int i = threadIdx.x; i < nr * nvec; i += blockDim.x) {
-      const int rr = i / nvec, v = i - rr * nvec;
-      cp_async16(buf + rr * srow_bytes + v * 16,
-                 reinterpret_cast<const uint8_t *>(a.src) + ((r0 + rr) * a.ld) * ES + v * 16);
-    }
-  } else {
-    for (int i = threadIdx.x; i < nr * a.K; i += blockDim.x) {
-      const int rr = i / a.K, c = i - rr * a.K;
-      const int64_t gi = (r0 + rr) * a.ld + c;
-      if constexpr (F32)
-        reinterpret_cast<float *>(buf + rr * srow_bytes)[c] = __ldg(reinterpret_cast<const float *>(a.src) + gi);
-      else
-        reinterpret_cast<unsigned short *>(buf + rr * srow_bytes)[c] =
-            __ldg(reinterpret_cast<const unsigned short *>(a.src) + gi);
-    }
+  const int lane = threadIdx.x & 31;
+  const int64_t r0 = batch * a.rows_per_batch;
+  const int nr = static_cast<int>(min(static_cast<int64_t>(a.rows_per_batch), a.rows - r0));
+  const uint32_t row_bytes = static_cast<uint32_t>(a.K) * ES;
+  const uint8_t *src = reinterpret_cast<const uint8_t *>(a.src) + r0 * a.ld * ES;
+  // the buffer's previous contents were read through the generic proxy
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  if (lane == 0) ptx::mbar_arrive_expect_tx(bar, row_bytes * nr);
+  __syncwarp();
+  for (int rr = lane; rr < nr; rr += 32) ptx::bulk_load(buf + rr * srow_bytes, src + rr * a.ld * ES, row_bytes, bar);
+}
+
+// One lane's item of a work unit: gathers block b of segment g (width M) of
+// staged row `srow` through the table and codes it into row `row`.
+template <int M, bool F32>
+__device__ __forceinline__ void code_item(const QuantArgs &a, int g, int b, const uint32_t *tab, const uint8_t *srow,
+                                          int64_t row) {
+  const uint4 *tw = reinterpret_cast<const uint4 *>(tab + (a.boff[g] + b) * kTabWordsPerBlock);
+  float v[kBlock];
+#pragma unroll
+  for (int j = 0; j < kBlock / 4; ++j) {
+    const uint4 w = tw[j];
+    v[4 * j] = staged_elem<F32>(srow, w.x);
+    v[4 * j + 1] = staged_elem<F32>(srow, w.y);
+    v[4 * j + 2] = staged_elem<F32>(srow, w.z);
+    v[4 * j + 3] = staged_elem<F32>(srow, w.w);
   }
+  encode_store<M>(v, a.codes[g] + row * a.cpitch[g] + b * (kBlock * M / 8), a.scales[g] + row * a.spitch[g] + b);
 }
 
-// Persistent CTAs.  Prologue: the permutation is copied into shared memory
-// (cp.async, all requests in flight) and turned into a gather table that maps
-// every padded position of the layout to its source column (or to a zero
-// slot past the row end), 32 uint16 entries per block in 17 words.  Loop:
-// batches of rows stream through two staging buffers -- the copies of batch
-// i+1 are in flight while one thread per block of batch i gathers its 32
-// values through the table, codes and stores them.
+__device__ __forceinline__ bool spin_until_equal(volatile int *p, int want, long long limit) {
+  if (*p == want) return true;
+  const long long t0 = clock64();
+  while (*p != want)
+    if (clock64() - t0 > limit) return false;
+  return true;
+}
+
+// Persistent CTAs over their batches (local batch i = global batch
+// blockIdx.x + i * gridDim.x, in buffer i mod kQStages).  Prologue: warp 0
+// issues the first kQStages batches; meanwhile the CTA builds the gather
+// table (every padded position of the layout -> its source column, or a zero
+// slot past the row end, as byte offsets; 36 words per block) and writes
+// the zero slots.  Loop (per warp): take the next unit, wait until its batch
+// has been issued and has landed, code it, and count it done; the warp that
+// completes a batch refills that buffer with the batch kQStages ahead.
 template <bool F32>
-__global__ void __launch_bounds__(kQuantThreads) quant_staged_kernel(QuantArgs a) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint32_t *tab = reinterpret_cast<uint32_t *>(smem);
-  uint8_t *bufs = smem + quant_table_bytes(a.nb_total);
+__global__ void __launch_bounds__(kQuantThreads, 1) quant_tile_kernel(QuantArgs a, int *status) {
+  extern __shared__ __align__(128) uint8_t smem[];
   constexpr int ES = F32 ? 4 : 2;
+  uint32_t *tab = reinterpret_cast<uint32_t *>(smem);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + quant_table_bytes(a.nb_total));
+  uint8_t *bufs = smem + quant_table_bytes(a.nb_total) + 128;
+  __shared__ int next_unit, abort_flag;
+  __shared__ int done_cnt[kQStages];
+  __shared__ int issued[kQStages];
+  const int lane = threadIdx.x & 31;
   const int RB = a.rows_per_batch;
   const int64_t srow_bytes = static_cast<int64_t>(a.row_stride) * ES;
   const int64_t buf_bytes = RB * srow_bytes;
+  const int64_t nbatches = (a.rows + RB - 1) / RB;
+  const int nloc = blockIdx.x < nbatches ? static_cast<int>((nbatches - blockIdx.x + gridDim.x - 1) / gridDim.x) : 0;
 
-  // prologue: permutation -> shared memory (the staging buffers are free yet)
-  int32_t *sperm = reinterpret_cast<int32_t *>(bufs);
-  if (a.perm) {
-    if ((a.K & 3) == 0 && (reinterpret_cast<uintptr_t>(a.perm) & 15u) == 0) {
-      for (int i = threadIdx.x; i < a.K / 4; i += blockDim.x) cp_async16(sperm + 4 * i, a.perm + 4 * i);
-      cp_async_commit();
-      cp_async_wait<0>();
-    } else {
-      for (int i = threadIdx.x; i < a.K; i += blockDim.x) sperm[i] = __ldg(a.perm + i);
+  if (threadIdx.x == 0) {
+    next_unit = 0;
+    abort_flag = 0;
+#pragma unroll
+    for (int st = 0; st < kQStages; ++st) {
+      ptx::mbar_init(&bar[st], 1);
+      done_cnt[st] = 0;
+      issued[st] = -1;
+    }
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    for (int st = 0; st < kQStages && st < nloc; ++st)
+      issue_batch<F32>(a, blockIdx.x + static_cast<int64_t>(st) * gridDim.x, bufs + st * buf_bytes, srow_bytes,
+                       &bar[st]);
+    __syncwarp();
+    if (lane == 0)
+      for (int st = 0; st < kQStages; ++st) issued[st] = st;
+  }
+  // gather table: 8 permutation loads in flight per thread
+  for (int g = 0; g < 3; ++g) {
+    const int n = a.nb[g] * kBlock;
+    for (int p0 = threadIdx.x; p0 < n; p0 += 8 * kQuantThreads) {
+      int col[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int p = p0 + u * kQuantThreads;
+        col[u] = a.K;                                  // zero slot
+        if (p < a.k_real[g]) col[u] = a.perm ? __ldg(a.perm + a.real_off[g] + p) : a.real_off[g] + p;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int p = p0 + u * kQuantThreads;
+        if (p < n) tab[(a.boff[g] + (p >> 5)) * kTabWordsPerBlock + (p & 31)] = static_cast<uint32_t>(col[u] * ES);
+      }
     }
   }
-  __syncthreads();
-  unsigned short *tab16 = reinterpret_cast<unsigned short *>(tab);
-  for (int i = threadIdx.x; i < a.nb_total * kBlock; i += blockDim.x) {
-    const int blk = i >> 5, t = i & 31;
-    int g, b;
-    locate_block(a, blk, g, b);
-    const int p = b * kBlock + t;
-    int col = a.K;                                   // zero slot
-    if (p < a.k_real[g]) col = a.perm ? sperm[a.real_off[g] + p] : a.real_off[g] + p;
-    tab16[blk * (2 * kTabWordsPerBlock) + t] = static_cast<unsigned short>(col);
-  }
-  __syncthreads();
-  for (int rr = threadIdx.x; rr < 2 * RB; rr += blockDim.x) {     // zero slots of both buffers
+  for (int rr = threadIdx.x; rr < kQStages * RB; rr += kQuantThreads) {   // zero slots (never copied over)
     if constexpr (F32) reinterpret_cast<float *>(bufs + rr * srow_bytes)[a.K] = 0.f;
     else reinterpret_cast<unsigned short *>(bufs + rr * srow_bytes)[a.K] = 0;
   }
+  __syncthreads();
 
-  const int64_t nbatches = (a.rows + RB - 1) / RB;
-  int64_t batch = blockIdx.x;
-  if (batch < nbatches) stage_rows<F32>(a, batch * RB, static_cast<int>(min(static_cast<int64_t>(RB), a.rows - batch * RB)), bufs, srow_bytes);
-  cp_async_commit();
-  for (int it = 0; batch < nbatches; batch += gridDim.x, ++it) {
-    const int64_t next = batch + gridDim.x;
-    uint8_t *cur = bufs + (it & 1) * buf_bytes;
-    if (next < nbatches)
-      stage_rows<F32>(a, next * RB, static_cast<int>(min(static_cast<int64_t>(RB), a.rows - next * RB)),
-                      bufs + ((it + 1) & 1) * buf_bytes, srow_bytes);
-    cp_async_commit();
-    cp_async_wait<1>();                              // the current batch has landed
-    __syncthreads();
-    const int64_t r0 = batch * RB;
-    const int nr = static_cast<int>(min(static_cast<int64_t>(RB), a.rows - r0));
-    const int items = nr * a.nb_total;
-    for (int item = threadIdx.x; item < items; item += blockDim.x) {
-      const int rr = item / a.nb_total, blk = item - rr * a.nb_total;
-      int g, b;
-      locate_block(a, blk, g, b);
-      const uint32_t *tw = tab + blk * kTabWordsPerBlock;
-      const uint8_t *srow = cur + rr * srow_bytes;
-      float v[kBlock];
-#pragma unroll
-      for (int j = 0; j < kBlock / 2; ++j) {
-        const uint32_t w = tw[j];
-        v[2 * j] = staged_elem<F32>(srow, w & 0xFFFFu);
-        v[2 * j + 1] = staged_elem<F32>(srow, w >> 16);
+  const int ups = a.units_per_batch;
+  const int qt = a.quads[0] + a.quads[1] + a.quads[2];
+  const int G = 1 << a.lg;
+  const int total = nloc * ups;
+  for (;;) {
+    int u = 0;
+    if (lane == 0) u = atomicAdd(&next_unit, 1);
+    u = __shfl_sync(0xffffffffu, u, 0);
+    if (u >= total || *reinterpret_cast<volatile int *>(&abort_flag)) break;
+    const int it = u / ups, ul = u - it * ups;
+    const int st = it % kQStages;
+    bool ok = spin_until_equal(&issued[st], it, kQuantWaitLimit);
+    ok = ok && ptx::mbar_wait_cycles(&bar[st], (it / kQStages) & 1, kQuantWaitLimit);
+    if (!__all_sync(0xffffffffu, ok)) {
+      if (lane == 0) {
+        abort_flag = 1;
+        atomicExch(status, static_cast<int>(MXS_ERR_TIMEOUT));
       }
-      code_block(a, r0 + rr, g, b, v);
+      break;
     }
-    __syncthreads();                                 // buffer free for the copy issued next iteration
+    // unit -> (row group, segment, quad); lane -> (row in group, block of quad)
+    const int rg = ul / qt;
+    int q = ul - rg * qt, g = 0;
+    if (q >= a.quads[0]) {
+      q -= a.quads[0];
+      g = 1;
+      if (q >= a.quads[1]) {
+        q -= a.quads[1];
+        g = 2;
+      }
+    }
+    const int64_t r0 = (blockIdx.x + static_cast<int64_t>(it) * gridDim.x) * RB;
+    const int rl = rg * G + (lane & (G - 1));
+    const int b = q * (32 >> a.lg) + (lane >> a.lg);
+    if (r0 + rl < a.rows && b < a.nb[g]) {
+      const uint8_t *srow = bufs + st * buf_bytes + rl * srow_bytes;
+      if (g == 0) code_item<8, F32>(a, 0, b, tab, srow, r0 + rl);
+      else if (g == 1) code_item<6, F32>(a, 1, b, tab, srow, r0 + rl);
+      else code_item<4, F32>(a, 2, b, tab, srow, r0 + rl);
+    }
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+      __threadfence_block();
+      last = atomicAdd(&done_cnt[st], 1) == ups - 1;
+    }
+    if (__shfl_sync(0xffffffffu, last, 0)) {
+      // every unit of batch it is done: its buffer is free
+      if (lane == 0) done_cnt[st] = 0;
+      const int nx = it + kQStages;
+      if (nx < nloc) {
+        issue_batch<F32>(a, blockIdx.x + static_cast<int64_t>(nx) * gridDim.x, bufs + st * buf_bytes, srow_bytes,
+                         &bar[st]);
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence_block();
+          atomicExch(&issued[st], nx);
+        }
+      }
+    }
   }
-  cp_async_wait<0>();
+  __syncthreads();
+  if (abort_flag && threadIdx.x == 0) {
+    // let copies still in flight land (bounded) before the shared memory is released
+    for (int st = 0; st < kQStages; ++st) {
+      const int it = issued[st];
+      if (it >= 0) ptx::mbar_wait_cycles(&bar[st], (it / kQStages) & 1, kQuantWaitLimit);
+    }
+  }
 }
 
-// Fallback when a staged row does not fit in shared memory (or K >= 65535):
-// flat grid over (row, block), values read straight from global memory.
+// Identity layout: one thread per (row, block), values read straight from
+// global memory (16-byte loads when the block's 32 source values are
+// aligned and all real).
 template <bool F32>
-__global__ void __launch_bounds__(128) quant_direct_kernel(QuantArgs a) {
+__global__ void __launch_bounds__(256) quant_contig_kernel(QuantArgs a) {
+  constexpr int ES = F32 ? 4 : 2;
   const int64_t total = a.rows * a.nb_total;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -347,20 +429,89 @@ __global__ void __launch_bounds__(128) quant_direct_kernel(QuantArgs a) {
     int g, b;
     locate_block(a, blk, g, b);
     const int p0 = b * kBlock;
-    const int64_t rbase = row * a.ld;
+    const int64_t e0 = row * a.ld + a.real_off[g] + p0;       // element index of position p0
+    const int n = min(kBlock, a.k_real[g] - p0);
     float v[kBlock];
+    const uint8_t *base = reinterpret_cast<const uint8_t *>(a.src) + e0 * ES;
+    if (n == kBlock && (reinterpret_cast<uintptr_t>(base) & 15u) == 0) {
 #pragma unroll
-    for (int t = 0; t < kBlock; ++t) {
-      const int p = p0 + t;
-      float x = 0.f;
-      if (p < a.k_real[g]) {
-        const int64_t col = a.perm ? __ldg(a.perm + a.real_off[g] + p) : a.real_off[g] + p;
-        if constexpr (F32) x = __ldg(reinterpret_cast<const float *>(a.src) + rbase + col);
-        else x = bf16_bits_to_float(__ldg(reinterpret_cast<const unsigned short *>(a.src) + rbase + col));
+      for (int j = 0; j < kBlock * ES / 16; ++j) {
+        const uint4 x = __ldg(reinterpret_cast<const uint4 *>(base) + j);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if constexpr (F32) {
+            v[4 * j + k] = __uint_as_float(w[k]);
+          } else {
+            v[8 * j + 2 * k] = __uint_as_float(w[k] << 16);
+            v[8 * j + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+          }
+        }
       }
-      v[t] = x;
+    } else {
+#pragma unroll
+      for (int t = 0; t < kBlock; ++t) {
+        float x = 0.f;
+        if (t < n) {
+          if constexpr (F32) x = __ldg(reinterpret_cast<const float *>(a.src) + e0 + t);
+          else x = bf16_bits_to_float(__ldg(reinterpret_cast<const unsigned short *>(a.src) + e0 + t));
+        }
+        v[t] = x;
+      }
     }
-    code_block(a, row, g, b, v);
+    uint8_t *cdst = a.codes[g] + row * a.cpitch[g] + static_cast<int64_t>(b) * kBlock * seg_bits(g) / 8;
+    uint8_t *sdst = a.scales[g] + row * a.spitch[g] + b;
+    if (g == 0) encode_store<8>(v, cdst, sdst);
+    else if (g == 1) encode_store<6>(v, cdst, sdst);
+    else encode_store<4>(v, cdst, sdst);
+  }
+}
+
+// One warp per (row, block), one lane per position.
+template <bool F32>
+__global__ void __launch_bounds__(256) quant_lane_kernel(QuantArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t total = a.rows * a.nb_total;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t w = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += nwarps) {
+    const int64_t row = w / a.nb_total;
+    const int blk = static_cast<int>(w - row * a.nb_total);
+    int g, b;
+    locate_block(a, blk, g, b);
+    const int m = seg_bits(g);
+    const int p = b * kBlock + lane;
+    float x = 0.f;
+    if (p < a.k_real[g]) {
+      const int64_t col = a.perm ? __ldg(a.perm + a.real_off[g] + p) : a.real_off[g] + p;
+      if constexpr (F32) x = __ldg(reinterpret_cast<const float *>(a.src) + row * a.ld + col);
+      else x = bf16_bits_to_float(__ldg(reinterpret_cast<const unsigned short *>(a.src) + row * a.ld + col));
+    }
+    const uint32_t ab = __reduce_max_sync(0xffffffffu, __float_as_uint(x) & 0x7FFFFFFFu);
+    const int ef = static_cast<int>(ab >> 23);
+    int k = m - 2 - (ef == 0 ? -127 : ef - 127);
+    if (k > 127) {                     // blocks below 2^-121: pre-scale by 2^64 (exact)
+      x *= 18446744073709551616.0f;
+      k -= 64;
+    }
+    const uint32_t L = (1u << (m - 1)) - 1u;
+    uint32_t q = __float_as_uint(fmaf(x, __uint_as_float(static_cast<uint32_t>(k + 127) << 23), 12582912.0f));
+    q = min(max(q, kMagic - L), kMagic + L);         // low m bits: the two's-complement code
+    uint8_t *cdst = a.codes[g] + row * a.cpitch[g] + static_cast<int64_t>(b) * kBlock * m / 8;
+    const uint32_t q1 = __shfl_down_sync(0xffffffffu, q, 1);
+    const uint32_t q2 = __shfl_down_sync(0xffffffffu, q, 2);
+    const uint32_t q3 = __shfl_down_sync(0xffffffffu, q, 3);
+    if (m == 8) {
+      cdst[lane] = static_cast<uint8_t>(q);
+    } else if (m == 4) {
+      if ((lane & 1) == 0) cdst[lane >> 1] = static_cast<uint8_t>((q & 0xFu) | ((q1 & 0xFu) << 4));
+    } else if ((lane & 3) == 0) {
+      const uint32_t w24 = (q & 63u) | ((q1 & 63u) << 6) | ((q2 & 63u) << 12) | ((q3 & 63u) << 18);
+      uint8_t *d = cdst + (lane >> 2) * 3;
+      d[0] = static_cast<uint8_t>(w24);
+      d[1] = static_cast<uint8_t>(w24 >> 8);
+      d[2] = static_cast<uint8_t>(w24 >> 16);
+    }
+    if (lane == 0) a.scales[g][row * a.spitch[g] + b] = static_cast<uint8_t>(ef);
   }
 }
 
@@ -508,37 +659,68 @@ static mxs_status quantize_impl(const void *src, mxs_dtype dt, int64_t rows, int
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool f32 = dt == MXS_F32;
   const int64_t es = static_cast<int64_t>(dtype_size(dt));
-  a.row_stride = static_cast<int32_t>(round_up(a.K + 1, 8));
-  a.vec_rows = aligned16(src) && (ld * es) % 16 == 0 && (a.K * es) % 16 == 0;
-  const int64_t tab_bytes = quant_table_bytes(a.nb_total);
-  const int64_t srow_bytes = a.row_stride * es;
-  // rows per batch: about 16 KB of staged rows (two buffers), at least enough
-  // blocks to occupy the CTA
-  int64_t rb = std::max<int64_t>(1, (16 * 1024) / srow_bytes);
-  rb = std::max<int64_t>(rb, (kQuantThreads + a.nb_total - 1) / a.nb_total);
-  rb = std::min<int64_t>(rb, std::min<int64_t>(rows, 256));
-  auto smem_of = [&](int64_t r) { return tab_bytes + std::max<int64_t>(2 * r * srow_bytes, round_up(a.K * 4, 16)); };
-  int64_t smem = smem_of(rb);
-  while (rb > 1 && smem > 160 * 1024) smem = smem_of(--rb);
-  a.rows_per_batch = static_cast<int32_t>(rb);
+  int32_t boff = 0;
+  for (int g = 0; g < 3; ++g) {
+    a.boff[g] = boff;
+    boff += a.nb[g];
+    // (nb == 1 divides trivially and has no 32-bit magic)
+    a.nb_magic[g] = a.nb[g] > 1 ? static_cast<uint32_t>((1ull << 32) / static_cast<uint64_t>(a.nb[g]) + 1) : 0u;
+  }
   const int nsm = sm_count();
-  const int64_t nbatch = (rows + rb - 1) / rb;
-  const bool small = rows * a.nb_total <= 8192;       // prologue would dominate: read straight from global
-  if (!small && a.K < 65535 && smem <= 200 * 1024) {
-    const int per_sm = std::max<int>(1, std::min<int>(4, static_cast<int>((220 * 1024) / (smem + 1024))));
-    const int grid = static_cast<int>(std::min<int64_t>(nbatch, static_cast<int64_t>(nsm) * per_sm));
+  const int64_t warps = rows * a.nb_total;
+  const bool tiny = warps <= 8192;                     // latency-bound: one warp per block
+  if (!tiny && !a.perm) {
+    const int grid = static_cast<int>(std::min<int64_t>((warps + 255) / 256, static_cast<int64_t>(nsm) * 8));
+    if (f32) quant_contig_kernel<true><<<grid, 256, 0, s>>>(a);
+    else quant_contig_kernel<false><<<grid, 256, 0, s>>>(a);
+    count_launch();
+    return cuda_status(cudaGetLastError());
+  }
+  // tiled path: rows bulk-copyable (16-byte aligned base, pitch and row
+  // length) and small enough to stage
+  const bool vec_rows = aligned16(src) && (ld * es) % 16 == 0 && (a.K * es) % 16 == 0;
+  bool tiled = !tiny && vec_rows;
+  int64_t smem = 0;
+  int grid = 0;
+  if (tiled) {
+    // pitch: room for the zero slot, 16 bytes mod 128
+    const int64_t pitch = round_up((a.K + 1) * es, 128) + 16;
+    a.row_stride = static_cast<int32_t>(pitch / es);
+    const int64_t fixed = quant_table_bytes(a.nb_total) + 128;
+    const int64_t rows_fit = std::min<int64_t>(256, (kQuantSmemBudget - fixed) / kQStages / pitch);
+    tiled = rows_fit >= 1;
+    if (tiled) {
+      a.lg = rows_fit >= 8 ? 3 : rows_fit >= 4 ? 2 : rows_fit >= 2 ? 1 : 0;
+      const int64_t G = 1 << a.lg;
+      // rows per batch: a multiple of G, every CTA about the same number of batches
+      const int64_t rb_max = rows_fit / G * G;
+      const int64_t rounds = (rows + nsm * rb_max - 1) / (nsm * rb_max);
+      const int64_t rb = std::min(rb_max, round_up((rows + nsm * rounds - 1) / (nsm * rounds), G));
+      a.rows_per_batch = static_cast<int32_t>(rb);
+      int32_t qsum = 0;
+      for (int g = 0; g < 3; ++g) {
+        a.quads[g] = static_cast<int32_t>((a.nb[g] * G + 31) / 32);
+        qsum += a.quads[g];
+      }
+      a.units_per_batch = static_cast<int32_t>(rb / G) * qsum;
+      grid = static_cast<int>(std::min<int64_t>(nsm, (rows + rb - 1) / rb));
+      smem = fixed + kQStages * rb * pitch;
+    }
+  }
+  if (tiled) {
+    int *status = device_status_word();
+    if (!status) return MXS_ERR_CUDA;
     if (f32) {
-      if (!ensure_smem(quant_staged_kernel<true>, 200 * 1024)) return MXS_ERR_CUDA;
-      quant_staged_kernel<true><<<grid, kQuantThreads, smem, s>>>(a);
+      if (!ensure_smem(quant_tile_kernel<true>, static_cast<int>(smem))) return MXS_ERR_CUDA;
+      quant_tile_kernel<true><<<grid, kQuantThreads, smem, s>>>(a, status);
     } else {
-      if (!ensure_smem(quant_staged_kernel<false>, 200 * 1024)) return MXS_ERR_CUDA;
-      quant_staged_kernel<false><<<grid, kQuantThreads, smem, s>>>(a);
+      if (!ensure_smem(quant_tile_kernel<false>, static_cast<int>(smem))) return MXS_ERR_CUDA;
+      quant_tile_kernel<false><<<grid, kQuantThreads, smem, s>>>(a, status);
     }
   } else {
-    const int64_t total = rows * a.nb_total;
-    const int grid = static_cast<int>(std::min<int64_t>((total + 127) / 128, static_cast<int64_t>(nsm) * 16));
-    if (f32) quant_direct_kernel<true><<<grid, 128, 0, s>>>(a);
-    else quant_direct_kernel<false><<<grid, 128, 0, s>>>(a);
+    const int lgrid = static_cast<int>(std::min<int64_t>((warps + 7) / 8, static_cast<int64_t>(nsm) * 16));
+    if (f32) quant_lane_kernel<true><<<lgrid, 256, 0, s>>>(a);
+    else quant_lane_kernel<false><<<lgrid, 256, 0, s>>>(a);
   }
   count_launch();
   return cuda_status(cudaGetLastError());

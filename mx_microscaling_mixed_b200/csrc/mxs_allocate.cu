@@ -13,14 +13,16 @@
 // gain/cost across layers (gain = layer weight x summed s, cost = 2 N count
 // bits), stopping at the first group that does not fit.
 //
-// Device work: an all-pairs rank count (a 2-D grid: each CTA ranks 256
-// columns against a tile of 1024 candidates staged in shared memory and adds
-// its counts atomically -- exact and order-free), the group gains (one thread
-// sums one group in rank order), and a single-CTA stable compaction that
-// writes the permutation segment by segment in ascending column order.  The
-// integer budget arithmetic and the cross-layer greedy are a few hundred
-// scalar steps and run on the host side of the call; only the multi-layer
-// greedy needs device data (the group gains) and so a stream synchronisation.
+// Device work: an all-pairs rank count (each CTA ranks 32 columns against
+// every candidate, 16 threads per column each taking a slice of every
+// candidate tile staged in shared memory, partial counts added in shared
+// memory -- exact and order-free, no atomics), the group gains (one thread
+// sums one group in rank order), and a single-CTA stable compaction (a
+// block-wide scan of per-thread segment counts) that writes the permutation
+// segment by segment in ascending column order.  The integer budget
+// arithmetic and the cross-layer greedy are a few hundred scalar steps and
+// run on the host side of the call; only the multi-layer greedy needs device
+// data (the group gains) and so a stream synchronisation.
 #include <algorithm>
 #include <vector>
 
@@ -28,27 +30,50 @@
 
 namespace mxs {
 
-constexpr int kRankThreads = 256;
-constexpr int kRankTile = 1024;
+constexpr int kRankCols = 32;                     // columns ranked per CTA
+constexpr int kRankParts = 16;                    // candidate slices per column
+constexpr int kRankThreads = kRankCols * kRankParts;
+constexpr int kRankTile = 2048;                   // candidates staged per pass
+constexpr int kRankSlice = kRankTile / kRankParts;
 
-// rank[j] += #{i in this CTA's tile : s_i > s_j, or s_i == s_j and i < j}.
-// Grid: (column blocks of 256) x (tiles of 1024 candidates); rank starts at 0.
+// rank[j] = #{i : s_i > s_j, or s_i == s_j and i < j}.  Thread (part, c)
+// counts candidate slice `part` of every tile for column j = 32 blockIdx.x + c.
+// Slices wholly before j count ties, slices wholly after j do not; only the
+// slice holding j compares indices.
 __global__ void __launch_bounds__(kRankThreads) rank_kernel(const double *s, int64_t K, int32_t *rank) {
   __shared__ double tile[kRankTile];
-  const int64_t j = static_cast<int64_t>(blockIdx.x) * kRankThreads + threadIdx.x;
-  const int64_t base = static_cast<int64_t>(blockIdx.y) * kRankTile;
-  const int n = static_cast<int>(min(static_cast<int64_t>(kRankTile), K - base));
-  for (int i = threadIdx.x; i < n; i += kRankThreads) tile[i] = s[base + i];
-  __syncthreads();
-  if (j >= K) return;
-  const double sj = s[j];
+  __shared__ int part_cnt[kRankParts][kRankCols];
+  const int c = threadIdx.x % kRankCols, part = threadIdx.x / kRankCols;
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * kRankCols + c;
+  const double sj = j < K ? s[j] : 0.0;
   int r = 0;
-  const int64_t jl = j - base;     // ties count for candidates with local index < jl
-  for (int i = 0; i < n; ++i) {
-    const double si = tile[i];
-    r += (si > sj) | ((si == sj) & (i < jl));
+  for (int64_t base = 0; base < K; base += kRankTile) {
+    const int n = static_cast<int>(min(static_cast<int64_t>(kRankTile), K - base));
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += kRankThreads) tile[i] = s[base + i];
+    __syncthreads();
+    const int i0 = part * kRankSlice, i1 = min(i0 + kRankSlice, n);
+    if (base + i1 <= j) {
+#pragma unroll 8
+      for (int i = i0; i < i1; ++i) r += tile[i] >= sj;
+    } else if (base + i0 > j) {
+#pragma unroll 8
+      for (int i = i0; i < i1; ++i) r += tile[i] > sj;
+    } else {
+      for (int i = i0; i < i1; ++i) {
+        const double si = tile[i];
+        r += (si > sj) | ((si == sj) & (base + i < j));
+      }
+    }
   }
-  if (r) atomicAdd(rank + j, r);
+  part_cnt[part][c] = r;
+  __syncthreads();
+  if (threadIdx.x < kRankCols && j < K) {
+    int tot = 0;
+#pragma unroll
+    for (int q = 0; q < kRankParts; ++q) tot += part_cnt[q][threadIdx.x];
+    rank[j] = tot;
+  }
 }
 
 __global__ void order_kernel(const int32_t *rank, int64_t K, int32_t *order) {
@@ -69,42 +94,50 @@ __global__ void group_gain_kernel(const double *s, const int32_t *order, int64_t
 
 constexpr int kPermThreads = 1024;
 
-// One CTA: columns in ascending order, segment of column j from its rank;
-// block-wide ballot scans give each column its slot inside its segment.
+// One CTA.  Thread t owns columns [t*ipt, (t+1)*ipt); pass 1 counts its
+// columns of segments 0 and 1 (two 32-bit fields of one 64-bit word), a
+// block-wide exclusive scan of those words gives every thread its starting
+// slot in each segment, pass 2 writes the permutation.
 __global__ void __launch_bounds__(kPermThreads) perm_kernel(const int32_t *rank, int64_t K, int64_t n8,
                                                             int64_t n6, int32_t *perm) {
-  __shared__ int warp_cnt[3][kPermThreads / 32];
-  __shared__ int64_t running[3];
+  __shared__ unsigned long long warp_tot[kPermThreads / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (threadIdx.x < 3) running[threadIdx.x] = 0;
-  const int64_t base_of[3] = {0, n8, n8 + n6};
-  for (int64_t t0 = 0; t0 < K; t0 += kPermThreads) {
-    const int64_t j = t0 + threadIdx.x;
-    int seg = -1;
-    if (j < K) {
-      const int64_t r = rank[j];
-      seg = r < n8 ? 0 : (r < n8 + n6 ? 1 : 2);
-    }
-    int within[3];
+  const int64_t ipt = (K + kPermThreads - 1) / kPermThreads;
+  const int64_t j0 = min(K, threadIdx.x * ipt), j1 = min(K, j0 + ipt);
+  unsigned long long cnt = 0;
+#pragma unroll 4
+  for (int64_t j = j0; j < j1; ++j) {
+    const int64_t r = rank[j];
+    cnt += r < n8 ? 1ull : (r < n8 + n6 ? (1ull << 32) : 0ull);
+  }
+  unsigned long long inc = cnt;                    // inclusive warp scan
 #pragma unroll
-    for (int g = 0; g < 3; ++g) {
-      const unsigned m = __ballot_sync(0xffffffffu, seg == g);
-      within[g] = __popc(m & ((1u << lane) - 1u));
-      if (lane == 0) warp_cnt[g][warp] = __popc(m);
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long v = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += v;
+  }
+  if (lane == 31) warp_tot[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    unsigned long long w = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long v = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += v;
     }
-    __syncthreads();
-    if (seg >= 0) {
-      int64_t before = running[seg] + within[seg];
-      for (int w = 0; w < warp; ++w) before += warp_cnt[seg][w];
-      perm[base_of[seg] + before] = static_cast<int32_t>(j);
-    }
-    __syncthreads();
-    if (threadIdx.x < 3) {
-      int64_t tot = 0;
-      for (int w = 0; w < kPermThreads / 32; ++w) tot += warp_cnt[threadIdx.x][w];
-      running[threadIdx.x] += tot;
-    }
-    __syncthreads();
+    warp_tot[lane] = w;                            // inclusive over warps
+  }
+  __syncthreads();
+  const unsigned long long before = (warp ? warp_tot[warp - 1] : 0ull) + inc - cnt;
+  int64_t c0 = static_cast<int64_t>(before & 0xFFFFFFFFull), c1 = static_cast<int64_t>(before >> 32);
+  int64_t c2 = j0 - c0 - c1;
+  for (int64_t j = j0; j < j1; ++j) {
+    const int64_t r = rank[j];
+    int64_t slot;
+    if (r < n8) slot = c0++;
+    else if (r < n8 + n6) slot = n8 + c1++;
+    else slot = n8 + n6 + c2++;
+    perm[slot] = static_cast<int32_t>(j);
   }
 }
 
@@ -169,11 +202,9 @@ extern "C" mxs_status mxs_allocate(int32_t n_layers, const int64_t *K, const int
     L[l].order = reinterpret_cast<int32_t *>(p + round_up(K[l] * 4, 256));
     L[l].gains = reinterpret_cast<double *>(p + 2 * round_up(K[l] * 4, 256));
     p += layer_ws_bytes(K[l]);
-    if (cudaMemsetAsync(L[l].rank, 0, static_cast<size_t>(K[l]) * 4, cs) != cudaSuccess) return MXS_ERR_CUDA;
-    const dim3 rgrid(static_cast<unsigned>((K[l] + kRankThreads - 1) / kRankThreads),
-                     static_cast<unsigned>((K[l] + kRankTile - 1) / kRankTile));
-    rank_kernel<<<rgrid, kRankThreads, 0, cs>>>(s[l], K[l], L[l].rank);
-    count_launch(2);
+    rank_kernel<<<static_cast<unsigned>((K[l] + kRankCols - 1) / kRankCols), kRankThreads, 0, cs>>>(s[l], K[l],
+                                                                                                   L[l].rank);
+    count_launch();
   }
 
   std::vector<int64_t> n8(n_layers, 0), n6(n_layers, 0);

@@ -533,13 +533,19 @@ struct StageOperand {
   int32_t nrg;          // row groups of 128 in sf
 };
 
+// Item space of the staging kernel, one item per (operand, row, block):
+// [wide A][wide B][4-bit A][4-bit B], each range starting at a multiple of 32
+// items.  Wide items cover the 8- and 6-bit blocks of the real rows; 4-bit
+// items cover the scale-chunk grid (rows padded to 128-row groups, blocks to
+// 4-block k-groups), the padding items writing only their 2^0 scale byte.
 struct StageArgs {
   StageOperand op[2];
   int32_t nb[3];        // blocks per segment
-  int32_t nb_total;
+  int32_t nbw;          // wide blocks per row: nb[0] + nb[1]
+  int32_t nb4p;         // 4-bit blocks per row padded to k-groups: nkg * 4
   int64_t k16, k4;
-  int64_t k6_off16;     // start of the 6-bit segment inside x16 rows
   int32_t nkg;          // k-groups of 4 blocks in the 4-bit segment
+  int32_t start[5];     // item ranges (the last entry is the end)
 };
 
 __device__ __forceinline__ int64_t sf_index(int64_t r, int64_t b, int32_t nrg) {
@@ -588,114 +594,61 @@ __device__ __forceinline__ void stage_wide_block(const uint8_t *c, uint8_t sbyte
   o[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
 }
 
-// Tiles of 128 rows x 32 blocks of one segment of one operand; a CTA takes
-// tiles in a grid-stride loop.  Each warp walks 16 rows of the tile with its
-// lanes on 32 consecutive blocks, so code loads (16/24/32 bytes per lane) and
-// the converted stores (32 or 64 bytes per lane) are contiguous across the
-// warp.  For the 4-bit segment the tile's E8M0 bytes are placed in shared
-// memory in the tensor core's 512-byte chunk layout (128 rows x 4 blocks per
-// chunk; 2^0 where the tile runs past the real rows or blocks) and written
-// out as whole chunks.
-constexpr int kStageRows = 128;
-constexpr int kStageBlocks = 32;
-
+// One thread per item, warps on consecutive items (consecutive blocks of a
+// row), so code loads and converted stores are contiguous across the warp.
+// 4-bit codes become E4M3 pairs through a 256-entry table (one byte = two
+// codes); a k-group's four scale bytes are gathered by shuffles and written
+// as one word of the tensor core's 512-byte chunk layout.
 __global__ void __launch_bounds__(256) gemm_stage_kernel(StageArgs a) {
   __shared__ uint16_t lut[256];                        // byte of two 4-bit codes -> their E4M3 pair (q/4)
-  __shared__ __align__(16) uint8_t sf_tile[kStageBlocks / 4][kSfChunk];
   {
     const int b = threadIdx.x;
     const int lo = (b & 0xF) >= 8 ? (b & 0xF) - 16 : (b & 0xF);
     const int hi = (b >> 4) >= 8 ? (b >> 4) - 16 : (b >> 4);
     lut[b] = static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(make_float2(0.25f * lo, 0.25f * hi), __NV_SATFINITE, __NV_E4M3));
   }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // tile counts per (operand, segment)
-  int ntile[2][3];
-  int total = 0;
-  for (int o = 0; o < 2; ++o)
-    for (int g = 0; g < 3; ++g) {
-      const int rt = static_cast<int>((a.op[o].rows + kStageRows - 1) / kStageRows);
-      const int bt = (a.nb[g] + kStageBlocks - 1) / kStageBlocks;
-      ntile[o][g] = g == 2 ? static_cast<int>(a.op[o].nrg) * ((a.nkg * 4 + kStageBlocks - 1) / kStageBlocks) : rt * bt;
-      if (a.nb[g] == 0) ntile[o][g] = 0;
-      total += ntile[o][g];
-    }
   __syncthreads();
-  for (int t = blockIdx.x; t < total; t += gridDim.x) {
-    int o = 0, g = 0, w = t;
-    while (w >= ntile[o][g]) {
-      w -= ntile[o][g];
-      if (++g == 3) { g = 0; ++o; }
-    }
-    const StageOperand &op = a.op[o];
-    const int m = seg_bits(g);
-    if (g == 2) {
-      // 4-bit: tiles cover the chunk grid (row groups x groups of 8 k-groups)
-      const int kg_tiles = (a.nkg * 4 + kStageBlocks - 1) / kStageBlocks;
-      const int rt = w / kg_tiles, bt = w - rt * kg_tiles;
-      const int r0 = rt * kStageRows, b0 = bt * kStageBlocks;
-      for (int i = threadIdx.x; i < (kStageBlocks / 4) * kSfChunk / 16; i += blockDim.x)
-        reinterpret_cast<uint4 *>(&sf_tile[0][0])[i] = make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-      __syncthreads();
-      const int blk = b0 + lane;
-      const bool blk_ok = blk < a.nb[2];
-      // 8 rows of loads in flight per warp, then convert and store them
-#pragma unroll 1
-      for (int r8 = 0; r8 < kStageRows / 8; r8 += 8) {
-        uint4 v[8];
-        uint8_t sb[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int rr = warp + 8 * (r8 + u);
-          const int64_t row = r0 + rr;
-          if (blk_ok && row < op.rows) {
-            v[u] = *reinterpret_cast<const uint4 *>(op.codes[2] + row * op.cpitch[2] + static_cast<int64_t>(blk) * 16);
-            sb[u] = op.scales[2][row * op.spitch[2] + blk];
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int rr = warp + 8 * (r8 + u);
-          const int64_t row = r0 + rr;
-          if (!blk_ok || row >= op.rows) continue;
-          const uint32_t in[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-          uint32_t out[8];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t x = in[j];
-            out[2 * j] = static_cast<uint32_t>(lut[x & 0xFF]) | (static_cast<uint32_t>(lut[(x >> 8) & 0xFF]) << 16);
-            out[2 * j + 1] = static_cast<uint32_t>(lut[(x >> 16) & 0xFF]) | (static_cast<uint32_t>(lut[x >> 24]) << 16);
-          }
-          uint4 *dst = reinterpret_cast<uint4 *>(op.x8 + row * a.k4 + static_cast<int64_t>(blk) * kBlock);
-          dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-          dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-          sf_tile[lane >> 2][(rr & 31) * 16 + ((rr >> 5) & 3) * 4 + (lane & 3)] = sb[u];
-        }
+  const int lane = threadIdx.x & 31;
+  const int nwarps = gridDim.x * (blockDim.x >> 5);
+  for (int base = (blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 32; base < a.start[4]; base += nwarps * 32) {
+    int rg = 0;                                        // range of this warp (uniform)
+    while (rg < 3 && base >= a.start[rg + 1]) ++rg;
+    const int i = base + lane - a.start[rg];
+    const bool in_range = base + lane < a.start[rg + 1];
+    const StageOperand &op = a.op[rg & 1];
+    if (rg < 2) {
+      const int row = i / a.nbw, b = i - row * a.nbw;
+      if (in_range && row < op.rows) {
+        const int g = b < a.nb[0] ? 0 : 1;
+        const int bb = g == 0 ? b : b - a.nb[0];
+        const uint8_t sbyte = op.scales[g][row * op.spitch[g] + bb];
+        __nv_bfloat16 *dst = op.x16 + static_cast<int64_t>(row) * a.k16 + static_cast<int64_t>(b) * kBlock;
+        if (g == 0) stage_wide_block<8>(op.codes[0] + row * op.cpitch[0] + static_cast<int64_t>(bb) * 32, sbyte, dst);
+        else stage_wide_block<6>(op.codes[1] + row * op.cpitch[1] + static_cast<int64_t>(bb) * 24, sbyte, dst);
       }
-      __syncthreads();
-      // whole chunks out: chunk (k-group b0/4 + c, row group rt)
-      const int nchunks = min(kStageBlocks / 4, a.nkg - b0 / 4);
-      for (int i = threadIdx.x; i < nchunks * kSfChunk / 16; i += blockDim.x) {
-        const int c = i / (kSfChunk / 16), e = i - c * (kSfChunk / 16);
-        uint4 *dst = reinterpret_cast<uint4 *>(op.sf + (static_cast<int64_t>(b0 / 4 + c) * op.nrg + rt) * kSfChunk);
-        dst[e] = reinterpret_cast<const uint4 *>(&sf_tile[c][0])[e];
-      }
-      __syncthreads();
     } else {
-      const int bt_n = (a.nb[g] + kStageBlocks - 1) / kStageBlocks;
-      const int rt = w / bt_n, bt = w - rt * bt_n;
-      const int blk = bt * kStageBlocks + lane;
-      if (blk >= a.nb[g]) continue;
-      const int64_t col = (g == 0 ? 0 : a.k6_off16) + static_cast<int64_t>(blk) * kBlock;
-#pragma unroll 4
-      for (int rr = warp; rr < kStageRows; rr += 8) {
-        const int64_t row = static_cast<int64_t>(rt) * kStageRows + rr;
-        if (row >= op.rows) break;
-        const uint8_t *c = op.codes[g] + row * op.cpitch[g] + static_cast<int64_t>(blk) * kBlock * m / 8;
-        const uint8_t sbyte = op.scales[g][row * op.spitch[g] + blk];
-        if (g == 0) stage_wide_block<8>(c, sbyte, op.x16 + row * a.k16 + col);
-        else stage_wide_block<6>(c, sbyte, op.x16 + row * a.k16 + col);
+      const int row = i / a.nb4p, b = i - row * a.nb4p;
+      uint32_t sb = 0x7Fu;                             // 2^0 for padding rows and blocks
+      if (in_range && row < op.rows && b < a.nb[2]) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(op.codes[2] + row * op.cpitch[2] + static_cast<int64_t>(b) * 16);
+        sb = op.scales[2][row * op.spitch[2] + b];
+        const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+        uint32_t out[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t x = in[j];
+          out[2 * j] = static_cast<uint32_t>(lut[x & 0xFF]) | (static_cast<uint32_t>(lut[(x >> 8) & 0xFF]) << 16);
+          out[2 * j + 1] = static_cast<uint32_t>(lut[(x >> 16) & 0xFF]) | (static_cast<uint32_t>(lut[x >> 24]) << 16);
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(op.x8 + static_cast<int64_t>(row) * a.k4 + static_cast<int64_t>(b) * kBlock);
+        dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+        dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
       }
+      // lanes 4j..4j+3 hold blocks 4k..4k+3 of one row (ranges and nb4p are multiples of 4)
+      sb |= __shfl_down_sync(0xffffffffu, sb, 1) << 8;
+      sb |= __shfl_down_sync(0xffffffffu, sb, 2) << 16;
+      if (in_range && (lane & 3) == 0)
+        *reinterpret_cast<uint32_t *>(op.sf + sf_index(row, b, op.nrg)) = sb;
     }
   }
 }
@@ -707,22 +660,29 @@ __global__ void __launch_bounds__(256) gemm_stage_kernel(StageArgs a) {
 // 32-position block both operands share one E8M0 scale each, so the block's
 // contribution is an integer dot product times an exact power of two:
 //   sum_t qa_t qw_t * 2^(ea - m + 2) * 2^(ew - m + 2).
-// The integer part runs on signed dp4a (4 byte products per instruction)
-// with each W code in the top bits of its byte (code * 2^(8-m), one mask per
-// word) and the activation codes sign-extended; |sum| < 2^22, so the integer
-// converts exactly and the scaling is exact; only the fp32 accumulation over
-// blocks (and the final bf16 rounding) rounds.
-// Each CTA stages the activations of one K chunk in shared memory as signed
-// bytes in the order that matches the W unpacking, then each warp runs a
-// group of R W rows: lane l takes blocks l, l+32, ... (U of them with their
-// loads in flight together) and a butterfly
-// over the warp sums the lanes.
-
+// Every code is widened to a signed byte holding code * 2^(8-m) (the code
+// in the top bits of the byte: a mask, no sign extension), so one 32-column
+// block of either operand is 32 int8 values and the block's integer dot
+// product is exactly one tensor-core mma.sync m16n8k32 (s8 x s8 -> s32),
+// 16 activation rows x 8 W rows.  |sum| < 2^22, so the int32 converts
+// exactly, and the scale 2^(ea-6) * 2^(ew-6) is exact; only the fp32
+// accumulation over blocks (and the final bf16 rounding) rounds.  The block
+// scaling forbids accumulating across blocks inside the tensor core, which
+// is why the block-sized warp-level MMA is used here rather than tcgen05.
+//
+// Each CTA owns 16 W rows (two n-tiles of 8); its eight warps split the K
+// blocks of each segment (warp w takes blocks w, w+8, ...).  One thread
+// bulk-copies (TMA) the activations' packed code and scale rows and the 16 W
+// rows' scale rows into shared memory; every lane then builds, per block, its
+// A fragment from the shared copy and its B fragments from the packed W
+// bytes in HBM (streaming loads, no L1 allocation, several blocks in
+// flight), widening only the two 4-code groups a fragment holds.  The warps'
+// partial sums are added in shared memory in warp order.  Calls whose packed
+// activation rows do not fit in shared memory take the tensor-core path.
 struct SmallArgs {
   int32_t M, N;
   int32_t nb[3];
   int32_t nb_total;
-  int32_t chunk_blocks;              // blocks staged per K chunk
   const uint8_t *a_codes[3];
   int64_t a_cpitch[3];
   const uint8_t *a_scales[3];
@@ -735,9 +695,10 @@ struct SmallArgs {
   int64_t ldy;
 };
 
-__device__ __forceinline__ int dp4a_ss(uint32_t a, uint32_t b, int c) {
-  return __dp4a(static_cast<int>(a), static_cast<int>(b), c);
-}
+constexpr int kDecRows = 16;                 // W rows per CTA (two n-tiles of 8)
+constexpr int kDecMaxM = 16;                 // activation rows: the MMA's 16 rows
+constexpr int kDecWarps = 8;                 // K slots
+constexpr int kDecThreads = kDecWarps * 32;
 
 __device__ __forceinline__ void small_locate(const SmallArgs &a, int gb, int &g, int &b) {
   if (gb < a.nb[0]) { g = 0; b = gb; }
@@ -745,248 +706,251 @@ __device__ __forceinline__ void small_locate(const SmallArgs &a, int gb, int &g,
   else { g = 2; b = gb - a.nb[0] - a.nb[1]; }
 }
 
-// Raw packed words of one W block (4-bit: 4 words, 6-bit: 6, 8-bit: 8).
-__device__ __forceinline__ void load_w_raw(const uint8_t *c, int g, uint32_t (&w)[8]) {
-  if (g == 2) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(c));
-    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-  } else if (g == 1) {
-    const uint2 x0 = __ldg(reinterpret_cast<const uint2 *>(c)), x1 = __ldg(reinterpret_cast<const uint2 *>(c + 8)),
-                x2 = __ldg(reinterpret_cast<const uint2 *>(c + 16));
-    w[0] = x0.x; w[1] = x0.y; w[2] = x1.x; w[3] = x1.y; w[4] = x2.x; w[5] = x2.y;
+// Four 4-bit codes (16 bits, code i in nibble i) -> four bytes code << 4.
+__device__ __forceinline__ uint32_t widen4(uint32_t x16) {
+  const uint32_t p = __byte_perm(x16, 0, 0x1100);       // bytes b0 b0 b1 b1
+  return ((p << 4) & 0x00F000F0u) | (p & 0xF000F000u);
+}
+// Four 6-bit codes (24 bits, code i at bits 6i) -> four bytes code << 2.
+__device__ __forceinline__ uint32_t widen6(uint32_t v) {
+  return ((v << 2) & 0xFCu) | ((v << 4) & 0xFC00u) | ((v << 6) & 0xFC0000u) | ((v << 8) & 0xFC000000u);
+}
+
+__device__ __forceinline__ void mma_s8_16x8x32(const uint4 &a, uint32_t b0, uint32_t b1, int (&c)[4]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%10, %11, %12, %13};"
+      : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1), "r"(0), "r"(0), "r"(0), "r"(0));
+}
+
+__device__ __forceinline__ uint32_t ld_stream_u16(const uint8_t *p) {
+  unsigned short v;
+  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_stream_u32(const uint8_t *p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
+// Per segment: raw words one lane loads for its B fragment of one W block,
+// and how many blocks a warp keeps in flight.
+template <int G> struct DecSeg;
+template <> struct DecSeg<0> { static constexpr int kRaw = 2, kU = 4; };   // 8-bit: words t, 4+t
+template <> struct DecSeg<1> { static constexpr int kRaw = 4, kU = 4; };   // 6-bit: two word pairs
+template <> struct DecSeg<2> { static constexpr int kRaw = 2, kU = 8; };   // 4-bit: two 16-bit groups
+
+__device__ __forceinline__ uint32_t lds_u16(const uint8_t *p) { return *reinterpret_cast<const unsigned short *>(p); }
+__device__ __forceinline__ uint32_t lds_u32(const uint8_t *p) { return *reinterpret_cast<const uint32_t *>(p); }
+
+// The words of block c (packed, m-bit) that lane-in-group t needs for its
+// fragment: code groups t and 4+t (codes 4t..4t+3 and 16+4t..16+4t+3).
+// SMEM: c points into shared memory (activations), else into global memory
+// (W, streaming loads).
+template <int G, bool SMEM>
+__device__ __forceinline__ void load_frag_raw(const uint8_t *c, int t, uint32_t (&r)[DecSeg<G>::kRaw]) {
+  if constexpr (G == 2) {
+    r[0] = SMEM ? lds_u16(c + 2 * t) : ld_stream_u16(c + 2 * t);
+    r[1] = SMEM ? lds_u16(c + 8 + 2 * t) : ld_stream_u16(c + 8 + 2 * t);
+  } else if constexpr (G == 0) {
+    r[0] = SMEM ? lds_u32(c + 4 * t) : ld_stream_u32(c + 4 * t);
+    r[1] = SMEM ? lds_u32(c + 16 + 4 * t) : ld_stream_u32(c + 16 + 4 * t);
   } else {
-    const uint4 v0 = __ldg(reinterpret_cast<const uint4 *>(c)), v1 = __ldg(reinterpret_cast<const uint4 *>(c + 16));
-    w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w; w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+    // group t: bytes 3t..3t+2, inside words (3t)/4 and (3t+2)/4
+    const int w0 = 4 * ((3 * t) >> 2), w1 = 4 * ((3 * t + 2) >> 2);
+    r[0] = SMEM ? lds_u32(c + w0) : ld_stream_u32(c + w0);
+    r[1] = SMEM ? lds_u32(c + w1) : ld_stream_u32(c + w1);
+    r[2] = SMEM ? lds_u32(c + 12 + w0) : ld_stream_u32(c + 12 + w0);
+    r[3] = SMEM ? lds_u32(c + 12 + w1) : ld_stream_u32(c + 12 + w1);
   }
 }
 
-// 32 codes of one block as the 8 signed-byte words the dp4a loop consumes,
-// W side: each code sits in the top bits of its byte, i.e. the byte is
-// code * 2^(8-m) (4-bit: 16q, 6-bit: 4q, 8-bit: q) -- exact in int8 and free
-// to form (a mask, no sign extension); the 2^(8-m) goes into the exact block
-// scale.  Word order: 4-bit word 2j = codes 8j, 8j+2, 8j+4, 8j+6 and word
-// 2j+1 the odd ones; 6-bit and 8-bit word j = codes 4j..4j+3.
-__device__ __forceinline__ void unpack_w(const uint32_t (&w)[8], int g, uint32_t (&u)[8]) {
-  if (g == 2) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      u[2 * j] = (w[j] << 4) & 0xF0F0F0F0u;
-      u[2 * j + 1] = w[j] & 0xF0F0F0F0u;
-    }
-  } else if (g == 1) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int pos = 24 * j, word = pos >> 5, off = pos & 31;
-      uint32_t v = w[word] >> off;
-      if (off > 8) v |= w[word + 1] << (32 - off);
-      u[j] = ((v << 2) & 0xFCu) | ((v << 4) & 0xFC00u) | ((v << 6) & 0xFC0000u) | ((v << 8) & 0xFC000000u);
-    }
+template <int G>
+__device__ __forceinline__ void widen_frag(const uint32_t (&r)[DecSeg<G>::kRaw], int t, uint32_t &b0, uint32_t &b1) {
+  if constexpr (G == 2) {
+    b0 = widen4(r[0]);
+    b1 = widen4(r[1]);
+  } else if constexpr (G == 0) {
+    b0 = r[0];
+    b1 = r[1];
   } else {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) u[j] = w[j];
+    const int sh = (3 * t & 3) * 8;
+    b0 = widen6(__funnelshift_r(r[0], r[1], sh));
+    b1 = widen6(__funnelshift_r(r[2], r[3], sh));
   }
 }
 
-// Activation side: sign-extended bytes in the same word order.
-__device__ __forceinline__ void stage_a_block(const uint8_t *c, int g, uint32_t (&wd)[8]) {
-  if (g == 2) {
-    const uint4 v = *reinterpret_cast<const uint4 *>(c);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+// Shared-memory image of one CTA: per segment g, the activations' packed
+// code rows (M rows at the source pitch), their scale rows, and the scale
+// rows of the CTA's 16 W rows (rows past N repeat row N-1).
+struct DecSmem {
+  int32_t a_code[3], a_scale[3], w_scale[3];
+  int32_t bytes;
+};
+
+__host__ __device__ inline DecSmem dec_smem_plan(const SmallArgs &a) {
+  DecSmem p{};
+  int32_t off = 0;
+  for (int g = 0; g < 3; ++g) {
+    p.a_code[g] = off;
+    off += a.nb[g] ? static_cast<int32_t>(a.M * a.a_cpitch[g]) : 0;
+  }
+  for (int g = 0; g < 3; ++g) {
+    p.a_scale[g] = off;
+    off += a.nb[g] ? static_cast<int32_t>(a.M * a.a_spitch[g]) : 0;
+  }
+  for (int g = 0; g < 3; ++g) {
+    p.w_scale[g] = off;
+    off += a.nb[g] ? static_cast<int32_t>(kDecRows * a.w_spitch[g]) : 0;
+  }
+  p.bytes = off;
+  return p;
+}
+
+// The blocks of segment G: warp w takes every 8th, kU per round with their
+// W loads in flight together.
+template <int G>
+__device__ __forceinline__ void dec_segment(const SmallArgs &a, const uint8_t *smem, const DecSmem &sp, int n0,
+                                            float (&acc)[2][4]) {
+  constexpr int MB = G == 0 ? 8 : (G == 1 ? 6 : 4);
+  constexpr int BB = kBlock * MB / 8;                 // bytes per packed block
+  constexpr int U = DecSeg<G>::kU, R = DecSeg<G>::kRaw;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int nbg = a.nb[G];
+  const uint8_t *wc = a.w_codes[G];
+  // this lane's rows: W rows n0 + 8j + gid (loads), activation rows gid, gid + 8
+  const uint8_t *wrow[2];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint32_t ev = 0, od = 0;
+  for (int j = 0; j < 2; ++j) wrow[j] = wc + static_cast<int64_t>(min(n0 + 8 * j + gid, a.N - 1)) * a.w_cpitch[G];
+  const bool a_lo = gid < a.M, a_hi = gid + 8 < a.M;   // rows past M read as zero
+  const uint8_t *arow_lo = smem + sp.a_code[G] + (a_lo ? gid : 0) * a.a_cpitch[G];
+  const uint8_t *arow_hi = smem + sp.a_code[G] + (a_hi ? gid + 8 : 0) * a.a_cpitch[G];
+  const uint8_t *asc = smem + sp.a_scale[G];
+  const uint8_t *wsc = smem + sp.w_scale[G];
+  for (int b0 = warp; b0 < nbg; b0 += kDecWarps * U) {
+    uint32_t raw[U][2][R];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int qe = static_cast<int>(w[j] << (28 - 8 * i)) >> 28;       // nibble 2i
-        const int qo = static_cast<int>(w[j] << (24 - 8 * i)) >> 28;       // nibble 2i+1
-        ev |= (static_cast<uint32_t>(qe) & 0xFFu) << (8 * i);
-        od |= (static_cast<uint32_t>(qo) & 0xFFu) << (8 * i);
+    for (int u = 0; u < U; ++u) {
+      const int bb = b0 + kDecWarps * u;
+      if (bb < nbg) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) load_frag_raw<G, false>(wrow[j] + bb * BB, tig, raw[u][j]);
       }
-      wd[2 * j] = ev;
-      wd[2 * j + 1] = od;
     }
-  } else if (g == 1) {
-    const uint2 x0 = *reinterpret_cast<const uint2 *>(c), x1 = *reinterpret_cast<const uint2 *>(c + 8),
-                x2 = *reinterpret_cast<const uint2 *>(c + 16);
-    const uint32_t w[6] = {x0.x, x0.y, x1.x, x1.y, x2.x, x2.y};
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      uint32_t o = 0;
+    for (int u = 0; u < U; ++u) {
+      const int bb = b0 + kDecWarps * u;
+      if (bb >= nbg) continue;
+      // A fragment: rows gid / gid+8, code groups tig / 4+tig
+      uint32_t ar[2][R];
+      load_frag_raw<G, true>(arow_lo + bb * BB, tig, ar[0]);
+      load_frag_raw<G, true>(arow_hi + bb * BB, tig, ar[1]);
+      uint4 af;
+      widen_frag<G>(ar[0], tig, af.x, af.z);
+      widen_frag<G>(ar[1], tig, af.y, af.w);
+      if (!a_lo) af.x = af.z = 0u;
+      if (!a_hi) af.y = af.w = 0u;
+      // bytes hold code * 2^(8-m): scale 2^(e-m+2) * 2^(m-8) = 2^(e-6)
+      const float fa_lo = pow2f(static_cast<int>(asc[(a_lo ? gid : 0) * a.a_spitch[G] + bb]) - 127 - 6);
+      const float fa_hi = pow2f(static_cast<int>(asc[(a_hi ? gid + 8 : 0) * a.a_spitch[G] + bb]) - 127 - 6);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int pos = 6 * (4 * j + i), word = pos >> 5, off = pos & 31;
-        uint32_t f = w[word] >> off;
-        if (off > 26) f |= w[word + 1] << (32 - off);
-        const int q = static_cast<int>(f << 26) >> 26;
-        o |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * i);
+      for (int j = 0; j < 2; ++j) {
+        uint32_t f0, f1;
+        widen_frag<G>(raw[u][j], tig, f0, f1);
+        int c[4];
+        mma_s8_16x8x32(af, f0, f1, c);
+        const float fw0 = pow2f(static_cast<int>(wsc[(8 * j + 2 * tig) * a.w_spitch[G] + bb]) - 127 - 6);
+        const float fw1 = pow2f(static_cast<int>(wsc[(8 * j + 2 * tig + 1) * a.w_spitch[G] + bb]) - 127 - 6);
+        acc[j][0] = fmaf(code_to_float(c[0]), fa_lo * fw0, acc[j][0]);
+        acc[j][1] = fmaf(code_to_float(c[1]), fa_lo * fw1, acc[j][1]);
+        acc[j][2] = fmaf(code_to_float(c[2]), fa_hi * fw0, acc[j][2]);
+        acc[j][3] = fmaf(code_to_float(c[3]), fa_hi * fw1, acc[j][3]);
       }
-      wd[j] = o;
     }
-  } else {
-    const uint4 v0 = *reinterpret_cast<const uint4 *>(c), v1 = *reinterpret_cast<const uint4 *>(c + 16);
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-    for (int j = 0; j < 8; ++j) wd[j] = w[j];
   }
 }
 
-// Activations in the dp4a word order, once per call, into the workspace:
-// codes [M][2][nb_total][16 B], then the block scales 2^(e-m+2) [M][NBP]
-// (float), NBP = nb_total rounded up to a multiple of 4 so every row starts
-// 16-byte aligned.  One thread per (activation row, block).
-__global__ void __launch_bounds__(128) gemm_small_prep_kernel(SmallArgs a, uint8_t *ws) {
-  const int NB = a.nb_total, NBP = (NB + 3) & ~3;
-  uint8_t *codes = ws;
-  float *fa = reinterpret_cast<float *>(ws + static_cast<int64_t>(a.M) * NB * 32);
-  const int it = blockIdx.x * blockDim.x + threadIdx.x;
-  if (it >= a.M * NB) return;
-  const int m = it / NB, b = it - m * NB;
-  int g, bb;
-  small_locate(a, b, g, bb);
-  const int mb = seg_bits(g);
-  uint32_t wd[8];
-  stage_a_block(a.a_codes[g] + m * a.a_cpitch[g] + static_cast<int64_t>(bb) * kBlock * mb / 8, g, wd);
-  const int e = static_cast<int>(a.a_scales[g][m * a.a_spitch[g] + bb]) - 127;
-  *reinterpret_cast<uint4 *>(codes + ((m * 2 + 0) * NB + b) * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-  *reinterpret_cast<uint4 *>(codes + ((m * 2 + 1) * NB + b) * 16) = make_uint4(wd[4], wd[5], wd[6], wd[7]);
-  fa[m * NBP + b] = pow2f(e - mb + 2);
-}
+constexpr long long kDecWaitLimit = 2000000000LL;    // cycles (~1 s)
 
-__device__ __forceinline__ void cp_async16_g(void *smem_dst, const void *gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
-               "l"(gsrc)
-               : "memory");
-}
-
-// MT: activation rows handled (>= M), R: W rows per warp, U: blocks per lane
-// whose loads are issued together, WPC: warps per CTA.
-template <int MT, int R, int U, int WPC>
-__global__ void __launch_bounds__(WPC * 32) gemm_small_kernel(SmallArgs a, const uint8_t *__restrict__ ws) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  const int CB = a.chunk_blocks, CBP = (CB + 3) & ~3;
-  uint8_t *sa = smem;                                               // [MT][2][CB][16 B]
-  float *sfa = reinterpret_cast<float *>(smem + static_cast<int64_t>(MT) * CB * 32);   // [MT][CBP]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = (blockIdx.x * WPC + warp) * R;
-  float acc[R][MT];
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int m = 0; m < MT; ++m) acc[r][m] = 0.f;
-
-  for (int c0 = 0; c0 < a.nb_total; c0 += CB) {
-    const int cb = min(CB, a.nb_total - c0);
-    __syncthreads();
-    {
-      // the chunk's activations, prepared once per call, copied in with every request in flight
-      const int NB = a.nb_total, NBP = (NB + 3) & ~3;
-      const float *gfa = reinterpret_cast<const float *>(ws + static_cast<int64_t>(a.M) * NB * 32);
-      for (int i = threadIdx.x; i < a.M * 2 * cb; i += blockDim.x) {
-        const int mh = i / cb, b = i - mh * cb;
-        cp_async16_g(sa + (mh * CB + b) * 16, ws + (static_cast<int64_t>(mh) * NB + c0 + b) * 16);
+// One CTA: W rows n0 .. n0+15.  Thread 0 bulk-copies the activations' code
+// and scale rows and the 16 W rows' scale rows into shared memory; the warps
+// then run the three segments and add their partial sums in warp order.
+__global__ void __launch_bounds__(kDecThreads) gemm_small_kernel(SmallArgs a, int *status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ __align__(8) uint64_t bar;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int n0 = blockIdx.x * kDecRows;
+  const DecSmem sp = dec_smem_plan(a);
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // copies: per segment, M activation code rows, M scale rows, 16 W scale rows
+    if (lane == 0) ptx::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(sp.bytes));
+    __syncwarp();
+    for (int g = 0; g < 3; ++g) {
+      if (!a.nb[g]) continue;
+      for (int r = lane; r < a.M; r += 32) {
+        ptx::bulk_load(smem + sp.a_code[g] + r * a.a_cpitch[g], a.a_codes[g] + r * a.a_cpitch[g],
+                       static_cast<uint32_t>(a.a_cpitch[g]), &bar);
+        ptx::bulk_load(smem + sp.a_scale[g] + r * a.a_spitch[g], a.a_scales[g] + r * a.a_spitch[g],
+                       static_cast<uint32_t>(a.a_spitch[g]), &bar);
       }
-      // 16-byte units of the scale rows (c0 is a multiple of 4; the last unit
-      // may carry padding entries, never read)
-      const int cbu = (cb + 3) / 4;
-      for (int i = threadIdx.x; i < a.M * cbu; i += blockDim.x) {
-        const int m = i / cbu, b = 4 * (i - m * cbu);
-        cp_async16_g(sfa + m * CBP + b, gfa + m * NBP + c0 + b);
-      }
-      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-    }
-    __syncthreads();
-    for (int b0 = lane; b0 < cb; b0 += 32 * U) {
-      uint32_t raw[U][R][8];
-      float fw[U][R];
-      int gs[U];
-      // issue every load of this round before using any of them
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int b = b0 + 32 * u;
-        gs[u] = -1;
-        if (b < cb) {
-          int g, bb;
-          small_locate(a, c0 + b, g, bb);
-          gs[u] = g;
-          const int mb = seg_bits(g);
-#pragma unroll
-          for (int r = 0; r < R; ++r) {
-            const int n = min(n0 + r, a.N - 1);     // rows past N load row N-1 and are never stored
-            load_w_raw(a.w_codes[g] + static_cast<int64_t>(n) * a.w_cpitch[g] + static_cast<int64_t>(bb) * kBlock * mb / 8,
-                       g, raw[u][r]);
-            // W bytes hold code * 2^(8-m): scale by 2^(e-m+2) * 2^(m-8) = 2^(e-6)
-            fw[u][r] = pow2f(static_cast<int>(__ldg(a.w_scales[g] + static_cast<int64_t>(n) * a.w_spitch[g] + bb)) - 127 - 6);
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int g = gs[u];
-        if (g < 0) continue;
-        const int b = b0 + 32 * u;
-        uint32_t uw[R][8];
-#pragma unroll
-        for (int r = 0; r < R; ++r) unpack_w(raw[u][r], g, uw[r]);
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-          if (m < a.M) {
-            const uint4 x0 = *reinterpret_cast<const uint4 *>(sa + ((m * 2 + 0) * CB + b) * 16);
-            const uint4 x1 = *reinterpret_cast<const uint4 *>(sa + ((m * 2 + 1) * CB + b) * 16);
-            const uint32_t av[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-            const float fa = sfa[m * CBP + b];
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-              int d = 0;
-#pragma unroll
-              for (int j = 0; j < 8; ++j) d = dp4a_ss(uw[r][j], av[j], d);
-              acc[r][m] = fmaf(code_to_float(d), fw[u][r] * fa, acc[r][m]);
-            }
-          }
-        }
-      }
+      for (int r = lane; r < kDecRows; r += 32)
+        ptx::bulk_load(smem + sp.w_scale[g] + r * a.w_spitch[g],
+                       a.w_scales[g] + static_cast<int64_t>(min(n0 + r, a.N - 1)) * a.w_spitch[g],
+                       static_cast<uint32_t>(a.w_spitch[g]), &bar);
     }
   }
-  // butterfly over the warp, then one lane per (row, activation) stores
+  float acc[2][4];
 #pragma unroll
-  for (int r = 0; r < R; ++r)
+  for (int j = 0; j < 2; ++j)
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      float v = acc[r][m];
+    for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
+  const bool landed = ptx::mbar_wait_cycles(&bar, 0, kDecWaitLimit);
+  if (__syncthreads_or(!landed)) {                    // uniform: every thread leaves together
+    if (threadIdx.x == 0) atomicExch(status, static_cast<int>(MXS_ERR_TIMEOUT));
+    return;     // the copies are the wait that expired: nothing else is in flight
+  }
+  dec_segment<0>(a, smem, sp, n0, acc);
+  dec_segment<1>(a, smem, sp, n0, acc);
+  dec_segment<2>(a, smem, sp, n0, acc);
+  // the warps' partial sums, added in warp order
+  __syncthreads();
+  float(*red)[16][kDecRows + 1] = reinterpret_cast<float(*)[16][kDecRows + 1]>(smem);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      acc[r][m] = v;
+  for (int j = 0; j < 2; ++j) {
+    red[warp][gid][8 * j + 2 * tig] = acc[j][0];
+    red[warp][gid][8 * j + 2 * tig + 1] = acc[j][1];
+    red[warp][gid + 8][8 * j + 2 * tig] = acc[j][2];
+    red[warp][gid + 8][8 * j + 2 * tig + 1] = acc[j][3];
+  }
+  __syncthreads();
+  {
+    const int m = threadIdx.x >> 4, r = threadIdx.x & 15, n = n0 + r;
+    if (m < a.M && n < a.N) {
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) sum += red[w][m][r];
+      a.Y[static_cast<int64_t>(m) * a.ldy + n] = __float2bfloat16_rn(sum);
     }
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int m = 0; m < MT; ++m)
-      if (lane == ((r * MT + m) & 31) && m < a.M && n0 + r < a.N)
-        a.Y[static_cast<int64_t>(m) * a.ldy + n0 + r] = __float2bfloat16_rn(acc[r][m]);
+  }
 }
 
-template <int MT, int R, int U, int WPC>
-static mxs_status launch_small(const SmallArgs &base, uint8_t *ws, cudaStream_t cs) {
-  SmallArgs a = base;
-  const int per_block_bytes = MT * (32 + 4);
-  // about 40 KB of staged activations per CTA (several CTAs per SM); chunks
-  // are multiples of 4 blocks so the int32/float slices copy in 16-byte units
-  a.chunk_blocks = std::max(32, std::min(a.nb_total, (40 * 1024) / per_block_bytes)) & ~3;
-  if (a.chunk_blocks > a.nb_total) a.chunk_blocks = a.nb_total;
-  const int smem = MT * (a.chunk_blocks * 32 + 4 * ((a.chunk_blocks + 3) & ~3));
-  if (!ensure_smem(gemm_small_kernel<MT, R, U, WPC>, 48 * 1024)) return MXS_ERR_CUDA;
-  gemm_small_prep_kernel<<<(a.M * a.nb_total + 127) / 128, 128, 0, cs>>>(a, ws);
-  const int rows_per_cta = WPC * R;
-  gemm_small_kernel<MT, R, U, WPC><<<(a.N + rows_per_cta - 1) / rows_per_cta, WPC * 32, smem, cs>>>(a, ws);
-  count_launch(2);
-  return cuda_status(cudaGetLastError());
+static int64_t small_smem_bytes(const SmallArgs &a) {
+  const int64_t red = static_cast<int64_t>(kDecWarps) * 16 * (kDecRows + 1) * 4;
+  return std::max<int64_t>(dec_smem_plan(a).bytes, red);
 }
 
-static size_t small_ws_bytes(int64_t M, int64_t nb_total) {
-  return static_cast<size_t>(M * nb_total * 32 + M * round_up(nb_total, 4) * 4 + 1024);
-}
+constexpr int64_t kDecSmemCap = 200 * 1024;
 
-static mxs_status gemm_small(const mxs_mxtensor *A, const mxs_mxtensor *W, void *Y, int64_t ldy, uint8_t *ws,
-                             cudaStream_t cs) {
+static SmallArgs small_args(const mxs_mxtensor *A, const mxs_mxtensor *W, void *Y, int64_t ldy) {
   SmallArgs a{};
   a.M = static_cast<int32_t>(A->rows);
   a.N = static_cast<int32_t>(W->rows);
@@ -1005,14 +969,27 @@ static mxs_status gemm_small(const mxs_mxtensor *A, const mxs_mxtensor *W, void 
   }
   a.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
   a.ldy = ldy;
-  if (a.M <= 1) return launch_small<1, 1, 4, 8>(a, ws, cs);
-  if (a.M <= 2) return launch_small<2, 1, 4, 8>(a, ws, cs);
-  if (a.M <= 4) return launch_small<4, 2, 2, 8>(a, ws, cs);
-  if (a.M <= 8) return launch_small<8, 4, 2, 4>(a, ws, cs);
-  return launch_small<16, 4, 1, 4>(a, ws, cs);
+  return a;
 }
 
-constexpr int64_t kSmallMaxM = 16;
+// True when the decode path takes this call (up to 16 activation rows whose
+// packed rows fit in shared memory).
+static bool small_fits(const mxs_mxtensor *A, const mxs_mxtensor *W) {
+  if (A->rows > kDecMaxM) return false;
+  return small_smem_bytes(small_args(A, W, nullptr, 0)) <= kDecSmemCap;
+}
+
+static mxs_status gemm_small(const mxs_mxtensor *A, const mxs_mxtensor *W, void *Y, int64_t ldy, cudaStream_t cs) {
+  const SmallArgs a = small_args(A, W, Y, ldy);
+  int *status = device_status_word();
+  if (!status) return MXS_ERR_CUDA;
+  const int smem = static_cast<int>(small_smem_bytes(a));
+  if (!ensure_smem(gemm_small_kernel, smem)) return MXS_ERR_CUDA;
+  gemm_small_kernel<<<(a.N + kDecRows - 1) / kDecRows, kDecThreads, smem, cs>>>(a, status);
+  count_launch();
+  return cuda_status(cudaGetLastError());
+}
+
 constexpr int64_t kPairMinM = 512;   // from here the 2-CTA pair kernel
 
 // ---------------------------------------------------------------- host side
@@ -1156,7 +1133,7 @@ extern "C" mxs_status mxs_gemm_workspace_bytes(const mxs_mxtensor *A, const mxs_
   if (!bytes) return MXS_ERR_ARG;
   mxs_status st = gemm_check(A, W);
   if (st != MXS_OK) return st;
-  *bytes = A->rows <= kSmallMaxM ? small_ws_bytes(A->rows, A->lay.K_pad / kBlock) : plan_workspace(A, W).total;
+  *bytes = small_fits(A, W) ? 0 : plan_workspace(A, W).total;   // the decode path needs none
   return MXS_OK;
 }
 
@@ -1175,11 +1152,7 @@ extern "C" mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, voi
     return cuda_status(cudaMemset2DAsync(Y, static_cast<size_t>(ldy) * 2, 0, static_cast<size_t>(N) * 2,
                                          static_cast<size_t>(M), cs));
   }
-  if (M <= kSmallMaxM) {
-    const size_t need = small_ws_bytes(M, A->lay.K_pad / kBlock);
-    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 1023u)) return MXS_ERR_WORKSPACE;
-    return gemm_small(A, W, Y, ldy, reinterpret_cast<uint8_t *>(ws), cs);
-  }
+  if (small_fits(A, W)) return gemm_small(A, W, Y, ldy, cs);
   const WsPlan p = plan_workspace(A, W);
   if (!ws || ws_bytes < p.total || (reinterpret_cast<uintptr_t>(ws) & 1023u)) return MXS_ERR_WORKSPACE;
   uint8_t *base = reinterpret_cast<uint8_t *>(ws);
@@ -1200,25 +1173,28 @@ extern "C" mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, voi
     op.sf = base + (o ? p.off_sfb : p.off_sfa);
     op.nrg = o ? p.nrg_b : p.nrg_a;
   }
-  sa.nb_total = 0;
-  for (int g = 0; g < 3; ++g) {
-    sa.nb[g] = static_cast<int32_t>(A->lay.seg[g].k_pad / kBlock);
-    sa.nb_total += sa.nb[g];
-  }
+  for (int g = 0; g < 3; ++g) sa.nb[g] = static_cast<int32_t>(A->lay.seg[g].k_pad / kBlock);
+  sa.nbw = sa.nb[0] + sa.nb[1];
+  sa.nb4p = p.nkg * 4;
   sa.k16 = p.k16;
   sa.k4 = p.k4;
-  sa.k6_off16 = A->lay.seg[0].k_pad;
   sa.nkg = p.nkg;
+  {
+    const int64_t sizes[4] = {M * sa.nbw, N * sa.nbw, static_cast<int64_t>(p.nrg_a) * 128 * sa.nb4p,
+                              static_cast<int64_t>(p.nrg_b) * 128 * sa.nb4p};
+    int64_t at = 0;
+    for (int r = 0; r < 4; ++r) {
+      if (at >= INT32_MAX) return MXS_ERR_SHAPE;
+      sa.start[r] = static_cast<int32_t>(at);
+      at += round_up(sizes[r], 32);
+    }
+    if (at >= INT32_MAX) return MXS_ERR_SHAPE;
+    sa.start[4] = static_cast<int32_t>(at);
+  }
   int dev = 0, nsm = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  int64_t stage_tiles = 0;
-  for (int g = 0; g < 3; ++g) {
-    if (sa.nb[g] == 0) continue;
-    const int64_t bt = g == 2 ? (p.nkg * 4 + kStageBlocks - 1) / kStageBlocks : (sa.nb[g] + kStageBlocks - 1) / kStageBlocks;
-    stage_tiles += (g == 2 ? (p.nrg_a + p.nrg_b) : ((M + kStageRows - 1) / kStageRows + (N + kStageRows - 1) / kStageRows)) * bt;
-  }
-  const int sgrid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(stage_tiles, static_cast<int64_t>(nsm) * 8)));
+  const int sgrid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((sa.start[4] + 255) / 256, static_cast<int64_t>(nsm) * 8)));
   gemm_stage_kernel<<<sgrid, 256, 0, cs>>>(sa);
   count_launch();
 

@@ -90,6 +90,10 @@ def test_gemm_argument_checks(capi):
     need = ctypes.c_size_t(0)
     assert capi._lib.mxs_gemm_workspace_bytes(ctypes.byref(A), ctypes.byref(W), ctypes.byref(need)) == 0
     assert need.value >= 100 * 96 * 2 + 300 * 96 * 2 + 100 * 160 + 300 * 160
+    # up to 16 activation rows: the decode path stages in shared memory, no workspace
+    A8 = _fake_tensor(capi, 8, lay)
+    assert capi._lib.mxs_gemm_workspace_bytes(ctypes.byref(A8), ctypes.byref(W), ctypes.byref(need)) == 0
+    assert need.value == 0
     # different layouts -> MXS_ERR_SHAPE, no launch
     lay2 = capi.mxs_layout_make(256, (32, 32, 192))
     W2 = _fake_tensor(capi, 300, lay2)

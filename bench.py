@@ -76,7 +76,7 @@ def gemm_roofline_s(M, N, counts, pk):
 class ClockSampler:
     """NVML samples of SM clock and throttle reasons while running."""
 
-    def __init__(self, index, period=0.005):
+    def __init__(self, index, period=0.001):
         self.index, self.period = index, period
         self.samples, self.reasons = [], set()
         self.max_mhz = None
@@ -163,36 +163,37 @@ class Path:
             "mxs_sensitivity": ("GB/s", (T_CAL + N_OUT) * K_IN * 2),
             "mxs_allocate": ("GB/s", K_IN * 8 + K_IN * 4),
             "mxs_quantize_weight": ("GB/s", layout_bytes(N_OUT, self.counts, 2)),
-            "mxs_quantize_kv": ("GB/s", layout_bytes(KV_SHAPE[0] * KV_SHAPE[1], (0, 0, KV_SHAPE[2]), 2)),
+            "mxs_quantize_kv0": ("GB/s", layout_bytes(KV_SHAPE[0] * KV_SHAPE[1], (0, 0, KV_SHAPE[2]), 2)),
+            "mxs_quantize_kv1": ("GB/s", layout_bytes(KV_SHAPE[0] * KV_SHAPE[1], (0, 0, KV_SHAPE[2]), 2)),
         }
         for M in M_LIST:
             self.work[f"mxs_quantize_act_M{M}"] = ("GB/s", layout_bytes(M, self.counts, 2))
             self.work[f"mxs_gemm_M{M}"] = ("TFLOP/s", 2 * M * N_OUT * K_IN)
         self.gemm_flops = sum(2 * M * N_OUT * K_IN for M in M_LIST)
 
-    def step(self, rec=None):
-        c, t = self.c, self.torch
+    def calls(self):
+        """The step as (name, call) pairs in order; each call is one C-ABI entry point."""
+        c = self.c
 
-        def timed(name, fn):
-            if rec is None:
-                return fn()
-            s, e = t.cuda.Event(enable_timing=True), t.cuda.Event(enable_timing=True)
-            s.record()
-            r = fn()
-            e.record()
-            rec.setdefault(name, []).append((s, e))
-            return r
-        timed("mxs_sensitivity", lambda: c.mxs_sensitivity(self.X, self.W, workspace=self.sens_ws,
-                                                            out=(self.H, self.E, self.s)))
-        _, counts = timed("mxs_allocate", lambda: c.mxs_allocate(
-            [self.s], [N_OUT], mode="budget", budget=BUDGET, perms=[self.perm], workspace=self.alloc_ws))
-        assert counts[0] == self.counts
-        timed("mxs_quantize_weight", lambda: c.mxs_quantize_weight(self.W, self.Wq))
+        def alloc():
+            _, counts = c.mxs_allocate([self.s], [N_OUT], mode="budget", budget=BUDGET, perms=[self.perm],
+                                       workspace=self.alloc_ws)
+            assert counts[0] == self.counts
+        out = [("mxs_sensitivity", lambda: c.mxs_sensitivity(self.X, self.W, workspace=self.sens_ws,
+                                                               out=(self.H, self.E, self.s))),
+               ("mxs_allocate", alloc),
+               ("mxs_quantize_weight", lambda: c.mxs_quantize_weight(self.W, self.Wq))]
         for M in M_LIST:
-            timed(f"mxs_quantize_act_M{M}", lambda M=M: c.mxs_quantize_act(self.A[M], self.Aq[M]))
-            timed(f"mxs_gemm_M{M}", lambda M=M: c.mxs_gemm(self.Aq[M], self.Wq, Y=self.Y[M], workspace=self.gemm_ws))
+            out.append((f"mxs_quantize_act_M{M}", lambda M=M: c.mxs_quantize_act(self.A[M], self.Aq[M])))
+            out.append((f"mxs_gemm_M{M}", lambda M=M: c.mxs_gemm(self.Aq[M], self.Wq, Y=self.Y[M],
+                                                                 workspace=self.gemm_ws)))
         for i in range(2):
-            timed("mxs_quantize_kv", lambda i=i: c.mxs_quantize_act(self.KV[i], self.KVq[i]))
+            out.append((f"mxs_quantize_kv{i}", lambda i=i: c.mxs_quantize_act(self.KV[i], self.KVq[i])))
+        return out
+
+    def step(self):
+        for _, fn in self.calls():
+            fn()
 
 
 def traffic_from_profile(pk_name: str):
@@ -202,7 +203,7 @@ def traffic_from_profile(pk_name: str):
         text = open(prof).read()
     except OSError:
         return None
-    m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m = re.search(r"dram_bytes_per_call:\s*([0-9.eE+]+)", text)
     h = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
     if not m or not h:
         return None
@@ -232,25 +233,61 @@ def run_gpu(args, rank, world, local_rank):
             dist.barrier()
         torch.cuda.synchronize()
 
+    # The step is captured once as one CUDA graph (its kernels back to back,
+    # no host launch gaps) and replayed once per timed step.  Every call is
+    # also captured alone; a second pass replays those in step order with
+    # CUDA events between them to time each call.
+    calls = path.calls()
+    cap = torch.cuda.Stream()
+    launches0 = c.mxs_launch_count()
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=cap):
+        for _, fn in calls:
+            fn()
+    launches_per_step = c.mxs_launch_count() - launches0
+    graphs = []
+    for name, fn in calls:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            fn()
+        graphs.append((name, g))
+    for _ in range(3):
+        path.flush.zero_()
+        g_step.replay()
+        path.flush.zero_()
+        for _, g in graphs:
+            g.replay()
+    c.mxs_sync()
+
     rec = {}
     step_ev = []
+    call_steps = min(args.steps, 50)
     barrier()
-    launches0 = c.mxs_launch_count()
     with ClockSampler(local_rank) as clocks:
         t0 = time.perf_counter()
         for _ in range(args.steps):
             path.flush.zero_()                      # L2 flush, outside the step events
             s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             s.record()
-            path.step(rec)
+            g_step.replay()
             e.record()
             step_ev.append((s, e))
         barrier()
         wall = time.perf_counter() - t0
-    launches = c.mxs_launch_count() - launches0
+        for _ in range(call_steps):
+            path.flush.zero_()
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)]
+            evs[0].record()
+            for i, (name, g) in enumerate(graphs):
+                g.replay()
+                evs[i + 1].record()
+                rec.setdefault(name, []).append((evs[i], evs[i + 1]))
+        barrier()
+    launches = launches_per_step * args.steps
     c.mxs_sync()
     step_ms = [s.elapsed_time(e) for s, e in step_ev]
     total_s = sum(step_ms) * 1e-3
+    call_step_ms = sum(s.elapsed_time(e) for evs in rec.values() for s, e in evs) / call_steps
     if world > 1:
         tt = torch.tensor([total_s], device=dev, dtype=torch.float64)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
@@ -263,7 +300,7 @@ def run_gpu(args, rank, world, local_rank):
         per = sum(ms) / len(ms) * 1e-3
         unit, work = path.work[name]
         ach = work / per / (1e12 if unit == "TFLOP/s" else 1e9)
-        kd = {"us": per * 1e6, "achieved": ach, "unit": unit, "share": sum(ms) / sum(step_ms)}
+        kd = {"us": per * 1e6, "achieved": ach, "unit": unit, "share": per * 1e3 / call_step_ms}
         if unit == "GB/s":
             kd["frac_hbm"] = ach / pk["hbm_gbs"]
             kd["frac_nominal_8tbs"] = ach / 8000.0
@@ -276,9 +313,9 @@ def run_gpu(args, rank, world, local_rank):
     # the dominant kernel: the prefill GEMM
     g = kernels["mxs_gemm_M2048"]
     rt = g["roofline_us"] * 1e-6
-    roof = {"kernel": "mxs_gemm M=2048 (stage + tcgen05 kernels)", "bound": "tensor",
+    roof = {"kernel": "mxs_gemm M=2048 (one call: gemm_stage_kernel + gemm_tc2_kernel)", "bound": "tensor",
             "achieved": g["achieved"], "peak": 2 * 2048 * N_OUT * K_IN / rt / 1e12, "unit": "TFLOP/s",
-            "frac": g["frac"], "traffic": traffic_from_profile("gemm_tc_attn_prefill_M2048.md"),
+            "frac": g["frac"], "traffic": traffic_from_profile("gemm_attn_prefill_M2048.md"),
             "peak_basis": f"4-bit segment at 2x measured bf16 ({pk['fp8_tflops']:.0f} TFLOP/s, no measured fp8), "
                           f"6/8-bit at measured bf16 ({pk['bf16_tflops']:.0f}); of {pk['source']}"}
 
@@ -289,7 +326,10 @@ def run_gpu(args, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "mxint4/6/8 codes; e4m3+bf16 MMA, f32 acc",
         "data": "synthetic (seeded; shapes and outlier structure of the workload)",
         "config": {"workload": WORKLOAD, "counts_n8_n6_n4": list(path.counts), "l2": "flushed between steps "
-                   "(512 MB write outside the step events)", "parallelism": f"replicas x{world} (no data-path collective)"},
+                   "(512 MB write outside the step events)", "parallelism": f"replicas x{world} (no data-path collective)",
+                   "timing": "step = one CUDA graph of all C-ABI calls, replayed per step between CUDA events; "
+                             "kernels{} from a second pass of per-call graphs in step order with events between",
+                   "launches_per_step": launches_per_step},
         "roofline": roof, "kernels": kernels, "e2e": e2e, "gpu_launches": launches,
         "clocks": clocks.summary(), "wall_s_timed_region": wall,
     }
@@ -426,7 +466,7 @@ def cpu_baseline():
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -157,6 +157,25 @@ mxs_status mxs_sensitivity(const void *X, mxs_dtype xt, int64_t T, int64_t K, in
                            double *H, double *E, double *s,
                            void *ws, size_t ws_bytes, void *stream);
 
+/* mxs_sensitivity_noalloc -- mxs_sensitivity without a caller workspace, for
+ * callers that cannot allocate device memory (code inside stream capture,
+ * runtimes without an allocator).  The pages have no counterpart: this is a
+ * library convenience around the same computation.
+ *   The chunk partials live in one library-owned device array of 16 MiB per
+ *   device (MXS_NOALLOC_SCRATCH_BYTES); shapes whose workspace
+ *   (mxs_sensitivity_workspace_bytes) exceeds it return MXS_ERR_WORKSPACE
+ *   before any launch.  No memory is allocated.
+ *   The first call on a device looks up the array's address (with that
+ *   device current); make one call on each device before any stream capture.
+ *   Every call shares the one array: calls that overlap on the GPU (other
+ *   streams, other host threads) race on it and must be serialised by the
+ *   caller.  Nothing in the array needs to start at zero.
+ *   Results are bit-identical to mxs_sensitivity. */
+#define MXS_NOALLOC_SCRATCH_BYTES (16u << 20)
+mxs_status mxs_sensitivity_noalloc(const void *X, mxs_dtype xt, int64_t T, int64_t K, int64_t ldx,
+                                   const void *W, mxs_dtype wt, int64_t N, int64_t ldw,
+                                   double *H, double *E, double *s, void *stream);
+
 /* ---------------------------------------------------------------------------
  * mxs_allocate -- 4/6/8-bit widths for n_layers layers and their column
  * permutations.  [TS §2.3: sort columns by sensitivity; the top block gets 8

@@ -76,6 +76,7 @@ _sig("mxs_layout_make", [_I64, _P, _P, ctypes.POINTER(LayoutC)])
 _sig("mxs_mxtensor_bytes", [_I64, ctypes.POINTER(LayoutC), _P, _P, _P, _P])
 _sig("mxs_sensitivity_workspace_bytes", [_I64, _I64, _I64, ctypes.POINTER(_SZ)])
 _sig("mxs_sensitivity", [_P, _ST, _I64, _I64, _I64, _P, _ST, _I64, _I64, _P, _P, _P, _P, _SZ, _P])
+_sig("mxs_sensitivity_noalloc", [_P, _ST, _I64, _I64, _I64, _P, _ST, _I64, _I64, _P, _P, _P, _P])
 _sig("mxs_allocate_workspace_bytes", [ctypes.c_int32, _P, ctypes.POINTER(_SZ)])
 _sig("mxs_allocate", [ctypes.c_int32, _P, _P, _P, _P, ctypes.POINTER(BudgetC), _P, _P, _P, _SZ, _P])
 _sig("mxs_quantize_weight", [_P, _ST, _I64, _I64, ctypes.POINTER(MXTensorC), _P])
@@ -85,7 +86,8 @@ _sig("mxs_gemm_workspace_bytes", [ctypes.POINTER(MXTensorC), ctypes.POINTER(MXTe
 _sig("mxs_gemm", [ctypes.POINTER(MXTensorC), ctypes.POINTER(MXTensorC), _P, _I64, _P, _SZ, _P])
 
 EXPORTS = ["mxs_status_str", "mxs_launch_count", "mxs_sync", "mxs_layout_make", "mxs_mxtensor_bytes",
-           "mxs_sensitivity_workspace_bytes", "mxs_sensitivity", "mxs_allocate_workspace_bytes",
+           "mxs_sensitivity_workspace_bytes", "mxs_sensitivity", "mxs_sensitivity_noalloc",
+           "mxs_allocate_workspace_bytes",
            "mxs_allocate", "mxs_quantize_weight", "mxs_quantize_act", "mxs_dequantize",
            "mxs_gemm_workspace_bytes", "mxs_gemm"]
 
@@ -221,6 +223,22 @@ def mxs_sensitivity(X: torch.Tensor, W: torch.Tensor, stream=None, workspace: Op
     _check(_lib.mxs_sensitivity(X.data_ptr(), _dt(X), T, K, _rowmajor(X), W.data_ptr(), _dt(W), N,
                                 _rowmajor(W), H.data_ptr(), E.data_ptr(), s.data_ptr(),
                                 _aligned_ptr(ws), need.value, _stream(stream)), "mxs_sensitivity")
+    return H, E, s
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def mxs_sensitivity_noalloc(X: torch.Tensor, W: torch.Tensor, out, stream=None):
+    """mxs_sensitivity with the library's fixed device scratch instead of a
+    workspace; `out` = (H, E, s) caller-allocated fp64 tensors of K."""
+    T, K = X.shape
+    N, K2 = W.shape
+    assert K == K2
+    H, E, s = out
+    _check(_lib.mxs_sensitivity_noalloc(X.data_ptr(), _dt(X), T, K, _rowmajor(X), W.data_ptr(), _dt(W), N,
+                                        _rowmajor(W), H.data_ptr(), E.data_ptr(), s.data_ptr(), _stream(stream)),
+           "mxs_sensitivity_noalloc")
     return H, E, s
 
 

@@ -25,6 +25,7 @@
 // that stages the chunk partials of 32 columns in shared memory, adds them in
 // chunk order and forms H, E and s.
 #include <algorithm>
+#include <mutex>
 
 #include "mxs_internal.cuh"
 #include "mxs_ptx.cuh"
@@ -405,4 +406,51 @@ extern "C" mxs_status mxs_sensitivity(const void *X, mxs_dtype xt, int64_t T, in
   sens_finalize_kernel<<<static_cast<unsigned>((K + kFinCols - 1) / kFinCols), kFinThreads, 0, cs>>>(a, H, E, s);
   count_launch(2);
   return cuda_status(cudaGetLastError());
+}
+
+// ------------------------------------------------------- no-allocation entry
+//
+// Some callers cannot call cudaMalloc at all: code running inside CUDA stream
+// capture (allocation is not a capturable stream operation), runtimes that
+// hand a library no allocator, and latency-critical paths that must not take
+// the allocator's locks.  For them the chunk partials live in one file-scope
+// device array of fixed size instead of a caller-provided workspace.
+namespace mxs {
+
+constexpr size_t kNoAllocScratchBytes = MXS_NOALLOC_SCRATCH_BYTES;   // 16 MiB: 2 Mi chunk partials
+__device__ __align__(256) uint8_t g_sens_scratch[kNoAllocScratchBytes];
+
+// Address of the scratch array on the current device, looked up once per
+// device (with that device current) and kept.
+static mxs_status sens_scratch(void **ptr) {
+  static void *addr[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MXS_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return MXS_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_sens_scratch) != cudaSuccess || !p) return MXS_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  return MXS_OK;
+}
+
+}  // namespace mxs
+
+extern "C" mxs_status mxs_sensitivity_noalloc(const void *X, mxs_dtype xt, int64_t T, int64_t K, int64_t ldx,
+                                              const void *W, mxs_dtype wt, int64_t N, int64_t ldw,
+                                              double *H, double *E, double *s, void *stream) {
+  size_t need = 0;
+  mxs_status st = mxs_sensitivity_workspace_bytes(T, N, K, &need);
+  if (st != MXS_OK) return st;
+  if (need > kNoAllocScratchBytes) return MXS_ERR_WORKSPACE;   // shape needs more than the fixed scratch
+  void *scratch = nullptr;
+  if ((st = check_device()) != MXS_OK) return st;
+  if ((st = sens_scratch(&scratch)) != MXS_OK) return st;
+  // every partial the finalize pass reads is written earlier in the same
+  // call, so nothing in the scratch has to start at zero
+  return mxs_sensitivity(X, xt, T, K, ldx, W, wt, N, ldw, H, E, s, scratch, kNoAllocScratchBytes, stream);
 }

@@ -463,6 +463,63 @@ def cpu_baseline():
             "parts_s": {k: round(v, 4) for k, v in parts.items()}}
 
 
+def run_mixed_overhead(args):
+    """Time mxs_gemm on one weight under three layouts -- uniform MXINT4, the
+    32 fixed 8-bit columns alone (budget 4.03125 bits) and the 4.5-bit budget
+    -- to measure what the wider blocks cost (the pages estimate ~3% at
+    ~4.03 bits).  CUDA-graph replays of one call, L2 flushed before each,
+    CUDA events around each replay."""
+    import torch
+    from mx_microscaling_mixed_b200 import build
+    build.build()
+    from mx_microscaling_mixed_b200 import capi as c, inputs
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    reps = max(10, min(args.steps, 100))
+    out = {"metric": "mxs_gemm time by layout", "unit": "us", "reps": reps, "shapes": []}
+    for (N, K) in ((4096, 4096), (14336, 4096)):
+        W = inputs.attn_weight(dev, SEED, N, K)
+        X = inputs.gaussian_acts(dev, SEED + 1, T_CAL, K)
+        _, _, s = c.mxs_sensitivity(X, W)
+        layouts = {"uniform4": ((0, 0, K), torch.arange(K, dtype=torch.int32, device=dev))}
+        for name, budget in (("b4.03125", (129, 32)), ("b4.5", (9, 2))):
+            perms, counts = c.mxs_allocate([s], [N], mode="budget", budget=budget)
+            layouts[name] = (counts[0], perms[0])
+        row = {"N": N, "K": K, "counts": {k: list(v[0]) for k, v in layouts.items()}, "us": {}}
+        for M in M_LIST:
+            A = inputs.gaussian_acts(dev, SEED + 2 + M, M, K)
+            for name, (counts, perm) in layouts.items():
+                lay = c.mxs_layout_make(K, counts, perm)
+                Wq, Aq = c.mxtensor_empty(N, lay, dev), c.mxtensor_empty(M, lay, dev)
+                c.mxs_quantize_weight(W, Wq)
+                c.mxs_quantize_act(A, Aq)
+                ws = torch.empty(c.mxs_gemm_workspace_bytes(Aq, Wq) + 1024, dtype=torch.uint8, device=dev)
+                Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+                call = lambda: c.mxs_gemm(Aq, Wq, Y=Y, workspace=ws)
+                for _ in range(3):
+                    call()
+                g = torch.cuda.CUDAGraph()
+                cap = torch.cuda.Stream()
+                with torch.cuda.graph(g, stream=cap):
+                    call()
+                ms = []
+                for _ in range(reps):
+                    flush.zero_()
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    g.replay()
+                    e1.record()
+                    ms.append((e0, e1))
+                torch.cuda.synchronize()
+                row["us"][f"M{M}/{name}"] = statistics.median(a.elapsed_time(b) for a, b in ms) * 1e3
+            base = row["us"][f"M{M}/uniform4"]
+            for name in ("b4.03125", "b4.5"):
+                row["us"][f"M{M}/{name}/overhead"] = row["us"][f"M{M}/{name}"] / base - 1.0
+        out["shapes"].append(row)
+    c.mxs_sync()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -470,12 +527,17 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mixed-overhead", action="store_true",
+                    help="time mxs_gemm under uniform-4-bit vs mixed layouts and exit")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.gpus == 1 else 1)))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.mixed_overhead:
+        print(json.dumps(run_mixed_overhead(args)), flush=True)
+        return
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args, world)), flush=True)

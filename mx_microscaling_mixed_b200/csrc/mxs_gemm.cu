@@ -559,9 +559,20 @@ __device__ __forceinline__ float code_to_float(int q) {
   return __uint_as_float(static_cast<uint32_t>(0x4B400000 + q)) - 12582912.0f;
 }
 
-// 6/8-bit block -> 32 exact bf16 values q * 2^(e-m+2), four 16-byte stores.
+// 6/8-bit block -> 32 exact bf16 values q * 2^(e-m+2), as 16 packed words.
+__device__ __forceinline__ void wide6_words_fast(const uint32_t (&w)[6], uint8_t sbyte, uint32_t (&pk)[16]);
+
 template <int M>
-__device__ __forceinline__ void stage_wide_block(const uint8_t *c, uint8_t sbyte, __nv_bfloat16 *dst) {
+__device__ __forceinline__ void wide_block_words(const uint8_t *c, uint8_t sbyte, uint32_t (&pk)[16]) {
+  if constexpr (M == 6) {
+    if (sbyte >= 13 && sbyte <= 251) {                     // 192 * step and the results are normal bf16
+      const uint2 a = *reinterpret_cast<const uint2 *>(c), b = *reinterpret_cast<const uint2 *>(c + 8),
+                  d = *reinterpret_cast<const uint2 *>(c + 16);
+      const uint32_t w[6] = {a.x, a.y, b.x, b.y, d.x, d.y};
+      wide6_words_fast(w, sbyte, pk);
+      return;
+    }
+  }
   const float step = pow2f(static_cast<int>(sbyte) - 127 - M + 2);
   int q[kBlock];
   if constexpr (M == 8) {
@@ -581,12 +592,46 @@ __device__ __forceinline__ void stage_wide_block(const uint8_t *c, uint8_t sbyte
       q[t] = static_cast<int>(f << 26) >> 26;    // sign-extend the 6-bit field
     }
   }
-  uint32_t pk[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     __nv_bfloat162 h = __floats2bfloat162_rn(code_to_float(q[2 * i]) * step, code_to_float(q[2 * i + 1]) * step);
     pk[i] = *reinterpret_cast<uint32_t *>(&h);
   }
+}
+
+// 6-bit block -> 32 exact bf16 values q * 2^(e-4) as 16 packed words, two
+// codes per instruction: a code's 16-bit lane is made the bf16 of 192 + q
+// (0x4320 + (f ^ 0x20) for the 6-bit field f; 192 + q stays in [128, 256),
+// where bf16 integers are exact), then one packed fma (192+q)*s - 192*s
+// gives q*s exactly (q*s is a bf16: <= 5 significant bits, exponent in range).
+__device__ __forceinline__ void wide6_words_fast(const uint32_t (&w)[6], uint8_t sbyte, uint32_t (&pk)[16]) {
+  const int e = static_cast<int>(sbyte) - 127 - 4;    // step 2^(e-m+2), m = 6
+  // the step is >= 2^-131; below 2^-126 bf16 has no normal encoding: use the fp32 path
+  const float step = pow2f(e);
+  const __nv_bfloat162 s2 = __floats2bfloat162_rn(step, step);
+  const __nv_bfloat162 c2 = __floats2bfloat162_rn(-192.f * step, -192.f * step);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    uint32_t f[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int pos = 6 * (2 * i + h), word = pos >> 5, off = pos & 31;
+      uint32_t v = w[word] >> off;
+      if (off > 26) v |= w[word + 1] << (32 - off);
+      f[h] = v & 0x3Fu;
+    }
+    const uint32_t x = (f[0] | (f[1] << 16)) ^ 0x00200020u;
+    const uint32_t b = x + 0x43204320u;
+    const __nv_bfloat162 r = __hfma2(*reinterpret_cast<const __nv_bfloat162 *>(&b), s2, c2);
+    pk[i] = *reinterpret_cast<const uint32_t *>(&r);
+  }
+}
+
+// 6/8-bit block -> 32 exact bf16 values, four 16-byte stores.
+template <int M>
+__device__ __forceinline__ void stage_wide_block(const uint8_t *c, uint8_t sbyte, __nv_bfloat16 *dst) {
+  uint32_t pk[16];
+  wide_block_words<M>(c, sbyte, pk);
   uint4 *o = reinterpret_cast<uint4 *>(dst);
   o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
   o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
@@ -989,6 +1034,7 @@ static mxs_status gemm_small(const mxs_mxtensor *A, const mxs_mxtensor *W, void 
   count_launch();
   return cuda_status(cudaGetLastError());
 }
+
 
 constexpr int64_t kPairMinM = 512;   // from here the 2-CTA pair kernel
 

@@ -106,6 +106,22 @@ def test_selector_weights_are_exact(c):
     assert np.array_equal(Y, Yref)
 
 
+def test_selector_extreme_scales_exact(c):
+    """Rows of A scaled across the exponent range (block scale bytes from ~10
+    to ~252) pass the staging conversions -- including the packed bf16 path
+    for 6-bit blocks and its fp32 fallback at the range ends -- exactly."""
+    K, M = 256, 24
+    A = inputs.random_matrix(M, K, device="cuda", seed=4, dtype=torch.float32, outlier_frac=0.0)
+    ks = [-118, -117, -116, -115, -114, -100, -60, -1, 0, 1, 60, 100, 118, 119, 120, 121, 122, 122,
+          -113, 30, -30, 90, -90, 2]
+    A = (A * torch.tensor([2.0 ** k for k in ks], device="cuda")[:, None]).to(torch.bfloat16)
+    W = torch.zeros(64, K, dtype=torch.bfloat16, device="cuda")
+    sel = np.random.default_rng(5).choice(K, 64, replace=False)
+    W[np.arange(64), sel] = 1.0
+    Y, Yref = _run(c, A, W, (32, 64, 160), seed=6)
+    assert np.array_equal(Y, Yref)
+
+
 def test_zero_k_segments_and_strided_output(c):
     K = 128
     A = inputs.random_matrix(70, K, device="cuda", seed=5, dtype=torch.bfloat16)

@@ -53,6 +53,12 @@ constexpr int kSfbBytes = (kBN / 128) * kSfChunk;
 constexpr int kTmemCols = 512;
 constexpr int kSfaCol = kBN;       // tensor-memory columns of the scale copies
 constexpr int kSfbCol = kBN + 4;
+// The scale copies rotate through kSfSlots slots of kSfSlotCols columns, so a
+// stage's copies never overwrite the scales the previous stage's MMAs still
+// read: the copy does not wait for those MMAs (256 + 4 x 12 = 304 of 512
+// columns).
+constexpr int kSfSlots = 4;
+constexpr int kSfSlotCols = 12;
 constexpr int kGemmThreads = 192;
 constexpr long long kWaitLimit = 4000000000LL;   // cycles (~2 s): then give up
 
@@ -172,15 +178,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         } else {
           const uint32_t sfa_s = ptx::smem_addr(smem + GemmSmem::sfa_off + s * kSfaBytes);
           const uint32_t sfb_s = ptx::smem_addr(smem + GemmSmem::sfb_off + s * kSfbBytes);
-          ptx::copy_sf_to_tmem(tsfa, ptx::desc_sf(sfa_s));
+          const uint32_t slot = kSfSlotCols * static_cast<uint32_t>(it % kSfSlots);
+          ptx::copy_sf_to_tmem(tsfa + slot, ptx::desc_sf(sfa_s));
 #pragma unroll
-          for (int c = 0; c < kBN / 128; ++c) ptx::copy_sf_to_tmem(tsfb + 4 * c, ptx::desc_sf(sfb_s + kSfChunk * c));
+          for (int c = 0; c < kBN / 128; ++c)
+            ptx::copy_sf_to_tmem(tsfb + slot + 4 * c, ptx::desc_sf(sfb_s + kSfChunk * c));
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const uint32_t idesc = kIdescMxf8 | (static_cast<uint32_t>(k) << 4) | (static_cast<uint32_t>(k) << 29);
             ptx::mma_mxf8(tmem, ptx::desc_sw128(a_base + 32 * k), ptx::desc_sw128(b_base + 32 * k), idesc,
-                          (it > 0 || k > 0) ? 1u : 0u, tsfa | (static_cast<uint32_t>(k) << 30),
-                          tsfb | (static_cast<uint32_t>(k) << 30));
+                          (it > 0 || k > 0) ? 1u : 0u, (tsfa + slot) | (static_cast<uint32_t>(k) << 30),
+                          (tsfb + slot) | (static_cast<uint32_t>(k) << 30));
           }
         }
         ptx::mma_commit(&empty[s]);
@@ -319,27 +327,33 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 }  // namespace ptx
 
-constexpr int kP2Stages = 6;
-constexpr int kP2Rows = 128;                       // rows of A and of B per CTA per stage
+constexpr int kP2Stages = 3;
+constexpr int kP2Sub = 2;                          // K slices per stage: 8 MMAs per barrier round
+constexpr int kP2Rows = 128;                       // rows of A per CTA per stage
+constexpr int kP2N = 240;                          // output columns per pair tile (W rows)
+constexpr int kP2BRows = kP2N / 2;                 // rows of B per CTA per stage
+constexpr int kP2AccCols = kP2N;                   // one accumulator buffer; two buffers at columns 0 and 240
+constexpr int kP2SfCol = 2 * kP2AccCols;           // scale slots from column 480: 2 x 12 columns
+constexpr int kP2SfSlots = 2;
 constexpr int kP2TileBytes = kP2Rows * kSliceBytes;
 constexpr int kP2SfaBytes = kSfChunk;              // own 128 A rows x 4 blocks
 constexpr int kP2SfbBytes = 2 * kSfChunk;          // the pair's 256 N rows x 4 blocks
 constexpr int kP2EpiWarps = 8;
 constexpr int kP2Threads = (2 + kP2EpiWarps) * 32;
-// cta_group::2, M = 256, N = 256
-constexpr uint32_t kIdesc2Bf16 = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(256 >> 3) << 17) |
+// cta_group::2, M = 256, N = 240
+constexpr uint32_t kIdesc2Bf16 = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kP2N >> 3) << 17) |
                                  (static_cast<uint32_t>(256 >> 4) << 24);
-constexpr uint32_t kIdesc2Mxf8 = (static_cast<uint32_t>(256 >> 3) << 17) | (1u << 23) |
+constexpr uint32_t kIdesc2Mxf8 = (static_cast<uint32_t>(kP2N >> 3) << 17) | (1u << 23) |
                                  (static_cast<uint32_t>(256 >> 4) << 24);
 
 struct P2Smem {
   static constexpr int a_off = 0;
-  static constexpr int b_off = a_off + kP2Stages * kP2TileBytes;
-  static constexpr int sfa_off = b_off + kP2Stages * kP2TileBytes;
-  static constexpr int sfb_off = sfa_off + kP2Stages * kP2SfaBytes;
-  static constexpr int bar_off = sfb_off + kP2Stages * kP2SfbBytes;
-  // full[S], empty[S], acc_full, acc_empty, tmem slot, abort flag
-  static constexpr int bytes = bar_off + (2 * kP2Stages + 2) * 8 + 16;
+  static constexpr int b_off = a_off + kP2Stages * kP2Sub * kP2TileBytes;
+  static constexpr int sfa_off = b_off + kP2Stages * kP2Sub * kP2TileBytes;
+  static constexpr int sfb_off = sfa_off + kP2Stages * kP2Sub * kP2SfaBytes;
+  static constexpr int bar_off = sfb_off + kP2Stages * kP2Sub * kP2SfbBytes;
+  // full[S], empty[S], acc_full[2], acc_empty[2], tmem slot, abort flag
+  static constexpr int bytes = bar_off + (2 * kP2Stages + 4) * 8 + 16;
 };
 constexpr int kP2SmemBytes = P2Smem::bytes + 1024;
 
@@ -361,16 +375,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + P2Smem::bar_off);
   uint64_t *empty = full + kP2Stages;
-  uint64_t *acc_full = empty + kP2Stages;
-  uint64_t *acc_empty = acc_full + 1;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 1);
+  uint64_t *acc_full = empty + kP2Stages;             // [2]: one per accumulator buffer
+  uint64_t *acc_empty = acc_full + 2;                 // [2]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = ptx::cluster_rank();
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  const int n_iters = g.n16_stages + g.n8_stages;
+  const int n16s = (g.n16_stages + kP2Sub - 1) / kP2Sub, n8s = (g.n8_stages + kP2Sub - 1) / kP2Sub;
+  const int n_iters = n16s + n8s;                      // stages of kP2Sub slices
   const int n_tiles_total = g.m_tiles * g.n_tiles;
 
   if (threadIdx.x == 0) {
@@ -378,8 +393,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
       ptx::mbar_init(&full[s], 1);
       ptx::mbar_init(&empty[s], 1);
     }
-    ptx::mbar_init(acc_full, 1);
-    ptx::mbar_init(acc_empty, 2 * kP2EpiWarps);
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&acc_full[b], 1);
+      ptx::mbar_init(&acc_empty[b], 2 * kP2EpiWarps);
+    }
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -394,42 +411,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      const uint32_t bytes16 = 2 * (2 * kP2TileBytes);
-      const uint32_t bytes8 = 2 * (2 * kP2TileBytes + kP2SfaBytes + kP2SfbBytes);
+      const uint32_t bytes16 = 2 * (kP2TileBytes + kP2BRows * kSliceBytes);           // per slice, both CTAs
+      const uint32_t bytes8 = 2 * (kP2TileBytes + kP2BRows * kSliceBytes + kP2SfaBytes + kP2SfbBytes);
       int it = 0;
       for (int t = pair; t < n_tiles_total && !*abort_flag; t += npairs) {
         const int mt = t / g.n_tiles, nt = t - mt * g.n_tiles;
         const int am = mt * 256 + static_cast<int>(rank) * kP2Rows;      // this CTA's A rows
-        const int bn = nt * 256 + static_cast<int>(rank) * kP2Rows;      // this CTA's B rows
+        const int bn = nt * kP2N + static_cast<int>(rank) * kP2BRows;    // this CTA's B rows
         for (int k = 0; k < n_iters; ++k, ++it) {
           const int s = it % kP2Stages;
           if (it >= kP2Stages && !wait_bounded(&empty[s], ((it / kP2Stages) - 1) & 1, abort_flag)) break;
           const uint32_t lbar = ptx::map_to_rank(ptx::smem_addr(&full[s]), 0);
-          uint8_t *sa = smem + P2Smem::a_off + s * kP2TileBytes;
-          uint8_t *sb = smem + P2Smem::b_off + s * kP2TileBytes;
-          if (k < g.n16_stages) {
-            if (leader) ptx::mbar_arrive_expect_tx(&full[s], bytes16);
-            ptx::tma_load_2d_pair(sa, &tmA16, lbar, k * 64, am);
-            ptx::tma_load_2d_pair(sb, &tmB16, lbar, k * 64, bn);
-          } else {
-            const int j = k - g.n16_stages;
-            if (leader) ptx::mbar_arrive_expect_tx(&full[s], bytes8);
-            ptx::tma_load_2d_pair(sa, &tmA8, lbar, j * 128, am);
-            ptx::tma_load_2d_pair(sb, &tmB8, lbar, j * 128, bn);
-            ptx::tma_load_2d_pair(smem + P2Smem::sfa_off + s * kP2SfaBytes, &tmSFA, lbar, 0,
-                                  4 * (j * g.nrg_a + am / 128));
-            ptx::tma_load_2d_pair(smem + P2Smem::sfb_off + s * kP2SfbBytes, &tmSFB, lbar, 0,
-                                  4 * (j * g.nrg_b + nt * 2));
+          const bool wide = k < n16s;
+          const int j0 = kP2Sub * (wide ? k : k - n16s);                    // first slice of the stage
+          const int nsub = min(kP2Sub, (wide ? g.n16_stages : g.n8_stages) - j0);
+          if (leader) ptx::mbar_arrive_expect_tx(&full[s], nsub * (wide ? bytes16 : bytes8));
+          for (int h = 0; h < nsub; ++h) {
+            const int j = j0 + h;
+            uint8_t *sa = smem + P2Smem::a_off + (s * kP2Sub + h) * kP2TileBytes;
+            uint8_t *sb = smem + P2Smem::b_off + (s * kP2Sub + h) * kP2TileBytes;
+            if (wide) {
+              ptx::tma_load_2d_pair(sa, &tmA16, lbar, j * 64, am);
+              ptx::tma_load_2d_pair(sb, &tmB16, lbar, j * 64, bn);
+            } else {
+              ptx::tma_load_2d_pair(sa, &tmA8, lbar, j * 128, am);
+              ptx::tma_load_2d_pair(sb, &tmB8, lbar, j * 128, bn);
+              ptx::tma_load_2d_pair(smem + P2Smem::sfa_off + (s * kP2Sub + h) * kP2SfaBytes, &tmSFA, lbar, 0,
+                                    4 * (j * g.nrg_a + am / 128));
+              ptx::tma_load_2d_pair(smem + P2Smem::sfb_off + (s * kP2Sub + h) * kP2SfbBytes, &tmSFB, lbar, 0,
+                                    4 * (j * g.nrg_b + nt * 2));
+            }
           }
         }
       }
     }
   } else if (warp == 1) {
     if (leader && lane == 0) {
-      const uint32_t tsfa = tmem + kSfaCol, tsfb = tmem + kSfbCol;
+      const uint32_t tsfa = tmem + kP2SfCol, tsfb = tsfa + 4;
       int it = 0, tl = 0;
       for (int t = pair; t < n_tiles_total && !*abort_flag; t += npairs, ++tl) {
-        if (tl > 0 && !wait_bounded(acc_empty, (tl - 1) & 1, abort_flag)) break;
+        const int buf = tl & 1;
+        const uint32_t acc = tmem + buf * kP2AccCols;
+        // the buffer's previous tile (tl - 2) must have been drained
+        if (tl >= 2 && !wait_bounded(&acc_empty[buf], ((tl >> 1) - 1) & 1, abort_flag)) break;
         ptx::tc_fence_after();
         bool ok = true;
         for (int k = 0; k < n_iters; ++k, ++it) {
@@ -438,49 +462,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
             ok = false;
             break;
           }
-          const uint32_t a_base = ptx::smem_addr(smem + P2Smem::a_off + s * kP2TileBytes);
-          const uint32_t b_base = ptx::smem_addr(smem + P2Smem::b_off + s * kP2TileBytes);
-          if (k < g.n16_stages) {
+          const bool wide = k < n16s;
+          const int j0 = kP2Sub * (wide ? k : k - n16s);
+          const int nsub = min(kP2Sub, (wide ? g.n16_stages : g.n8_stages) - j0);
+          for (int h = 0; h < nsub; ++h) {
+            const uint32_t a_base = ptx::smem_addr(smem + P2Smem::a_off + (s * kP2Sub + h) * kP2TileBytes);
+            const uint32_t b_base = ptx::smem_addr(smem + P2Smem::b_off + (s * kP2Sub + h) * kP2TileBytes);
+            if (wide) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              ptx::mma2_bf16(tmem, ptx::desc_sw128(a_base + 32 * q), ptx::desc_sw128(b_base + 32 * q), kIdesc2Bf16,
-                             (k > 0 || q > 0) ? 1u : 0u);
-          } else {
-            const uint32_t sfa_s = ptx::smem_addr(smem + P2Smem::sfa_off + s * kP2SfaBytes);
-            const uint32_t sfb_s = ptx::smem_addr(smem + P2Smem::sfb_off + s * kP2SfbBytes);
-            ptx::copy_sf_to_tmem2(tsfa, ptx::desc_sf(sfa_s));
-            ptx::copy_sf_to_tmem2(tsfb, ptx::desc_sf(sfb_s));
-            ptx::copy_sf_to_tmem2(tsfb + 4, ptx::desc_sf(sfb_s + kSfChunk));
+              for (int q = 0; q < 4; ++q)
+                ptx::mma2_bf16(acc, ptx::desc_sw128(a_base + 32 * q), ptx::desc_sw128(b_base + 32 * q), kIdesc2Bf16,
+                               (k > 0 || h > 0 || q > 0) ? 1u : 0u);
+            } else {
+              const uint32_t sfa_s = ptx::smem_addr(smem + P2Smem::sfa_off + (s * kP2Sub + h) * kP2SfaBytes);
+              const uint32_t sfb_s = ptx::smem_addr(smem + P2Smem::sfb_off + (s * kP2Sub + h) * kP2SfbBytes);
+              const uint32_t slot = kSfSlotCols * static_cast<uint32_t>((kP2Sub * it + h) % kP2SfSlots);
+              ptx::copy_sf_to_tmem2(tsfa + slot, ptx::desc_sf(sfa_s));
+              ptx::copy_sf_to_tmem2(tsfb + slot, ptx::desc_sf(sfb_s));
+              ptx::copy_sf_to_tmem2(tsfb + slot + 4, ptx::desc_sf(sfb_s + kSfChunk));
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint32_t idesc = kIdesc2Mxf8 | (static_cast<uint32_t>(q) << 4) | (static_cast<uint32_t>(q) << 29);
-              ptx::mma2_mxf8(tmem, ptx::desc_sw128(a_base + 32 * q), ptx::desc_sw128(b_base + 32 * q), idesc,
-                             (k > 0 || q > 0) ? 1u : 0u, tsfa | (static_cast<uint32_t>(q) << 30),
-                             tsfb | (static_cast<uint32_t>(q) << 30));
+              for (int q = 0; q < 4; ++q) {
+                const uint32_t idesc = kIdesc2Mxf8 | (static_cast<uint32_t>(q) << 4) | (static_cast<uint32_t>(q) << 29);
+                ptx::mma2_mxf8(acc, ptx::desc_sw128(a_base + 32 * q), ptx::desc_sw128(b_base + 32 * q), idesc,
+                               (k > 0 || h > 0 || q > 0) ? 1u : 0u, (tsfa + slot) | (static_cast<uint32_t>(q) << 30),
+                               (tsfb + slot) | (static_cast<uint32_t>(q) << 30));
+              }
             }
           }
           ptx::mma2_commit_both(&empty[s]);
         }
         if (!ok) break;
-        ptx::mma2_commit_both(acc_full);
+        ptx::mma2_commit_both(&acc_full[buf]);
       }
     }
   } else {
-    // epilogue: warp w reads lanes 32*(w%4)..+31, columns 128*h..128*h+127
+    // epilogue: warp w reads lanes 32*(w%4)..+31 and columns 120h..120h+119
+    // (h = 0, 1) of the tile's accumulator buffer; loads are 32 columns wide,
+    // so the last one reads 8 columns past the half, which are not stored
     const int q = warp & 3, h = (warp - 2) >> 2;
-    const uint32_t acc_empty_leader = ptx::map_to_rank(ptx::smem_addr(acc_empty), 0);
     int tl = 0;
     for (int t = pair; t < n_tiles_total; t += npairs, ++tl) {
-      if (!wait_bounded(acc_full, tl & 1, abort_flag)) break;
+      const int buf = tl & 1;
+      if (!wait_bounded(&acc_full[buf], (tl >> 1) & 1, abort_flag)) break;
       ptx::tc_fence_after();
       uint32_t r[4][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        ptx::tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + 128 * h + 32 * c, r[c]);
+        ptx::tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * kP2AccCols + (kP2N / 2) * h + 32 * c, r[c]);
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive_cluster(acc_empty_leader);
+      if (lane == 0) ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&acc_empty[buf]), 0));
       const int mt = t / g.n_tiles, nt = t - mt * g.n_tiles;
       const int row = mt * 256 + static_cast<int>(rank) * kP2Rows + q * 32 + lane;
       if (row < g.M) {
@@ -489,7 +521,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
         for (int c = 0; c < 4; ++c) {
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
-            const int n = nt * 256 + 128 * h + 32 * c + 8 * v;
+            if (32 * c + 8 * v >= kP2N / 2) continue;           // the other half's columns
+            const int n = nt * kP2N + (kP2N / 2) * h + 32 * c + 8 * v;
             if (g.y_vec && n + 8 <= g.N) {
               uint32_t pk[4];
 #pragma unroll
@@ -531,6 +564,7 @@ struct StageOperand {
   uint8_t *x8;          // rows x k4 E4M3 bytes
   uint8_t *sf;          // scale chunks [k-group][row-group][512]
   int32_t nrg;          // row groups of 128 in sf
+  int32_t tile_rows;    // rows per output tile: tile t's rows fill chunk rows 256 t .. 256 t + tile_rows - 1
 };
 
 // Item space of the staging kernel, one item per (operand, row, block):
@@ -672,11 +706,12 @@ __global__ void __launch_bounds__(256) gemm_stage_kernel(StageArgs a) {
         else stage_wide_block<6>(op.codes[1] + row * op.cpitch[1] + static_cast<int64_t>(bb) * 24, sbyte, dst);
       }
     } else {
-      const int row = i / a.nb4p, b = i - row * a.nb4p;
+      const int row = i / a.nb4p, b = i - row * a.nb4p;     // row of the chunk grid
+      const int lr = row & 255, real = (row >> 8) * op.tile_rows + lr;   // the operand row it holds
       uint32_t sb = 0x7Fu;                             // 2^0 for padding rows and blocks
-      if (in_range && row < op.rows && b < a.nb[2]) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(op.codes[2] + row * op.cpitch[2] + static_cast<int64_t>(b) * 16);
-        sb = op.scales[2][row * op.spitch[2] + b];
+      if (in_range && lr < op.tile_rows && real < op.rows && b < a.nb[2]) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(op.codes[2] + real * op.cpitch[2] + static_cast<int64_t>(b) * 16);
+        sb = op.scales[2][real * op.spitch[2] + b];
         const uint32_t in[4] = {v.x, v.y, v.z, v.w};
         uint32_t out[8];
 #pragma unroll
@@ -685,7 +720,7 @@ __global__ void __launch_bounds__(256) gemm_stage_kernel(StageArgs a) {
           out[2 * j] = static_cast<uint32_t>(lut[x & 0xFF]) | (static_cast<uint32_t>(lut[(x >> 8) & 0xFF]) << 16);
           out[2 * j + 1] = static_cast<uint32_t>(lut[(x >> 16) & 0xFF]) | (static_cast<uint32_t>(lut[x >> 24]) << 16);
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(op.x8 + static_cast<int64_t>(row) * a.k4 + static_cast<int64_t>(b) * kBlock);
+        uint4 *dst = reinterpret_cast<uint4 *>(op.x8 + static_cast<int64_t>(real) * a.k4 + static_cast<int64_t>(b) * kBlock);
         dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
         dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
       }
@@ -1042,7 +1077,7 @@ constexpr int64_t kPairMinM = 512;   // from here the 2-CTA pair kernel
 
 struct WsPlan {
   int64_t k16, k4;
-  int32_t nkg, nrg_a, nrg_b;
+  int32_t nkg, nrg_a, nrg_b, b_tile_rows;
   size_t off_a16, off_b16, off_a8, off_b8, off_sfa, off_sfb, total;
 };
 
@@ -1053,7 +1088,10 @@ static WsPlan plan_workspace(const mxs_mxtensor *A, const mxs_mxtensor *W) {
   p.k4 = A->lay.seg[2].k_pad;
   p.nkg = static_cast<int32_t>((p.k4 + 127) / 128);
   p.nrg_a = static_cast<int32_t>((M + kBM - 1) / kBM);
-  p.nrg_b = static_cast<int32_t>((N + kBN - 1) / kBN * (kBN / 128));
+  // B's scale chunks follow the output tiles: 256-row tiles (one CTA) or
+  // 240-row tiles (2-CTA pairs), two 128-row chunks per tile
+  p.b_tile_rows = M >= kPairMinM ? kP2N : kBN;
+  p.nrg_b = static_cast<int32_t>((N + p.b_tile_rows - 1) / p.b_tile_rows * 2);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -1218,6 +1256,7 @@ extern "C" mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, voi
     op.x8 = base + (o ? p.off_b8 : p.off_a8);
     op.sf = base + (o ? p.off_sfb : p.off_sfa);
     op.nrg = o ? p.nrg_b : p.nrg_a;
+    op.tile_rows = o ? p.b_tile_rows : 256;
   }
   for (int g = 0; g < 3; ++g) sa.nb[g] = static_cast<int32_t>(A->lay.seg[g].k_pad / kBlock);
   sa.nbw = sa.nb[0] + sa.nb[1];
@@ -1265,11 +1304,11 @@ extern "C" mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, voi
           !make_rows_map(&mSFB, base + p.off_sfb, static_cast<int64_t>(p.nkg) * p.nrg_b * kSfChunk, 8))
         return MXS_ERR_CUDA;
     }
-    if (p.k16 > 0) {   // the pair kernel loads 128-row boxes of B
-      if (!make_map(&mB16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base + p.off_b16, p.k16, N, kP2Rows)) return MXS_ERR_CUDA;
+    if (p.k16 > 0) {   // the pair kernel loads 120-row boxes of B
+      if (!make_map(&mB16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base + p.off_b16, p.k16, N, kP2BRows)) return MXS_ERR_CUDA;
     }
     if (p.k4 > 0) {
-      if (!make_map(&mB8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + p.off_b8, p.k4, N, kP2Rows)) return MXS_ERR_CUDA;
+      if (!make_map(&mB8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + p.off_b8, p.k4, N, kP2BRows)) return MXS_ERR_CUDA;
     }
     P2Args pa{};
     pa.M = static_cast<int32_t>(M);
@@ -1277,7 +1316,7 @@ extern "C" mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, voi
     pa.n16_stages = n16_stages;
     pa.n8_stages = n8_stages;
     pa.m_tiles = static_cast<int32_t>((M + 255) / 256);
-    pa.n_tiles = static_cast<int32_t>((N + 255) / 256);
+    pa.n_tiles = static_cast<int32_t>((N + kP2N - 1) / kP2N);
     pa.nrg_a = p.nrg_a;
     pa.nrg_b = p.nrg_b;
     pa.Y = reinterpret_cast<__nv_bfloat16 *>(Y);

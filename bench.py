@@ -37,6 +37,7 @@ N_OUT, K_IN, T_CAL = 4096, 4096, 2048
 KV_SHAPE = (8192, 8, 128)
 BUDGET = (9, 2)
 SEED = 2000
+CALL_REPS, CALL_TRIALS = 10, 5   # per-call timing: calls per graph, replays per graph
 METRIC = "mxs_gemm TFLOP/s (% of roofline); MXINT quantize GB/s (% of HBM peak)"
 WORKLOAD = ("llama3-8b attention projection: W 4096x4096 bf16 (3% t3 columns), calib X 2048x4096 bf16 "
             "(8 channels x50), budget 4.5 bits, GEMM M in {2048,16,1}; + K/V cache 8192x8x128 bf16 x2")
@@ -157,6 +158,7 @@ class Path:
         gws = max(c.mxs_gemm_workspace_bytes(self.Aq[M], self.Wq) for M in M_LIST)
         self.gemm_ws = torch.empty(gws + 1024, dtype=torch.uint8, device=dev)
         self.flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+        self.flush_small = self.flush[: 256 << 20]          # per-call timing: twice the L2
         # algorithmic bytes / FLOPs per launch of each timed call
         n8, n6, n4 = self.counts
         self.work = {
@@ -234,9 +236,12 @@ def run_gpu(args, rank, world, local_rank):
         torch.cuda.synchronize()
 
     # The step is captured once as one CUDA graph (its kernels back to back,
-    # no host launch gaps) and replayed once per timed step.  Every call is
-    # also captured alone; a second pass replays those in step order with
-    # CUDA events between them to time each call.
+    # no host launch gaps) and replayed once per timed step.  Each call is
+    # then timed on its own by difference: a graph of CALL_REPS x (L2 flush,
+    # call) against a graph of CALL_REPS flushes alone, both replayed
+    # between CUDA events; the call's time is the difference / CALL_REPS, so
+    # neither graph-launch gaps nor the flush enter it, and every call starts
+    # with a cold L2.
     calls = path.calls()
     cap = torch.cuda.Stream()
     launches0 = c.mxs_launch_count()
@@ -245,62 +250,65 @@ def run_gpu(args, rank, world, local_rank):
         for _, fn in calls:
             fn()
     launches_per_step = c.mxs_launch_count() - launches0
-    graphs = []
-    for name, fn in calls:
+
+    def rep_graph(fn):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=cap):
-            fn()
-        graphs.append((name, g))
+            for _ in range(CALL_REPS):
+                path.flush_small.zero_()
+                if fn is not None:
+                    fn()
+        return g
+    g_flush = rep_graph(None)
+    graphs = [(name, rep_graph(fn)) for name, fn in calls]
     for _ in range(3):
         path.flush.zero_()
         g_step.replay()
-        path.flush.zero_()
+        g_flush.replay()
         for _, g in graphs:
             g.replay()
     c.mxs_sync()
 
+    def timed(g):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        g.replay()
+        e.record()
+        return s, e
+
     rec = {}
     step_ev = []
-    call_steps = min(args.steps, 50)
     barrier()
     with ClockSampler(local_rank) as clocks:
         t0 = time.perf_counter()
         for _ in range(args.steps):
             path.flush.zero_()                      # L2 flush, outside the step events
-            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            s.record()
-            g_step.replay()
-            e.record()
-            step_ev.append((s, e))
+            step_ev.append(timed(g_step))
         barrier()
         wall = time.perf_counter() - t0
-        for _ in range(call_steps):
-            path.flush.zero_()
-            evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)]
-            evs[0].record()
-            for i, (name, g) in enumerate(graphs):
-                g.replay()
-                evs[i + 1].record()
-                rec.setdefault(name, []).append((evs[i], evs[i + 1]))
+        for _ in range(CALL_TRIALS):
+            rec.setdefault("", []).append(timed(g_flush))
+            for name, g in graphs:
+                rec.setdefault(name, []).append(timed(g))
         barrier()
     launches = launches_per_step * args.steps
     c.mxs_sync()
     step_ms = [s.elapsed_time(e) for s, e in step_ev]
     total_s = sum(step_ms) * 1e-3
-    call_step_ms = sum(s.elapsed_time(e) for evs in rec.values() for s, e in evs) / call_steps
     if world > 1:
         tt = torch.tensor([total_s], device=dev, dtype=torch.float64)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         total_s = float(tt.item())
     value = world * path.gemm_flops * args.steps / total_s / 1e12
+    best = {name: min(s.elapsed_time(e) for s, e in evs) * 1e-3 for name, evs in rec.items()}
+    per_call = {name: max(best[name] - best[""], 0.0) / CALL_REPS for name, _ in calls}
+    call_sum = sum(per_call.values())
 
     kernels = {}
-    for name, evs in rec.items():
-        ms = [s.elapsed_time(e) for s, e in evs]
-        per = sum(ms) / len(ms) * 1e-3
+    for name, per in per_call.items():
         unit, work = path.work[name]
         ach = work / per / (1e12 if unit == "TFLOP/s" else 1e9)
-        kd = {"us": per * 1e6, "achieved": ach, "unit": unit, "share": per * 1e3 / call_step_ms}
+        kd = {"us": per * 1e6, "achieved": ach, "unit": unit, "share": per / call_sum}
         if unit == "GB/s":
             kd["frac_hbm"] = ach / pk["hbm_gbs"]
             kd["frac_nominal_8tbs"] = ach / 8000.0
@@ -328,7 +336,8 @@ def run_gpu(args, rank, world, local_rank):
         "config": {"workload": WORKLOAD, "counts_n8_n6_n4": list(path.counts), "l2": "flushed between steps "
                    "(512 MB write outside the step events)", "parallelism": f"replicas x{world} (no data-path collective)",
                    "timing": "step = one CUDA graph of all C-ABI calls, replayed per step between CUDA events; "
-                             "kernels{} from a second pass of per-call graphs in step order with events between",
+                             f"kernels{{}}: per call, (graph of {CALL_REPS} x [L2 flush, call]) - (graph of "
+                             f"{CALL_REPS} flushes), best of {CALL_TRIALS} replays each, / {CALL_REPS}; cold L2 per call",
                    "launches_per_step": launches_per_step},
         "roofline": roof, "kernels": kernels, "e2e": e2e, "gpu_launches": launches,
         "clocks": clocks.summary(), "wall_s_timed_region": wall,

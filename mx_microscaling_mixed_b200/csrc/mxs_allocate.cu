@@ -41,6 +41,7 @@ constexpr int kRankSlice = kRankTile / kRankParts;
 // Slices wholly before j count ties, slices wholly after j do not; only the
 // slice holding j compares indices.
 __global__ void __launch_bounds__(kRankThreads) rank_kernel(const double *s, int64_t K, int32_t *rank) {
+  pdl_wait();
   __shared__ double tile[kRankTile];
   __shared__ int part_cnt[kRankParts][kRankCols];
   const int c = threadIdx.x % kRankCols, part = threadIdx.x / kRankCols;
@@ -77,6 +78,7 @@ __global__ void __launch_bounds__(kRankThreads) rank_kernel(const double *s, int
 }
 
 __global__ void order_kernel(const int32_t *rank, int64_t K, int32_t *order) {
+  pdl_wait();
   const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (j < K) order[rank[j]] = static_cast<int32_t>(j);
 }
@@ -84,6 +86,7 @@ __global__ void order_kernel(const int32_t *rank, int64_t K, int32_t *order) {
 // gains[g] = sum of s over ranks [n8 + 32 g, min(n8 + 32 g + 32, K)), in rank order.
 __global__ void group_gain_kernel(const double *s, const int32_t *order, int64_t K, int64_t n8,
                                   int64_t ngroups, double *gains) {
+  pdl_wait();
   const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (g >= ngroups) return;
   const int64_t r0 = n8 + 32 * g, r1 = min(r0 + 32, K);
@@ -100,6 +103,7 @@ constexpr int kPermThreads = 1024;
 // slot in each segment, pass 2 writes the permutation.
 __global__ void __launch_bounds__(kPermThreads) perm_kernel(const int32_t *rank, int64_t K, int64_t n8,
                                                             int64_t n6, int32_t *perm) {
+  pdl_wait();
   __shared__ unsigned long long warp_tot[kPermThreads / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t ipt = (K + kPermThreads - 1) / kPermThreads;
@@ -202,7 +206,7 @@ extern "C" mxs_status mxs_allocate(int32_t n_layers, const int64_t *K, const int
     L[l].order = reinterpret_cast<int32_t *>(p + round_up(K[l] * 4, 256));
     L[l].gains = reinterpret_cast<double *>(p + 2 * round_up(K[l] * 4, 256));
     p += layer_ws_bytes(K[l]);
-    rank_kernel<<<static_cast<unsigned>((K[l] + kRankCols - 1) / kRankCols), kRankThreads, 0, cs>>>(s[l], K[l],
+    launch_pdl(rank_kernel, dim3(static_cast<unsigned>((K[l] + kRankCols - 1) / kRankCols)), dim3(kRankThreads), 0, cs, s[l], K[l],
                                                                                                    L[l].rank);
     count_launch();
   }
@@ -227,9 +231,9 @@ extern "C" mxs_status mxs_allocate(int32_t n_layers, const int64_t *K, const int
         const int64_t ng = (K[l] - n8[l] + 31) / 32;
         gains[l].assign(static_cast<size_t>(std::max<int64_t>(ng, 1)), 0.0);
         if (ng > 0) {
-          order_kernel<<<static_cast<unsigned>((K[l] + 255) / 256), 256, 0, cs>>>(L[l].rank, K[l], L[l].order);
+          launch_pdl(order_kernel, dim3(static_cast<unsigned>((K[l] + 255) / 256)), dim3(256), 0, cs, L[l].rank, K[l], L[l].order);
           count_launch();
-          group_gain_kernel<<<static_cast<unsigned>((ng + 127) / 128), 128, 0, cs>>>(s[l], L[l].order, K[l],
+          launch_pdl(group_gain_kernel, dim3(static_cast<unsigned>((ng + 127) / 128)), dim3(128), 0, cs, s[l], L[l].order, K[l],
                                                                                     n8[l], ng, L[l].gains);
           count_launch();
           if (cudaMemcpyAsync(gains[l].data(), L[l].gains, static_cast<size_t>(ng) * 8,
@@ -266,7 +270,7 @@ extern "C" mxs_status mxs_allocate(int32_t n_layers, const int64_t *K, const int
   }
 
   for (int l = 0; l < n_layers; ++l) {
-    perm_kernel<<<1, kPermThreads, 0, cs>>>(L[l].rank, K[l], n8[l], n6[l], perm[l]);
+    launch_pdl(perm_kernel, dim3(1), dim3(kPermThreads), 0, cs, L[l].rank, K[l], n8[l], n6[l], perm[l]);
     count_launch();
     counts[3 * l + 0] = n8[l];
     counts[3 * l + 1] = n6[l];

@@ -109,6 +109,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA16, const __grid_constant__ CUtensorMap tmB16,
                    const __grid_constant__ CUtensorMap tmA8, const __grid_constant__ CUtensorMap tmB8,
                    GemmArgs g) {
+  pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + GemmSmem::bar_off);
@@ -371,6 +372,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA16, const __grid_constant__ CUtensorMap tmB16,
                     const __grid_constant__ CUtensorMap tmA8, const __grid_constant__ CUtensorMap tmB8,
                     const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB, P2Args g) {
+  pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + P2Smem::bar_off);
@@ -679,6 +681,7 @@ __device__ __forceinline__ void stage_wide_block(const uint8_t *c, uint8_t sbyte
 // codes); a k-group's four scale bytes are gathered by shuffles and written
 // as one word of the tensor core's 512-byte chunk layout.
 __global__ void __launch_bounds__(256) gemm_stage_kernel(StageArgs a) {
+  pdl_wait();
   __shared__ uint16_t lut[256];                        // byte of two 4-bit codes -> their E4M3 pair (q/4)
   {
     const int b = threadIdx.x;
@@ -959,6 +962,7 @@ constexpr long long kDecWaitLimit = 2000000000LL;    // cycles (~1 s)
 // and scale rows and the 16 W rows' scale rows into shared memory; the warps
 // then run the three segments and add their partial sums in warp order.
 __global__ void __launch_bounds__(kDecThreads) gemm_small_kernel(SmallArgs a, int *status) {
+  pdl_wait();
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t bar;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1065,7 +1069,7 @@ static mxs_status gemm_small(const mxs_mxtensor *A, const mxs_mxtensor *W, void 
   if (!status) return MXS_ERR_CUDA;
   const int smem = static_cast<int>(small_smem_bytes(a));
   if (!ensure_smem(gemm_small_kernel, smem)) return MXS_ERR_CUDA;
-  gemm_small_kernel<<<(a.N + kDecRows - 1) / kDecRows, kDecThreads, smem, cs>>>(a, status);
+  launch_pdl(gemm_small_kernel, dim3((a.N + kDecRows - 1) / kDecRows), dim3(kDecThreads), smem, cs, a, status);
   count_launch();
   return cuda_status(cudaGetLastError());
 }
@@ -1280,7 +1284,7 @@ extern "C" mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, voi
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   const int sgrid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((sa.start[4] + 255) / 256, static_cast<int64_t>(nsm) * 8)));
-  gemm_stage_kernel<<<sgrid, 256, 0, cs>>>(sa);
+  launch_pdl(gemm_stage_kernel, dim3(sgrid), dim3(256), 0, cs, sa);
   count_launch();
 
   CUtensorMap mA16{}, mB16{}, mA8{}, mB8{};
@@ -1325,7 +1329,7 @@ extern "C" mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, voi
     if (!ensure_smem(gemm_tc2_kernel, kP2SmemBytes)) return MXS_ERR_CUDA;
     const int tiles = pa.m_tiles * pa.n_tiles;
     const int pairs = std::max(1, std::min(tiles, nsm / 2));
-    gemm_tc2_kernel<<<2 * pairs, kP2Threads, kP2SmemBytes, cs>>>(mA16, mB16, mA8, mB8, mSFA, mSFB, pa);
+    launch_pdl(gemm_tc2_kernel, dim3(2 * pairs), dim3(kP2Threads), kP2SmemBytes, cs, mA16, mB16, mA8, mB8, mSFA, mSFB, pa);
     count_launch();
     return cuda_status(cudaGetLastError());
   }
@@ -1343,7 +1347,7 @@ extern "C" mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, voi
   ga.y_vec = y_vec;
   if (!ensure_smem(gemm_tc_kernel, kGemmSmemBytes)) return MXS_ERR_CUDA;
   dim3 grid(static_cast<unsigned>((N + kBN - 1) / kBN), static_cast<unsigned>((M + kBM - 1) / kBM));
-  gemm_tc_kernel<<<grid, kGemmThreads, kGemmSmemBytes, cs>>>(mA16, mB16, mA8, mB8, ga);
+  launch_pdl(gemm_tc_kernel, dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, cs, mA16, mB16, mA8, mB8, ga);
   count_launch();
   return cuda_status(cudaGetLastError());
 }

@@ -206,6 +206,83 @@ __device__ __forceinline__ void encode_store(float (&v)[kBlock], uint8_t *cdst, 
   }
 }
 
+// bf16 source, 4- and 6-bit codes: the same rule on packed pairs.  p[i]
+// holds positions 2i (low half) and 2i+1 (high half) as bf16 bits.  The
+// block maximum is an unsigned 16-bit max of the bit patterns with the sign
+// cleared (monotonic in |x|), so the E8M0 byte is its exponent field, as
+// for fp32.  Rounding: one bf16x2 fma x*2^k + 192 (a single rounding of the
+// exact value; 192 + q stays in [128, 256), where bf16 steps by 1) leaves
+// the lane's bits at 0x4340 + q, so clamping is an unsigned 16-bit min/max
+// and the code is the low m bits.  When k > 125 the block is tiny and takes
+// the fp32 path, so that subnormal inputs never meet the bf16 fma.
+__device__ __forceinline__ uint32_t fma_bf16x2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+template <int M>
+__device__ __forceinline__ void encode_store_bf16(const uint32_t (&p)[kBlock / 2], uint8_t *cdst, uint8_t *sdst) {
+  static_assert(M == 4 || M == 6, "packed path for 4- and 6-bit codes");
+  uint32_t m2 = 0;
+#pragma unroll
+  for (int i = 0; i < kBlock / 2; ++i) m2 = __vmaxu2(m2, p[i] & 0x7FFF7FFFu);
+  const int ef = static_cast<int>(max(m2 & 0xFFFFu, m2 >> 16) >> 7);
+  const int k = M - 2 - (ef == 0 ? -127 : ef - 127);
+  if (k > 125) {
+    float v[kBlock];
+#pragma unroll
+    for (int i = 0; i < kBlock / 2; ++i) {
+      v[2 * i] = __uint_as_float(p[i] << 16);
+      v[2 * i + 1] = __uint_as_float(p[i] & 0xFFFF0000u);
+    }
+    encode_store<M>(v, cdst, sdst);
+    return;
+  }
+  const uint32_t sb = static_cast<uint32_t>(k + 127) << 7;
+  const uint32_t s2 = sb | (sb << 16);
+  constexpr uint32_t L = (1u << (M - 1)) - 1u;
+  constexpr uint32_t lo2 = (0x4340u - L) * 0x10001u, hi2 = (0x4340u + L) * 0x10001u;
+  uint32_t r[kBlock / 2];
+#pragma unroll
+  for (int i = 0; i < kBlock / 2; ++i) r[i] = __vminu2(__vmaxu2(fma_bf16x2(p[i], s2, 0x43404340u), lo2), hi2);
+  *sdst = static_cast<uint8_t>(ef);
+  if constexpr (M == 4) {
+    // bytes of positions 4j..4j+3 (low byte of each lane), then each
+    // byte's nibble joined with the next byte's: bytes 0 and 2 hold two codes
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t x = __byte_perm(r[4 * j], r[4 * j + 1], 0x6420);
+      const uint32_t y = __byte_perm(r[4 * j + 2], r[4 * j + 3], 0x6420);
+      const uint32_t zx = (x & 0x0F0F0F0Fu) | ((x >> 4) & 0xF0F0F0F0u);
+      const uint32_t zy = (y & 0x0F0F0F0Fu) | ((y >> 4) & 0xF0F0F0F0u);
+      w[j] = __byte_perm(zx, zy, 0x6420);
+    }
+    *reinterpret_cast<uint4 *>(cdst) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+    // 24-bit groups of four codes, then eight groups into six words
+    uint32_t u[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t x = __byte_perm(r[2 * j], r[2 * j + 1], 0x6420);
+      const uint32_t z = (x & 0x003F003Fu) | ((x >> 2) & 0x0FC00FC0u);
+      u[j] = (z & 0xFFFu) | ((z >> 4) & 0xFFF000u);
+    }
+    uint32_t w[6];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      w[3 * h] = u[4 * h] | (u[4 * h + 1] << 24);
+      w[3 * h + 1] = (u[4 * h + 1] >> 8) | (u[4 * h + 2] << 16);
+      w[3 * h + 2] = (u[4 * h + 2] >> 16) | (u[4 * h + 3] << 8);
+    }
+    uint2 *q = reinterpret_cast<uint2 *>(cdst);
+    q[0] = make_uint2(w[0], w[1]);
+    q[1] = make_uint2(w[2], w[3]);
+    q[2] = make_uint2(w[4], w[5]);
+  }
+}
+
 // Value at byte offset `off` of a staged row.
 template <bool F32>
 __device__ __forceinline__ float staged_elem(const uint8_t *row, uint32_t off) {
@@ -255,23 +332,42 @@ template <int M, bool F32>
 __device__ __forceinline__ void code_item(const QuantArgs &a, int g, int b, const uint32_t *tab, const uint8_t *srow,
                                           int64_t row) {
   const uint4 *tw = reinterpret_cast<const uint4 *>(tab + (a.boff[g] + b) * kTabWordsPerBlock);
-  float v[kBlock];
+  if constexpr (!F32 && M != 8) {
+    uint32_t p[kBlock / 2];
 #pragma unroll
-  for (int j = 0; j < kBlock / 4; ++j) {
-    const uint4 w = tw[j];
-    v[4 * j] = staged_elem<F32>(srow, w.x);
-    v[4 * j + 1] = staged_elem<F32>(srow, w.y);
-    v[4 * j + 2] = staged_elem<F32>(srow, w.z);
-    v[4 * j + 3] = staged_elem<F32>(srow, w.w);
+    for (int j = 0; j < kBlock / 4; ++j) {
+      const uint4 w = tw[j];
+      p[2 * j] = static_cast<uint32_t>(*reinterpret_cast<const unsigned short *>(srow + w.x)) |
+                 (static_cast<uint32_t>(*reinterpret_cast<const unsigned short *>(srow + w.y)) << 16);
+      p[2 * j + 1] = static_cast<uint32_t>(*reinterpret_cast<const unsigned short *>(srow + w.z)) |
+                     (static_cast<uint32_t>(*reinterpret_cast<const unsigned short *>(srow + w.w)) << 16);
+    }
+    encode_store_bf16<M>(p, a.codes[g] + row * a.cpitch[g] + b * (kBlock * M / 8), a.scales[g] + row * a.spitch[g] + b);
+  } else {
+    float v[kBlock];
+#pragma unroll
+    for (int j = 0; j < kBlock / 4; ++j) {
+      const uint4 w = tw[j];
+      v[4 * j] = staged_elem<F32>(srow, w.x);
+      v[4 * j + 1] = staged_elem<F32>(srow, w.y);
+      v[4 * j + 2] = staged_elem<F32>(srow, w.z);
+      v[4 * j + 3] = staged_elem<F32>(srow, w.w);
+    }
+    encode_store<M>(v, a.codes[g] + row * a.cpitch[g] + b * (kBlock * M / 8), a.scales[g] + row * a.spitch[g] + b);
   }
-  encode_store<M>(v, a.codes[g] + row * a.cpitch[g] + b * (kBlock * M / 8), a.scales[g] + row * a.spitch[g] + b);
 }
 
+// Polls with a growing sleep between reads, so that waiting warps leave the
+// issue slots to the warps that are coding.
 __device__ __forceinline__ bool spin_until_equal(volatile int *p, int want, long long limit) {
   if (*p == want) return true;
   const long long t0 = clock64();
-  while (*p != want)
+  unsigned ns = 32;
+  while (*p != want) {
     if (clock64() - t0 > limit) return false;
+    __nanosleep(ns);
+    ns = min(ns * 2, 512u);
+  }
   return true;
 }
 
@@ -285,6 +381,7 @@ __device__ __forceinline__ bool spin_until_equal(volatile int *p, int want, long
 // completes a batch refills that buffer with the batch kQStages ahead.
 template <bool F32>
 __global__ void __launch_bounds__(kQuantThreads, 1) quant_tile_kernel(QuantArgs a, int *status) {
+  pdl_wait();
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int ES = F32 ? 4 : 2;
   uint32_t *tab = reinterpret_cast<uint32_t *>(smem);
@@ -420,6 +517,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quant_tile_kernel(QuantArgs 
 // aligned and all real).
 template <bool F32>
 __global__ void __launch_bounds__(256) quant_contig_kernel(QuantArgs a) {
+  pdl_wait();
   constexpr int ES = F32 ? 4 : 2;
   const int64_t total = a.rows * a.nb_total;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
@@ -433,6 +531,22 @@ __global__ void __launch_bounds__(256) quant_contig_kernel(QuantArgs a) {
     const int n = min(kBlock, a.k_real[g] - p0);
     float v[kBlock];
     const uint8_t *base = reinterpret_cast<const uint8_t *>(a.src) + e0 * ES;
+    uint8_t *cdst = a.codes[g] + row * a.cpitch[g] + static_cast<int64_t>(b) * kBlock * seg_bits(g) / 8;
+    uint8_t *sdst = a.scales[g] + row * a.spitch[g] + b;
+    if (!F32 && g != 0 && n == kBlock && (reinterpret_cast<uintptr_t>(base) & 15u) == 0) {
+      uint32_t p[kBlock / 2];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 x = __ldg(reinterpret_cast<const uint4 *>(base) + j);
+        p[4 * j] = x.x;
+        p[4 * j + 1] = x.y;
+        p[4 * j + 2] = x.z;
+        p[4 * j + 3] = x.w;
+      }
+      if (g == 1) encode_store_bf16<6>(p, cdst, sdst);
+      else encode_store_bf16<4>(p, cdst, sdst);
+      continue;
+    }
     if (n == kBlock && (reinterpret_cast<uintptr_t>(base) & 15u) == 0) {
 #pragma unroll
       for (int j = 0; j < kBlock * ES / 16; ++j) {
@@ -459,8 +573,6 @@ __global__ void __launch_bounds__(256) quant_contig_kernel(QuantArgs a) {
         v[t] = x;
       }
     }
-    uint8_t *cdst = a.codes[g] + row * a.cpitch[g] + static_cast<int64_t>(b) * kBlock * seg_bits(g) / 8;
-    uint8_t *sdst = a.scales[g] + row * a.spitch[g] + b;
     if (g == 0) encode_store<8>(v, cdst, sdst);
     else if (g == 1) encode_store<6>(v, cdst, sdst);
     else encode_store<4>(v, cdst, sdst);
@@ -470,6 +582,7 @@ __global__ void __launch_bounds__(256) quant_contig_kernel(QuantArgs a) {
 // One warp per (row, block), one lane per position.
 template <bool F32>
 __global__ void __launch_bounds__(256) quant_lane_kernel(QuantArgs a) {
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t total = a.rows * a.nb_total;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -531,6 +644,7 @@ struct DequantArgs {
 };
 
 __global__ void dequant_kernel(DequantArgs a) {
+  pdl_wait();
   const int64_t total = a.rows * a.nb_total;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -671,8 +785,8 @@ static mxs_status quantize_impl(const void *src, mxs_dtype dt, int64_t rows, int
   const bool tiny = warps <= 8192;                     // latency-bound: one warp per block
   if (!tiny && !a.perm) {
     const int grid = static_cast<int>(std::min<int64_t>((warps + 255) / 256, static_cast<int64_t>(nsm) * 8));
-    if (f32) quant_contig_kernel<true><<<grid, 256, 0, s>>>(a);
-    else quant_contig_kernel<false><<<grid, 256, 0, s>>>(a);
+    if (f32) launch_pdl(quant_contig_kernel<true>, dim3(grid), dim3(256), 0, s, a);
+    else launch_pdl(quant_contig_kernel<false>, dim3(grid), dim3(256), 0, s, a);
     count_launch();
     return cuda_status(cudaGetLastError());
   }
@@ -712,15 +826,15 @@ static mxs_status quantize_impl(const void *src, mxs_dtype dt, int64_t rows, int
     if (!status) return MXS_ERR_CUDA;
     if (f32) {
       if (!ensure_smem(quant_tile_kernel<true>, static_cast<int>(smem))) return MXS_ERR_CUDA;
-      quant_tile_kernel<true><<<grid, kQuantThreads, smem, s>>>(a, status);
+      launch_pdl(quant_tile_kernel<true>, dim3(grid), dim3(kQuantThreads), smem, s, a, status);
     } else {
       if (!ensure_smem(quant_tile_kernel<false>, static_cast<int>(smem))) return MXS_ERR_CUDA;
-      quant_tile_kernel<false><<<grid, kQuantThreads, smem, s>>>(a, status);
+      launch_pdl(quant_tile_kernel<false>, dim3(grid), dim3(kQuantThreads), smem, s, a, status);
     }
   } else {
     const int lgrid = static_cast<int>(std::min<int64_t>((warps + 7) / 8, static_cast<int64_t>(nsm) * 16));
-    if (f32) quant_lane_kernel<true><<<lgrid, 256, 0, s>>>(a);
-    else quant_lane_kernel<false><<<lgrid, 256, 0, s>>>(a);
+    if (f32) launch_pdl(quant_lane_kernel<true>, dim3(lgrid), dim3(256), 0, s, a);
+    else launch_pdl(quant_lane_kernel<false>, dim3(lgrid), dim3(256), 0, s, a);
   }
   count_launch();
   return cuda_status(cudaGetLastError());
@@ -759,7 +873,7 @@ extern "C" mxs_status mxs_dequantize(const mxs_mxtensor *in, float *out, int64_t
   a.ldo = ldo;
   const int64_t total = a.rows * a.nb_total;
   const int grid = static_cast<int>(std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(sm_count()) * 8));
-  dequant_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  launch_pdl(dequant_kernel, dim3(grid), dim3(256), 0, reinterpret_cast<cudaStream_t>(stream), a);
   count_launch();
   return cuda_status(cudaGetLastError());
 }

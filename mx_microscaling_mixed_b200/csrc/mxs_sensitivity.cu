@@ -116,6 +116,7 @@ __device__ __forceinline__ double q4_err_term_tiny(float w, int e) {
 
 template <bool XF32, bool WF32, bool XVEC, bool WVEC>
 __global__ void __launch_bounds__(kSensThreads) sens_partial_kernel(SensArgs a) {
+  pdl_wait();
   const int64_t gtid = static_cast<int64_t>(blockIdx.x) * kSensThreads + threadIdx.x;
   const int64_t c0 = gtid * kColsPerThread;
   double acc[kColsPerThread];
@@ -229,6 +230,7 @@ template <bool XF32, bool WF32>
 __global__ void __launch_bounds__(kTileThreads)
     sens_tile_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapW, SensArgs a,
                      int32_t ctiles, int *status) {
+  pdl_wait();
   extern __shared__ __align__(128) uint8_t tile[];
   __shared__ __align__(8) uint64_t bar;
   const int nx = a.nchunk_x * ctiles;
@@ -285,6 +287,7 @@ constexpr int kFinSlab = 128;      // chunk partials staged per pass (32 KB)
 // Stages the partials of 32 columns, kFinSlab chunks at a time, with every
 // thread's loads in flight; one warp then adds them in chunk order.
 __global__ void __launch_bounds__(kFinThreads) sens_finalize_kernel(SensArgs a, double *H, double *E, double *s) {
+  pdl_wait();
   __shared__ double sp[kFinSlab][kFinCols];
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kFinCols;
   const int nch = a.nchunk_x + a.nchunk_w;
@@ -317,10 +320,10 @@ __global__ void __launch_bounds__(kFinThreads) sens_finalize_kernel(SensArgs a, 
 
 template <bool XF, bool WF>
 static void launch_partials(const SensArgs &a, bool xvec, bool wvec, dim3 grid, cudaStream_t st) {
-  if (xvec && wvec) sens_partial_kernel<XF, WF, true, true><<<grid, kSensThreads, 0, st>>>(a);
-  else if (xvec) sens_partial_kernel<XF, WF, true, false><<<grid, kSensThreads, 0, st>>>(a);
-  else if (wvec) sens_partial_kernel<XF, WF, false, true><<<grid, kSensThreads, 0, st>>>(a);
-  else sens_partial_kernel<XF, WF, false, false><<<grid, kSensThreads, 0, st>>>(a);
+  if (xvec && wvec) launch_pdl(sens_partial_kernel<XF, WF, true, true>, dim3(grid), dim3(kSensThreads), 0, st, a);
+  else if (xvec) launch_pdl(sens_partial_kernel<XF, WF, true, false>, dim3(grid), dim3(kSensThreads), 0, st, a);
+  else if (wvec) launch_pdl(sens_partial_kernel<XF, WF, false, true>, dim3(grid), dim3(kSensThreads), 0, st, a);
+  else launch_pdl(sens_partial_kernel<XF, WF, false, false>, dim3(grid), dim3(kSensThreads), 0, st, a);
 }
 
 static int64_t chunks(int64_t rows) { return (rows + kSumChunk - 1) / kSumChunk; }
@@ -384,15 +387,15 @@ extern "C" mxs_status mxs_sensitivity(const void *X, mxs_dtype xt, int64_t T, in
       const int32_t ct = static_cast<int32_t>(ctiles);
       if (xf && wf) {
         if (!ensure_smem(sens_tile_kernel<true, true>, smem)) return MXS_ERR_CUDA;
-        sens_tile_kernel<true, true><<<g, kTileThreads, smem, cs>>>(mx, mw, a, ct, status);
+        launch_pdl(sens_tile_kernel<true, true>, dim3(g), dim3(kTileThreads), smem, cs, mx, mw, a, ct, status);
       } else if (xf) {
         if (!ensure_smem(sens_tile_kernel<true, false>, smem)) return MXS_ERR_CUDA;
-        sens_tile_kernel<true, false><<<g, kTileThreads, smem, cs>>>(mx, mw, a, ct, status);
+        launch_pdl(sens_tile_kernel<true, false>, dim3(g), dim3(kTileThreads), smem, cs, mx, mw, a, ct, status);
       } else if (wf) {
         if (!ensure_smem(sens_tile_kernel<false, true>, smem)) return MXS_ERR_CUDA;
-        sens_tile_kernel<false, true><<<g, kTileThreads, smem, cs>>>(mx, mw, a, ct, status);
+        launch_pdl(sens_tile_kernel<false, true>, dim3(g), dim3(kTileThreads), smem, cs, mx, mw, a, ct, status);
       } else {
-        sens_tile_kernel<false, false><<<g, kTileThreads, smem, cs>>>(mx, mw, a, ct, status);
+        launch_pdl(sens_tile_kernel<false, false>, dim3(g), dim3(kTileThreads), smem, cs, mx, mw, a, ct, status);
       }
       tiled = true;
     }
@@ -403,7 +406,7 @@ extern "C" mxs_status mxs_sensitivity(const void *X, mxs_dtype xt, int64_t T, in
     else if (wf) launch_partials<false, true>(a, xvec, wvec, grid, cs);
     else launch_partials<false, false>(a, xvec, wvec, grid, cs);
   }
-  sens_finalize_kernel<<<static_cast<unsigned>((K + kFinCols - 1) / kFinCols), kFinThreads, 0, cs>>>(a, H, E, s);
+  launch_pdl(sens_finalize_kernel, dim3(static_cast<unsigned>((K + kFinCols - 1) / kFinCols)), dim3(kFinThreads), 0, cs, a, H, E, s);
   count_launch(2);
   return cuda_status(cudaGetLastError());
 }

@@ -29,21 +29,36 @@ def _random_layout(c, K, seed, counts=None):
 
 
 def _edge_matrix(rows, K, dtype, seed):
-    """Zeros, fp32 subnormals, exact powers of two, half-step ties, huge and
-    tiny magnitudes, negative block maxima."""
+    """Row r takes pattern r % 8: zeros, fp32 subnormals, exact powers of two,
+    half-step ties, huge magnitudes, negative block maxima, blocks just above
+    the smallest normal scale with subnormal neighbours (where the scaled
+    subnormals decide codes), and a different random scale per block."""
     g = torch.Generator().manual_seed(seed)
     X = torch.randn(rows, K, generator=g)
-    X[0] = 0.0
-    if rows > 1:
-        X[1] = torch.randn(K, generator=g) * 1e-40          # subnormal (bf16 shares fp32's exponent range)
-    if rows > 2:
-        X[2] = 2.0 ** torch.randint(-20, 20, (K,), generator=g).float()
-    if rows > 3:
-        X[3] = (torch.randint(-60, 60, (K,), generator=g).float() + 0.5) * 2.0 ** -6
-    if rows > 4:
-        X[4] = torch.randn(K, generator=g) * 1e37
-    if rows > 5:
-        X[5] = -torch.rand(K, generator=g) - 1.0
+    nbk = (K + 31) // 32
+    for r in range(rows):
+        kind = r % 8
+        if kind == 0:
+            X[r] = 0.0
+        elif kind == 1:
+            X[r] = torch.randn(K, generator=g) * 1e-40          # subnormal (bf16 shares fp32's exponent range)
+        elif kind == 2:
+            X[r] = 2.0 ** torch.randint(-20, 20, (K,), generator=g).float()
+        elif kind == 3:
+            X[r] = (torch.randint(-60, 60, (K,), generator=g).float() + 0.5) * 2.0 ** -6
+        elif kind == 4:
+            X[r] = torch.randn(K, generator=g) * 1e37
+        elif kind == 5:
+            X[r] = -torch.rand(K, generator=g) - 1.0
+        elif kind == 6:
+            e = torch.randint(-127, -119, (nbk,), generator=g).float().repeat_interleave(32)[:K]
+            x = torch.randn(K, generator=g) * 2.0 ** e
+            sub = torch.rand(K, generator=g) < 0.5
+            x[sub] = torch.randint(-127, 128, (int(sub.sum()),), generator=g).float() * 2.0 ** -133
+            X[r] = x
+        else:
+            e = torch.randint(-130, 120, (nbk,), generator=g).float().repeat_interleave(32)[:K]
+            X[r] = torch.randn(K, generator=g) * 2.0 ** e
     return X.to(dtype)
 
 
@@ -58,6 +73,8 @@ CASES = [
     (3, 30000, torch.float32, (32, 960, 29008), "random"),   # too large to stage: direct path
     (5, 33, torch.bfloat16, (1, 0, 32), "random"),
     (64, 4096, torch.bfloat16, (32, 960, 3104), "random"),
+    (320, 1024, torch.bfloat16, None, "edge"),               # staged path (more than 8192 blocks)
+    (320, 1024, torch.float32, None, "edge"),
 ]
 
 
@@ -92,6 +109,18 @@ def test_kv_identity_layout(c, rows, K):
     c.mxs_quantize_act(src, t)
     oc, os_ = oracle.quantize_rows(parity.host64(src), None, (0, 0, K))
     parity.assert_codes_equal(t, oc, os_, "kv")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_identity_layout_edge(c, dtype):
+    """Unpermuted mixed layout on the direct path, edge values in every width."""
+    rows, K, counts = 320, 1024, (96, 200, 728)
+    src = _edge_matrix(rows, K, dtype, seed=5).cuda()
+    lay = c.mxs_layout_make(K, counts)
+    t = c.mxtensor_empty(rows, lay)
+    c.mxs_quantize_act(src, t)
+    oc, os_ = oracle.quantize_rows(parity.host64(src), None, counts)
+    parity.assert_codes_equal(t, oc, os_, "identity edge")
 
 
 def test_kv_cache_shape(c):

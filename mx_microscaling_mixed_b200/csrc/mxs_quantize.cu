@@ -143,6 +143,51 @@ struct QuantArgs {
   int32_t units_per_batch; // (rows_per_batch / G) * (quads[0] + quads[1] + quads[2])
 };
 
+// Maximum of |v[0..31]| (bit patterns of |x|, or of each 16-bit half),
+// as a five-level tree: the chain of dependent max operations is 5 long.
+__device__ __forceinline__ float absmax32(const float (&v)[kBlock]) {
+  float m[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) m[i] = fmaxf(fabsf(v[i]), fabsf(v[i + 16]));
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
+  return m[0];
+}
+// Packed bf16x2 magnitude max / min: max(|a|, |b|) or min(|a|, |b|) per
+// half, carrying the XOR of the operands' signs (finite operands).
+__device__ __forceinline__ uint32_t maxabs_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t minabs_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("min.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+// Per half: the largest |x| over p[0..N-1], as bf16 bits with the sign clear.
+template <int N>
+__device__ __forceinline__ uint32_t absmax_u16x2(const uint32_t (&p)[N]) {
+  uint32_t m[N / 2];
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) m[i] = maxabs_bf16x2(p[i], p[i + N / 2]);
+#pragma unroll
+  for (int w = N / 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) m[i] = maxabs_bf16x2(m[i], m[i + w]);
+  return m[0] & 0x7FFF7FFFu;
+}
+// bf16 bits of (2^(m-1) - 1) * 2^-k, the largest magnitude that codes
+// below the clamp at width m (k in [-125, 128]).
+template <int M>
+__device__ __forceinline__ uint32_t clamp_bits(int k) {
+  static_assert(M == 4 || M == 6, "packed path for 4- and 6-bit codes");
+  return M == 4 ? (static_cast<uint32_t>(2 - k + 127) << 7) | 0x60u      // 7 = 1.75 * 2^2
+                : (static_cast<uint32_t>(4 - k + 127) << 7) | 0x78u;     // 31 = 1.9375 * 2^4
+}
+
 constexpr uint32_t kMagic = 0x4B400000u;   // bits of 1.5 * 2^23: x + it rounds x to an integer, ties to even
 
 // Codes one block: v[] holds the 32 values of the block in position order.
@@ -152,9 +197,7 @@ constexpr uint32_t kMagic = 0x4B400000u;   // bits of 1.5 * 2^23: x + it rounds 
 // patterns as unsigned integers.
 template <int M>
 __device__ __forceinline__ void encode_store(float (&v)[kBlock], uint8_t *cdst, uint8_t *sdst) {
-  float amax = 0.f;
-#pragma unroll
-  for (int t = 0; t < kBlock; ++t) amax = fmaxf(amax, fabsf(v[t]));
+  const float amax = absmax32(v);
   const int ef = static_cast<int>(__float_as_uint(amax) >> 23);   // E8M0 byte of the block
   int k = M - 2 - (ef == 0 ? -127 : ef - 127);
   if (k > 127) {                     // blocks below 2^-121: pre-scale by 2^64 (exact)
@@ -208,13 +251,14 @@ __device__ __forceinline__ void encode_store(float (&v)[kBlock], uint8_t *cdst, 
 
 // bf16 source, 4- and 6-bit codes: the same rule on packed pairs.  p[i]
 // holds positions 2i (low half) and 2i+1 (high half) as bf16 bits.  The
-// block maximum is an unsigned 16-bit max of the bit patterns with the sign
-// cleared (monotonic in |x|), so the E8M0 byte is its exponent field, as
-// for fp32.  Rounding: one bf16x2 fma x*2^k + 192 (a single rounding of the
-// exact value; 192 + q stays in [128, 256), where bf16 steps by 1) leaves
-// the lane's bits at 0x4340 + q, so clamping is an unsigned 16-bit min/max
-// and the code is the low m bits.  When k > 125 the block is tiny and takes
-// the fp32 path, so that subnormal inputs never meet the bf16 fma.
+// block maximum is a bf16x2 max of the magnitudes, so the E8M0 byte is its
+// exponent field, as for fp32.  The clamp comes first, on the magnitude:
+// |x| is cut to L * 2^-k (L = 2^(m-1) - 1, sign kept), which codes to the
+// same integer as clamping after the rounding.  Rounding: one bf16x2 fma
+// x*2^k + 192 (a single rounding of the exact value; 192 + q stays in
+// [128, 256), where bf16 steps by 1) leaves the lane's bits at 0x4340 + q,
+// and the code is the low m bits.  When k > 125 the block is tiny and takes the fp32
+// path, so that subnormal inputs never reach the bf16 fma.
 __device__ __forceinline__ uint32_t fma_bf16x2(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t d;
   asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
@@ -224,9 +268,7 @@ __device__ __forceinline__ uint32_t fma_bf16x2(uint32_t a, uint32_t b, uint32_t 
 template <int M>
 __device__ __forceinline__ void encode_store_bf16(const uint32_t (&p)[kBlock / 2], uint8_t *cdst, uint8_t *sdst) {
   static_assert(M == 4 || M == 6, "packed path for 4- and 6-bit codes");
-  uint32_t m2 = 0;
-#pragma unroll
-  for (int i = 0; i < kBlock / 2; ++i) m2 = __vmaxu2(m2, p[i] & 0x7FFF7FFFu);
+  const uint32_t m2 = absmax_u16x2(p);
   const int ef = static_cast<int>(max(m2 & 0xFFFFu, m2 >> 16) >> 7);
   const int k = M - 2 - (ef == 0 ? -127 : ef - 127);
   if (k > 125) {
@@ -241,11 +283,11 @@ __device__ __forceinline__ void encode_store_bf16(const uint32_t (&p)[kBlock / 2
   }
   const uint32_t sb = static_cast<uint32_t>(k + 127) << 7;
   const uint32_t s2 = sb | (sb << 16);
-  constexpr uint32_t L = (1u << (M - 1)) - 1u;
-  constexpr uint32_t lo2 = (0x4340u - L) * 0x10001u, hi2 = (0x4340u + L) * 0x10001u;
+  const uint32_t cb = clamp_bits<M>(k);
+  const uint32_t c2 = cb | (cb << 16);
   uint32_t r[kBlock / 2];
 #pragma unroll
-  for (int i = 0; i < kBlock / 2; ++i) r[i] = __vminu2(__vmaxu2(fma_bf16x2(p[i], s2, 0x43404340u), lo2), hi2);
+  for (int i = 0; i < kBlock / 2; ++i) r[i] = fma_bf16x2(minabs_bf16x2(p[i], c2), s2, 0x43404340u);
   *sdst = static_cast<uint8_t>(ef);
   if constexpr (M == 4) {
     // bytes of positions 4j..4j+3 (low byte of each lane), then each
@@ -510,6 +552,395 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quant_tile_kernel(QuantArgs 
       if (it >= 0) ptx::mbar_wait_cycles(&bar[st], (it / kQStages) & 1, kQuantWaitLimit);
     }
   }
+}
+
+// ------------------------------------------- transposed quantiser (bf16)
+//
+// For bf16 sources with a permuted layout.  A batch is 8 source rows, bulk
+// copied (one copy per row) into a row-major buffer.  Four transposer warps
+// turn it, 8 x 8 at a time (ldmatrix .trans, stmatrix), into a copy T in
+// which each column of the batch is 16 contiguous bytes: rows 2p and 2p+1
+// form 32-bit word p.  The coding warps then gather a block's 32 positions
+// for two rows with one 32-bit load each and code both rows at once in
+// packed bf16 pairs (one row per half).  T is double-buffered, so the
+// transposers fill the next batch while the coders drain this one; coders
+// take 32-lane units (4 row pairs x 8 blocks of one segment) from a shared
+// counter.  Within a segment the layout keeps the columns in ascending
+// order, so in a dense segment the 8 blocks of a unit read columns 32
+// apart; T therefore stores column c in slot c ^ ((c >> 3 ^ c >> 6) & 7) of
+// its 8-column group, which spreads such strides over the banks.  Hand-off: monotone
+// counters in shared memory, the transposers publishing the batch a buffer
+// holds and the coders counting finished units per buffer.
+
+constexpr int kTrRows = 8;                 // rows per batch
+constexpr int kTrThreads = 640;
+constexpr int kTrTransposers = 4;          // warps 0..3
+
+struct TrArgs {
+  QuantArgs q;
+  int32_t kc;             // columns of T holding data (K rounded up to 32); column kc is zero
+  int32_t nt;             // T buffers (1 or 2)
+  int32_t pitch;          // bytes per staged source row (16 mod 128)
+  int32_t units[3];       // coding units per batch in each segment
+  int32_t U;              // units per batch
+  uint32_t U_magic;       // floor(2^32 / U) + 1 (0 when U == 1)
+  int32_t t_off, raw_off, tab_off;   // shared-memory layout (bytes)
+};
+
+// T slot of column c (a bijection within each aligned group of 8 columns).
+__host__ __device__ inline int32_t tr_slot(int32_t c) { return (c & ~7) | ((c ^ (c >> 3) ^ (c >> 6)) & 7); }
+__host__ __device__ inline int64_t tr_t_bytes(int64_t kc) { return (kc + 8) * 16; }
+
+// Both rows of a T word pair (low half: row 2p, high half: row 2p+1) coded
+// at width M into their own rows.  Per row the rule is that of
+// encode_store_bf16; rows whose block is tiny take the fp32 coder.
+template <int M>
+__device__ __forceinline__ void encode2_store(const uint32_t (&v)[kBlock], uint8_t *c0, uint8_t *s0, uint8_t *c1,
+                                              uint8_t *s1, bool has1) {
+  const uint32_t m2 = absmax_u16x2(v);
+  const int ef0 = static_cast<int>((m2 & 0xFFFFu) >> 7), ef1 = static_cast<int>(m2 >> 23);
+  const int k0 = M - 2 - (ef0 == 0 ? -127 : ef0 - 127), k1 = M - 2 - (ef1 == 0 ? -127 : ef1 - 127);
+  if (M == 8 || k0 > 125 || k1 > 125) {
+    float x[kBlock];
+#pragma unroll
+    for (int t = 0; t < kBlock; ++t) x[t] = __uint_as_float(v[t] << 16);
+    encode_store<M>(x, c0, s0);
+    if (has1) {
+#pragma unroll
+      for (int t = 0; t < kBlock; ++t) x[t] = __uint_as_float(v[t] & 0xFFFF0000u);
+      encode_store<M>(x, c1, s1);
+    }
+    return;
+  }
+  if constexpr (M != 8) {
+    const uint32_t s2 = (static_cast<uint32_t>(k0 + 127) << 7) | (static_cast<uint32_t>(k1 + 127) << 23);
+    const uint32_t c2 = clamp_bits<M>(k0) | (clamp_bits<M>(k1) << 16);
+    uint32_t r[kBlock];
+#pragma unroll
+    for (int t = 0; t < kBlock; ++t) r[t] = fma_bf16x2(minabs_bf16x2(v[t], c2), s2, 0x43404340u);
+    *s0 = static_cast<uint8_t>(ef0);
+    if (has1) *s1 = static_cast<uint8_t>(ef1);
+    // x0[j] / x1[j]: the low bytes of positions 4j..4j+3 of row 0 / row 1
+    uint32_t x0[8], x1[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t A = __byte_perm(r[4 * j], r[4 * j + 1], 0x6240);
+      const uint32_t B = __byte_perm(r[4 * j + 2], r[4 * j + 3], 0x6240);
+      x0[j] = __byte_perm(A, B, 0x5410);
+      x1[j] = __byte_perm(A, B, 0x7632);
+    }
+    if constexpr (M == 4) {
+      uint32_t w0[4], w1[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t a0 = (x0[2 * j] & 0x0F0F0F0Fu) | ((x0[2 * j] >> 4) & 0xF0F0F0F0u);
+        const uint32_t b0 = (x0[2 * j + 1] & 0x0F0F0F0Fu) | ((x0[2 * j + 1] >> 4) & 0xF0F0F0F0u);
+        w0[j] = __byte_perm(a0, b0, 0x6420);
+        const uint32_t a1 = (x1[2 * j] & 0x0F0F0F0Fu) | ((x1[2 * j] >> 4) & 0xF0F0F0F0u);
+        const uint32_t b1 = (x1[2 * j + 1] & 0x0F0F0F0Fu) | ((x1[2 * j + 1] >> 4) & 0xF0F0F0F0u);
+        w1[j] = __byte_perm(a1, b1, 0x6420);
+      }
+      *reinterpret_cast<uint4 *>(c0) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+      if (has1) *reinterpret_cast<uint4 *>(c1) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+    } else {
+      uint32_t u0[8], u1[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t z0 = (x0[j] & 0x003F003Fu) | ((x0[j] >> 2) & 0x0FC00FC0u);
+        u0[j] = (z0 & 0xFFFu) | ((z0 >> 4) & 0xFFF000u);
+        const uint32_t z1 = (x1[j] & 0x003F003Fu) | ((x1[j] >> 2) & 0x0FC00FC0u);
+        u1[j] = (z1 & 0xFFFu) | ((z1 >> 4) & 0xFFF000u);
+      }
+      uint32_t w0[6], w1[6];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        w0[3 * h] = u0[4 * h] | (u0[4 * h + 1] << 24);
+        w0[3 * h + 1] = (u0[4 * h + 1] >> 8) | (u0[4 * h + 2] << 16);
+        w0[3 * h + 2] = (u0[4 * h + 2] >> 16) | (u0[4 * h + 3] << 8);
+        w1[3 * h] = u1[4 * h] | (u1[4 * h + 1] << 24);
+        w1[3 * h + 1] = (u1[4 * h + 1] >> 8) | (u1[4 * h + 2] << 16);
+        w1[3 * h + 2] = (u1[4 * h + 2] >> 16) | (u1[4 * h + 3] << 8);
+      }
+      uint2 *q0 = reinterpret_cast<uint2 *>(c0);
+      q0[0] = make_uint2(w0[0], w0[1]);
+      q0[1] = make_uint2(w0[2], w0[3]);
+      q0[2] = make_uint2(w0[4], w0[5]);
+      if (has1) {
+        uint2 *q1 = reinterpret_cast<uint2 *>(c1);
+        q1[0] = make_uint2(w1[0], w1[1]);
+        q1[1] = make_uint2(w1[2], w1[3]);
+        q1[2] = make_uint2(w1[4], w1[5]);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(ptx::smem_addr(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void stsm_x4(uint32_t addr, const uint32_t (&r)[4]) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(r[0]), "r"(r[1]),
+               "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// Bounded poll of a shared counter until it reaches `want` (monotone).
+__device__ __forceinline__ bool spin_until_at_least(volatile int *p, int want, long long limit) {
+  if (*p >= want) return true;
+  const long long t0 = clock64();
+  unsigned ns = 32;
+  while (*p < want) {
+    if (clock64() - t0 > limit) return false;
+    __nanosleep(ns);
+    ns = min(ns * 2, 256u);
+  }
+  return true;
+}
+
+// All-or-nothing decision of the transposer warps: every thread of the
+// 128 passes its flag; every thread returns the OR.
+__device__ __forceinline__ bool transposers_any(bool f) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(f))
+      : "memory");
+  return r != 0;
+}
+
+// Warp-wide: bulk-copies the rows of local batch i into the staging
+// buffer, one row per lane, completing on `bar`.  The buffer's previous
+// batch was read into registers and written to T before the transposers'
+// barrier that precedes this call, so the copies overwrite nothing that is
+// still to be read.
+__device__ __forceinline__ void tr_issue_batch(const TrArgs &ta, int i, int nloc, uint8_t *raw, uint64_t *bar) {
+  const QuantArgs &a = ta.q;
+  const int lane = threadIdx.x & 31;
+  const int64_t r0 = (blockIdx.x + static_cast<int64_t>(i) * gridDim.x) * kTrRows;
+  const int nr = static_cast<int>(min(static_cast<int64_t>(kTrRows), a.rows - r0));
+  const uint32_t bytes = static_cast<uint32_t>(a.K) * 2;
+  const uint8_t *src = reinterpret_cast<const uint8_t *>(a.src);
+  if (lane == 0) ptx::mbar_arrive_expect_tx(bar, bytes * nr);
+  __syncwarp();
+  if (lane < nr) ptx::bulk_load(raw + lane * ta.pitch, src + (r0 + lane) * a.ld * 2, bytes, bar);
+  // the batch after: into L2 now, so that its copies wait on L2 only
+  if (i + 1 < nloc) {
+    const int64_t r1 = r0 + static_cast<int64_t>(gridDim.x) * kTrRows;
+    if (lane < kTrRows && r1 + lane < a.rows)
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src + (r1 + lane) * a.ld * 2), "r"(bytes)
+                   : "memory");
+  }
+}
+
+__global__ void __launch_bounds__(kTrThreads, 1) quant_tr_kernel(TrArgs ta, int *status) {
+  pdl_wait();
+  extern __shared__ __align__(128) uint8_t smem[];
+  const QuantArgs &a = ta.q;
+  uint32_t *tab = reinterpret_cast<uint32_t *>(smem + ta.tab_off);
+  uint8_t *tbuf = smem + ta.t_off;
+  uint8_t *raw = smem + ta.raw_off;
+  __shared__ __align__(8) uint64_t raw_full;
+  __shared__ int next_unit, abort_flag;
+  __shared__ int ready[2], done[2];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t nbatches = (a.rows + kTrRows - 1) / kTrRows;
+  const int nloc = blockIdx.x < nbatches ? static_cast<int>((nbatches - blockIdx.x + gridDim.x - 1) / gridDim.x) : 0;
+  const int64_t tbytes = round_up(tr_t_bytes(ta.kc), 128);
+  volatile int *vabort = &abort_flag;
+
+  if (threadIdx.x == 0) {
+    next_unit = 0;
+    abort_flag = 0;
+    ready[0] = ready[1] = -1;
+    done[0] = done[1] = 0;
+    ptx::mbar_init(&raw_full, 1);
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == 0 && nloc > 0) tr_issue_batch(ta, 0, nloc, raw, &raw_full);
+  // gather table: T byte offset (slot * 16) of each layout position's
+  // column, the zero column for padding; every position's permutation load
+  // is independent, 8 in flight per thread
+  const int npos = a.nb_total * kBlock;
+  for (int p0 = threadIdx.x; p0 < npos; p0 += 8 * kTrThreads) {
+    int col[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int pa = p0 + u * kTrThreads;
+      const int g = pa < a.boff[1] * kBlock ? 0 : (pa < a.boff[2] * kBlock ? 1 : 2);
+      const int p = pa - a.boff[g] * kBlock;
+      col[u] = ta.kc;
+      if (pa < npos && p < a.k_real[g]) col[u] = __ldg(a.perm + a.real_off[g] + p);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int pa = p0 + u * kTrThreads;
+      if (pa < npos) tab[(pa >> 5) * kTabWordsPerBlock + (pa & 31)] = static_cast<uint32_t>(tr_slot(col[u])) * 16u;
+    }
+  }
+  if (threadIdx.x < ta.nt)
+    *reinterpret_cast<uint4 *>(tbuf + threadIdx.x * tbytes + tr_slot(ta.kc) * 16) = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+
+  if (warp < kTrTransposers) {
+    const int ngroups = ta.kc / 32;
+    const int m = lane >> 3, r = lane & 7;
+    const uint32_t raw_row = ptx::smem_addr(raw + r * ta.pitch + 16 * m);
+    int inflight = nloc > 0 ? 0 : -1;                 // batch whose rows are being copied
+    for (int i = 0; i < nloc; ++i) {
+      const int s = ta.nt == 2 ? (i & 1) : 0;
+      const uint32_t T = ptx::smem_addr(tbuf + s * tbytes) + 128 * m;
+      // T[s] is free once every unit of the batches it held is done; the
+      // batch's rows have landed
+      bool bad = false;
+      // (one thread waits; the others take the completed phase after the
+      // barrier, which a non-blocking test then observes at once)
+      if (threadIdx.x == 0)
+        bad = !spin_until_at_least(&done[s], (ta.nt == 2 ? (i >> 1) : i) * ta.U, kQuantWaitLimit) ||
+              !ptx::mbar_wait_cycles(&raw_full, i & 1, kQuantWaitLimit);
+      if (transposers_any(bad || *vabort)) {
+        if (threadIdx.x == 0) *vabort = 1;
+        break;
+      }
+      if (threadIdx.x != 0 && !mbar_test_wait(&raw_full, i & 1)) ptx::mbar_wait_cycles(&raw_full, i & 1, kQuantWaitLimit);
+      inflight = -1;
+      __threadfence_block();
+      for (int g0 = warp; g0 < ngroups; g0 += 4 * kTrTransposers) {
+        uint32_t v[4][4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int gi = g0 + k * kTrTransposers;
+          if (gi < ngroups) ldsm_x4_trans(raw_row + gi * 64, v[k]);
+        }
+        // stmatrix writes row r of matrix m, i.e. T column c = 32 gi + 8 m + r,
+        // at the address this lane gives: the slot keeps the group (c & ~7)
+        // and XORs the low 3 bits with (c >> 3 ^ c >> 6)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int gi = g0 + k * kTrTransposers;
+          if (gi < ngroups) {
+            const uint32_t h = static_cast<uint32_t>((4 * gi + m) ^ (gi >> 1)) & 7u;
+            stsm_x4(T + static_cast<uint32_t>(gi) * 512 + ((static_cast<uint32_t>(r) ^ h) << 4), v[k]);
+          }
+        }
+      }
+      // every transposer is done: the batch is published and the staging
+      // buffer takes the next batch
+      transposers_any(false);
+      if (threadIdx.x == 0) {
+        __threadfence_block();
+        *reinterpret_cast<volatile int *>(&ready[s]) = i;
+      }
+      if (i + 1 < nloc) {
+        if (warp == 0) tr_issue_batch(ta, i + 1, nloc, raw, &raw_full);
+        inflight = i + 1;
+      }
+    }
+    // an aborted run leaves no bulk copy in flight
+    if (threadIdx.x == 0 && inflight >= 0) ptx::mbar_wait_cycles(&raw_full, inflight & 1, kQuantWaitLimit);
+  } else {
+    const int total = nloc * ta.U;
+    for (;;) {
+      int v = 0;
+      if (lane == 0) v = atomicAdd(&next_unit, 1);
+      v = __shfl_sync(0xffffffffu, v, 0);
+      if (v >= total || *vabort) break;
+      const int i = ta.U == 1 ? v : static_cast<int>(__umulhi(static_cast<uint32_t>(v), ta.U_magic));
+      const int u = v - i * ta.U;
+      const int s = ta.nt == 2 ? (i & 1) : 0;
+      int ok = 1;
+      if (lane == 0) {
+        const long long t0 = clock64();
+        unsigned ns = 32;
+        while (*reinterpret_cast<volatile int *>(&ready[s]) < i) {
+          if (*vabort || clock64() - t0 > kQuantWaitLimit) {
+            ok = 0;
+            break;
+          }
+          __nanosleep(ns);
+          ns = min(ns * 2, 64u);
+        }
+        __threadfence_block();
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        if (lane == 0) *vabort = 1;
+        break;
+      }
+      int g = 0, qd = u;
+      if (qd >= ta.units[0]) {
+        qd -= ta.units[0];
+        g = 1;
+        if (qd >= ta.units[1]) {
+          qd -= ta.units[1];
+          g = 2;
+        }
+      }
+      const int pr = lane & 3, bb = qd * 8 + (lane >> 2);
+      const int64_t r0 = (blockIdx.x + static_cast<int64_t>(i) * gridDim.x) * kTrRows + 2 * pr;
+      if (bb < a.nb[g] && r0 < a.rows) {
+        const uint32_t T = ptx::smem_addr(tbuf + s * tbytes) + pr * 4;
+        const uint32_t tw = ptx::smem_addr(tab + (a.boff[g] + bb) * kTabWordsPerBlock);
+        uint32_t x[kBlock];
+#pragma unroll
+        for (int j = 0; j < kBlock / 4; ++j) {
+          const uint4 w = lds128(tw + 16 * j);
+          x[4 * j] = lds32(T + w.x);
+          x[4 * j + 1] = lds32(T + w.y);
+          x[4 * j + 2] = lds32(T + w.z);
+          x[4 * j + 3] = lds32(T + w.w);
+        }
+        const bool has1 = r0 + 1 < a.rows;
+        uint8_t *s0 = a.scales[g] + r0 * a.spitch[g] + bb;
+        if (g == 0) {
+          uint8_t *c0 = a.codes[0] + r0 * a.cpitch[0] + bb * 32;
+          encode2_store<8>(x, c0, s0, c0 + a.cpitch[0], s0 + a.spitch[0], has1);
+        } else if (g == 1) {
+          uint8_t *c0 = a.codes[1] + r0 * a.cpitch[1] + bb * 24;
+          encode2_store<6>(x, c0, s0, c0 + a.cpitch[1], s0 + a.spitch[1], has1);
+        } else {
+          uint8_t *c0 = a.codes[2] + r0 * a.cpitch[2] + bb * 16;
+          encode2_store<4>(x, c0, s0, c0 + a.cpitch[2], s0 + a.spitch[2], has1);
+        }
+      }
+      // every lane's reads of T are done before the unit counts as finished
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence_block();
+        atomicAdd(&done[s], 1);
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && *vabort) atomicExch(status, static_cast<int>(MXS_ERR_TIMEOUT));
 }
 
 // Identity layout: one thread per (row, block), values read straight from
@@ -790,9 +1221,41 @@ static mxs_status quantize_impl(const void *src, mxs_dtype dt, int64_t rows, int
     count_launch();
     return cuda_status(cudaGetLastError());
   }
-  // tiled path: rows bulk-copyable (16-byte aligned base, pitch and row
+  // staged paths: rows bulk-copyable (16-byte aligned base, pitch and row
   // length) and small enough to stage
   const bool vec_rows = aligned16(src) && (ld * es) % 16 == 0 && (a.K * es) % 16 == 0;
+  if (!tiny && vec_rows && !f32) {
+    // transposed path when two column-major copies of a batch, its staged
+    // rows and the gather table fit
+    TrArgs ta{};
+    ta.kc = static_cast<int32_t>(round_up(a.K, 32));
+    ta.pitch = static_cast<int32_t>(round_up(static_cast<int64_t>(a.K) * 2, 128) + 16);
+    const int64_t tb = round_up(tr_t_bytes(ta.kc), 128);
+    const int64_t tab = quant_table_bytes(a.nb_total);
+    const int64_t rawb = round_up(static_cast<int64_t>(kTrRows) * ta.pitch, 128);
+    ta.nt = tab + 2 * tb + rawb <= kQuantSmemBudget ? 2 : 0;
+    if (ta.nt > 0) {
+      ta.q = a;
+      ta.U = 0;
+      for (int g = 0; g < 3; ++g) {
+        ta.units[g] = (a.nb[g] + 7) / 8;
+        ta.U += ta.units[g];
+      }
+      ta.U_magic = ta.U > 1 ? static_cast<uint32_t>((1ull << 32) / static_cast<uint64_t>(ta.U) + 1) : 0u;
+      ta.tab_off = 0;
+      ta.t_off = static_cast<int32_t>(tab);
+      ta.raw_off = static_cast<int32_t>(tab + ta.nt * tb);
+      const int64_t tsmem = ta.raw_off + rawb;
+      const int64_t nbatches = (rows + kTrRows - 1) / kTrRows;
+      const int tgrid = static_cast<int>(std::min<int64_t>(nsm, nbatches));
+      int *status = device_status_word();
+      if (!status) return MXS_ERR_CUDA;
+      if (!ensure_smem(quant_tr_kernel, static_cast<int>(tsmem))) return MXS_ERR_CUDA;
+      launch_pdl(quant_tr_kernel, dim3(tgrid), dim3(kTrThreads), tsmem, s, ta, status);
+      count_launch();
+      return cuda_status(cudaGetLastError());
+    }
+  }
   bool tiled = !tiny && vec_rows;
   int64_t smem = 0;
   int grid = 0;

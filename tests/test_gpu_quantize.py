@@ -75,6 +75,9 @@ CASES = [
     (64, 4096, torch.bfloat16, (32, 960, 3104), "random"),
     (320, 1024, torch.bfloat16, None, "edge"),               # staged path (more than 8192 blocks)
     (320, 1024, torch.float32, None, "edge"),
+    (333, 1000, torch.bfloat16, None, "random"),             # ragged last batch and last piece
+    (1001, 520, torch.bfloat16, None, "edge"),               # odd rows: a lone row in the last pair
+    (2048, 4096, torch.bfloat16, (32, 960, 3104), "random"),  # the attention projection's activations
 ]
 
 
@@ -91,6 +94,14 @@ def test_quantize_matches_oracle(c, rows, K, dtype, counts, kind):
         t, oc, os_ = parity.quantize_both(c, src, lay, perm, counts, weight)
         torch.cuda.synchronize()
         parity.assert_codes_equal(t, oc, os_, what=f"{kind} weight={weight}")
+
+
+def test_strided_rows_staged(c):
+    wide = inputs.random_matrix(400, 1024, device="cuda", seed=5, dtype=torch.bfloat16)
+    src = wide[:, :1000]                     # pitch 1024 elements, K = 1000, staged path
+    lay, perm, counts = _random_layout(c, 1000, seed=6)
+    t, oc, os_ = parity.quantize_both(c, src, lay, perm, counts, weight=True)
+    parity.assert_codes_equal(t, oc, os_, "strided staged")
 
 
 def test_strided_rows(c):

@@ -42,6 +42,7 @@ constexpr int kRankSlice = kRankTile / kRankParts;
 // slice holding j compares indices.
 __global__ void __launch_bounds__(kRankThreads) rank_kernel(const double *s, int64_t K, int32_t *rank) {
   pdl_wait();
+  pdl_trigger();
   __shared__ double tile[kRankTile];
   __shared__ int part_cnt[kRankParts][kRankCols];
   const int c = threadIdx.x % kRankCols, part = threadIdx.x / kRankCols;
@@ -79,6 +80,7 @@ __global__ void __launch_bounds__(kRankThreads) rank_kernel(const double *s, int
 
 __global__ void order_kernel(const int32_t *rank, int64_t K, int32_t *order) {
   pdl_wait();
+  pdl_trigger();
   const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (j < K) order[rank[j]] = static_cast<int32_t>(j);
 }
@@ -87,6 +89,7 @@ __global__ void order_kernel(const int32_t *rank, int64_t K, int32_t *order) {
 __global__ void group_gain_kernel(const double *s, const int32_t *order, int64_t K, int64_t n8,
                                   int64_t ngroups, double *gains) {
   pdl_wait();
+  pdl_trigger();
   const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (g >= ngroups) return;
   const int64_t r0 = n8 + 32 * g, r1 = min(r0 + 32, K);
@@ -104,6 +107,7 @@ constexpr int kPermThreads = 1024;
 __global__ void __launch_bounds__(kPermThreads) perm_kernel(const int32_t *rank, int64_t K, int64_t n8,
                                                             int64_t n6, int32_t *perm) {
   pdl_wait();
+  pdl_trigger();
   __shared__ unsigned long long warp_tot[kPermThreads / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t ipt = (K + kPermThreads - 1) / kPermThreads;

@@ -110,6 +110,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                    const __grid_constant__ CUtensorMap tmA8, const __grid_constant__ CUtensorMap tmB8,
                    GemmArgs g) {
   pdl_wait();
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + GemmSmem::bar_off);
@@ -372,7 +373,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA16, const __grid_constant__ CUtensorMap tmB16,
                     const __grid_constant__ CUtensorMap tmA8, const __grid_constant__ CUtensorMap tmB8,
                     const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB, P2Args g) {
-  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + P2Smem::bar_off);
@@ -406,10 +407,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
     ptx::tmem_alloc2(tmem_slot, kTmemCols);
     ptx::tmem_relinquish2();
   }
+  if (threadIdx.x == 32) {
+    const CUtensorMap *maps[6] = {&tmA16, &tmB16, &tmA8, &tmB8, &tmSFA, &tmSFB};
+    for (int i = 0; i < 6; ++i) asm volatile("prefetch.tensormap [%0];" ::"l"(maps[i]) : "memory");
+  }
   ptx::tc_fence_before();
   ptx::cluster_sync();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the staged operands and Y belong to earlier kernels in the stream
+  pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -682,6 +689,7 @@ __device__ __forceinline__ void stage_wide_block(const uint8_t *c, uint8_t sbyte
 // as one word of the tensor core's 512-byte chunk layout.
 __global__ void __launch_bounds__(256) gemm_stage_kernel(StageArgs a) {
   pdl_wait();
+  pdl_trigger();
   __shared__ uint16_t lut[256];                        // byte of two 4-bit codes -> their E4M3 pair (q/4)
   {
     const int b = threadIdx.x;
@@ -963,6 +971,7 @@ constexpr long long kDecWaitLimit = 2000000000LL;    // cycles (~1 s)
 // then run the three segments and add their partial sums in warp order.
 __global__ void __launch_bounds__(kDecThreads) gemm_small_kernel(SmallArgs a, int *status) {
   pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t bar;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;

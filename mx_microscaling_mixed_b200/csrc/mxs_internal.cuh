@@ -49,12 +49,14 @@ inline bool ensure_smem(Kernel k, int bytes) {
 }
 
 // Programmatic dependent launch.  Every kernel of the library is launched
-// with programmatic stream serialisation, so the hardware may schedule it
-// while the previous kernel in the stream is still draining; each kernel's
-// first statement is pdl_wait(), which returns once that previous kernel
-// has completed and its memory operations are visible.  No kernel signals
-// its dependents early, so a waiting grid never holds resources that the
-// grid it waits for still needs.
+// with programmatic stream serialisation and calls pdl_trigger() at its
+// start, so the next kernel in the stream may be scheduled once every CTA
+// of this one is running (none of this grid is still waiting for an SM, so
+// the early CTAs take only resources this grid does not need).  Before its
+// first access to global memory, each kernel calls pdl_wait(), which
+// returns once the previous kernel has completed and its memory operations
+// are visible; only setup that touches no global memory (barriers, tensor
+// memory, descriptor prefetch) may come before it.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                               Args &&...args) {
@@ -73,6 +75,7 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 
 // ---------------------------------------------------------------- device side
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);

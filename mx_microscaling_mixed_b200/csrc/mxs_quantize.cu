@@ -424,6 +424,7 @@ __device__ __forceinline__ bool spin_until_equal(volatile int *p, int want, long
 template <bool F32>
 __global__ void __launch_bounds__(kQuantThreads, 1) quant_tile_kernel(QuantArgs a, int *status) {
   pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int ES = F32 ? 4 : 2;
   uint32_t *tab = reinterpret_cast<uint32_t *>(smem);
@@ -763,6 +764,7 @@ __device__ __forceinline__ void tr_issue_batch(const TrArgs &ta, int i, int nloc
 
 __global__ void __launch_bounds__(kTrThreads, 1) quant_tr_kernel(TrArgs ta, int *status) {
   pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(128) uint8_t smem[];
   const QuantArgs &a = ta.q;
   uint32_t *tab = reinterpret_cast<uint32_t *>(smem + ta.tab_off);
@@ -949,6 +951,7 @@ __global__ void __launch_bounds__(kTrThreads, 1) quant_tr_kernel(TrArgs ta, int 
 template <bool F32>
 __global__ void __launch_bounds__(256) quant_contig_kernel(QuantArgs a) {
   pdl_wait();
+  pdl_trigger();
   constexpr int ES = F32 ? 4 : 2;
   const int64_t total = a.rows * a.nb_total;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
@@ -1014,6 +1017,7 @@ __global__ void __launch_bounds__(256) quant_contig_kernel(QuantArgs a) {
 template <bool F32>
 __global__ void __launch_bounds__(256) quant_lane_kernel(QuantArgs a) {
   pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t total = a.rows * a.nb_total;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -1076,6 +1080,7 @@ struct DequantArgs {
 
 __global__ void dequant_kernel(DequantArgs a) {
   pdl_wait();
+  pdl_trigger();
   const int64_t total = a.rows * a.nb_total;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {

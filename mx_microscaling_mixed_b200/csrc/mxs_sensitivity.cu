@@ -117,6 +117,7 @@ __device__ __forceinline__ double q4_err_term_tiny(float w, int e) {
 template <bool XF32, bool WF32, bool XVEC, bool WVEC>
 __global__ void __launch_bounds__(kSensThreads) sens_partial_kernel(SensArgs a) {
   pdl_wait();
+  pdl_trigger();
   const int64_t gtid = static_cast<int64_t>(blockIdx.x) * kSensThreads + threadIdx.x;
   const int64_t c0 = gtid * kColsPerThread;
   double acc[kColsPerThread];
@@ -231,6 +232,7 @@ __global__ void __launch_bounds__(kTileThreads)
     sens_tile_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapW, SensArgs a,
                      int32_t ctiles, int *status) {
   pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(128) uint8_t tile[];
   __shared__ __align__(8) uint64_t bar;
   const int nx = a.nchunk_x * ctiles;
@@ -288,6 +290,7 @@ constexpr int kFinSlab = 128;      // chunk partials staged per pass (32 KB)
 // thread's loads in flight; one warp then adds them in chunk order.
 __global__ void __launch_bounds__(kFinThreads) sens_finalize_kernel(SensArgs a, double *H, double *E, double *s) {
   pdl_wait();
+  pdl_trigger();
   __shared__ double sp[kFinSlab][kFinCols];
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kFinCols;
   const int nch = a.nchunk_x + a.nchunk_w;

@@ -13,17 +13,18 @@
 // difference W - Q4(W)), formed and added with explicit round-to-nearest
 // intrinsics so that no fused multiply-add can change the result.
 //
-// Two launches.  (1) Chunk partials: one CTA per 64-row chunk x 256-column
-// tile of X or of W; one thread issues a single TMA tile load (zero fill past
-// the matrix edge, which adds exact zeros and leaves block maxima alone) and
-// the 64 threads each own 4 consecutive columns, walking the chunk's rows in
-// order out of shared memory; on the W side the 8 lanes that own one
-// 32-column block share its maximum through three xor-shuffles.  Several
-// CTAs per SM keep their tile loads in flight while others compute.  Rows or
-// pitches that a TMA map cannot describe (unaligned base or pitch) take a
-// register-streaming variant with the same arithmetic.  (2) A per-column pass
-// that stages the chunk partials of 32 columns in shared memory, adds them in
-// chunk order and forms H, E and s.
+// Two launches.  (1) Chunk partials: one CTA (one warp) per 64-row chunk x
+// 256-column tile of X or of W; one thread streams the chunk through two
+// 8-row shared-memory buffers by TMA (zero fill past the matrix edge, which
+// adds exact zeros and leaves block maxima alone) and each lane owns 8
+// consecutive columns, walking the chunk's rows in order; on the W side the
+// 4 lanes that own one 32-column block share its maximum through two
+// xor-shuffles.  The small buffers let many CTAs share an SM, so loads stay
+// in flight while others compute.  Rows or pitches that a TMA map cannot
+// describe (unaligned base or pitch) take a register-streaming variant with
+// the same arithmetic.  (2) A per-column pass that stages the chunk
+// partials of 16 columns in shared memory (all of a thread's loads in flight
+// together), adds them in chunk order and forms H, E and s.
 #include <algorithm>
 #include <mutex>
 
@@ -186,47 +187,71 @@ __global__ void __launch_bounds__(kSensThreads) sens_partial_kernel(SensArgs a) 
 }
 
 constexpr int kTileCols = 256;                        // columns per tile
-constexpr int kTileThreads = kTileCols / kColsPerThread;
+constexpr int kTileCPT = 8;                           // columns per thread in the tile kernel
+constexpr int kTileThreads = kTileCols / kTileCPT;
 constexpr long long kTileWaitLimit = 2000000000LL;    // cycles (~1 s)
 
+// Row r of a staged tile: this thread's 8 values.
 template <bool F32>
-__device__ __forceinline__ void lds4(const uint8_t *tile, int r, int cl, float (&v)[kColsPerThread]) {
+__device__ __forceinline__ void lds8(const uint8_t *tile, int r, int cl, float (&v)[kTileCPT]) {
   if constexpr (F32) {
-    const float4 a = *reinterpret_cast<const float4 *>(tile + (static_cast<int64_t>(r) * kTileCols + cl) * 4);
+    const float4 *p = reinterpret_cast<const float4 *>(tile + (static_cast<int64_t>(r) * kTileCols + cl) * 4);
+    const float4 a = p[0], b = p[1];
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
   } else {
-    const uint2 a = *reinterpret_cast<const uint2 *>(tile + (static_cast<int64_t>(r) * kTileCols + cl) * 2);
-    v[0] = __uint_as_float(a.x << 16);
-    v[1] = __uint_as_float(a.x & 0xFFFF0000u);
-    v[2] = __uint_as_float(a.y << 16);
-    v[3] = __uint_as_float(a.y & 0xFFFF0000u);
+    const uint4 a = *reinterpret_cast<const uint4 *>(tile + (static_cast<int64_t>(r) * kTileCols + cl) * 2);
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = __uint_as_float(w[j] << 16);
+      v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
   }
 }
 
-// One row of 4 W values: adds (w - Q4(w))^2 to acc under the 32-column
-// block's maximum (shared by the 8 lanes of the block).
+// (w - Q4(w))^2 for a bf16 w in the common case (block exponent e >= -125):
+// the code comes from fma(w, 2^(2-e), 1.5*2^23) clamped on its bit pattern;
+// w - q*2^(e-2) has <= 9 significant bits, so the fma that forms it is exact.
+__device__ __forceinline__ double q4_err_term_bf16(float w, float sc, float step) {
+  uint32_t x = __float_as_uint(fmaf(w, sc, 12582912.0f));
+  x = min(max(x, 0x4B400000u - 7u), 0x4B400000u + 7u);
+  const float d = fmaf(-(__uint_as_float(x) - 12582912.0f), step, w);
+  const double dd = static_cast<double>(d);
+  return __dmul_rn(dd, dd);
+}
+
+// One row of 8 W values: adds (w - Q4(w))^2 to acc under the 32-column
+// block's maximum (shared by the 4 lanes of the block).
 template <bool F32>
-__device__ __forceinline__ void w_row_terms(const float (&v)[kColsPerThread], double (&acc)[kColsPerThread]) {
+__device__ __forceinline__ void w_row_terms8(const float (&v)[kTileCPT], double (&acc)[kTileCPT]) {
   uint32_t ab = 0;
 #pragma unroll
-  for (int i = 0; i < kColsPerThread; ++i) ab = max(ab, __float_as_uint(v[i]) & 0x7FFFFFFFu);
+  for (int i = 0; i < kTileCPT; ++i) ab = max(ab, __float_as_uint(v[i]) & 0x7FFFFFFFu);
   ab = max(ab, __shfl_xor_sync(0xffffffffu, ab, 1));
   ab = max(ab, __shfl_xor_sync(0xffffffffu, ab, 2));
-  ab = max(ab, __shfl_xor_sync(0xffffffffu, ab, 4));
   const int ef = static_cast<int>(ab >> 23);
   const int e = ef == 0 ? -127 : ef - 127;
   if (e >= -125) {
     const float sc = __uint_as_float(static_cast<uint32_t>(2 - e + 127) << 23);
     const float step = pow2f(e - 2);
 #pragma unroll
-    for (int i = 0; i < kColsPerThread; ++i) acc[i] = __dadd_rn(acc[i], q4_err_term<F32>(v[i], sc, step));
+    for (int i = 0; i < kTileCPT; ++i) {
+      if constexpr (F32) acc[i] = __dadd_rn(acc[i], q4_err_term<true>(v[i], sc, step));
+      else acc[i] = __dadd_rn(acc[i], q4_err_term_bf16(v[i], sc, step));
+    }
   } else {
 #pragma unroll
-    for (int i = 0; i < kColsPerThread; ++i) acc[i] = __dadd_rn(acc[i], q4_err_term_tiny(v[i], e));
+    for (int i = 0; i < kTileCPT; ++i) acc[i] = __dadd_rn(acc[i], q4_err_term_tiny(v[i], e));
   }
 }
 
-// Tiles in launch order: all X tiles (chunk-major), then all W tiles.
+// Tiles in launch order: all X tiles (chunk-major), then all W tiles.  A
+// tile (one 64-row chunk x 256 columns) streams through two shared-memory
+// buffers of kSubRows rows, so the next rows load while these are summed
+// and a CTA needs little shared memory: many CTAs share an SM.
+constexpr int kSubRows = 8;
+
 template <bool XF32, bool WF32>
 __global__ void __launch_bounds__(kTileThreads)
     sens_tile_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapW, SensArgs a,
@@ -234,88 +259,119 @@ __global__ void __launch_bounds__(kTileThreads)
   pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(128) uint8_t tile[];
-  __shared__ __align__(8) uint64_t bar;
+  __shared__ __align__(8) uint64_t bar[2];
   const int nx = a.nchunk_x * ctiles;
   const bool is_x = static_cast<int>(blockIdx.x) < nx;
   const int t = is_x ? blockIdx.x : blockIdx.x - nx;
   const int chunk = t / ctiles, ct = t - chunk * ctiles;
   const bool f32 = is_x ? XF32 : WF32;
+  const CUtensorMap *map = is_x ? &mapX : &mapW;
+  const uint32_t sub_bytes = static_cast<uint32_t>(kSubRows * kTileCols * (f32 ? 4 : 2));
+  const uint32_t buf_bytes = static_cast<uint32_t>(kSubRows * kTileCols * ((XF32 || WF32) ? 4 : 2));
+  const int64_t r0 = static_cast<int64_t>(chunk) * kSumChunk;
+  const int rows = static_cast<int>(min(static_cast<int64_t>(kSumChunk), (is_x ? a.T : a.N) - r0));
+  const int nsub = (rows + kSubRows - 1) / kSubRows;
   if (threadIdx.x == 0) {
-    ptx::mbar_init(&bar, 1);
+    ptx::mbar_init(&bar[0], 1);
+    ptx::mbar_init(&bar[1], 1);
     ptx::fence_mbar_init();
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    ptx::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(kSumChunk * kTileCols * (f32 ? 4 : 2)));
-    ptx::tma_load_2d(tile, is_x ? &mapX : &mapW, &bar, ct * kTileCols, chunk * kSumChunk);
-  }
-  if (!ptx::mbar_wait_cycles(&bar, 0, kTileWaitLimit)) {
-    atomicExch(status, static_cast<int>(MXS_ERR_TIMEOUT));
-    return;
-  }
-  const int cl = threadIdx.x * kColsPerThread;
-  const int64_t c0 = static_cast<int64_t>(ct) * kTileCols + cl;
-  const int64_t r0 = static_cast<int64_t>(chunk) * kSumChunk;
-  const int rows = static_cast<int>(min(static_cast<int64_t>(kSumChunk), (is_x ? a.T : a.N) - r0));
-  double acc[kColsPerThread];
-#pragma unroll
-  for (int i = 0; i < kColsPerThread; ++i) acc[i] = 0.0;
-  if (is_x) {
-#pragma unroll 8
-    for (int r = 0; r < rows; ++r) {
-      float v[kColsPerThread];
-      lds4<XF32>(tile, r, cl, v);
-#pragma unroll
-      for (int i = 0; i < kColsPerThread; ++i) acc[i] = __dadd_rn(acc[i], square_term(v[i]));
+    for (int b = 0; b < 2 && b < nsub; ++b) {
+      ptx::mbar_arrive_expect_tx(&bar[b], sub_bytes);
+      ptx::tma_load_2d(tile + b * buf_bytes, map, &bar[b], ct * kTileCols, static_cast<int>(r0) + b * kSubRows);
     }
-  } else {
+  }
+  const int cl = threadIdx.x * kTileCPT;
+  const int64_t c0 = static_cast<int64_t>(ct) * kTileCols + cl;
+  double acc[kTileCPT];
+#pragma unroll
+  for (int i = 0; i < kTileCPT; ++i) acc[i] = 0.0;
+  for (int sb = 0; sb < nsub; ++sb) {
+    const int buf = sb & 1;
+    if (!ptx::mbar_wait_cycles(&bar[buf], (sb >> 1) & 1, kTileWaitLimit)) {
+      // the other buffer's load, if any, lands before the CTA exits
+      if (threadIdx.x == 0) {
+        atomicExch(status, static_cast<int>(MXS_ERR_TIMEOUT));
+        if (sb + 1 < nsub) ptx::mbar_wait_cycles(&bar[buf ^ 1], ((sb + 1) >> 1) & 1, kTileWaitLimit);
+      }
+      return;
+    }
+    const uint8_t *sub = tile + buf * buf_bytes;
+    const int rr = min(kSubRows, rows - sb * kSubRows);
+    if (is_x) {
+#pragma unroll 8
+      for (int r = 0; r < rr; ++r) {
+        float v[kTileCPT];
+        lds8<XF32>(sub, r, cl, v);
+#pragma unroll
+        for (int i = 0; i < kTileCPT; ++i) acc[i] = __dadd_rn(acc[i], square_term(v[i]));
+      }
+    } else {
 #pragma unroll 4
-    for (int r = 0; r < rows; ++r) {     // rows is uniform over the CTA
-      float v[kColsPerThread];
-      lds4<WF32>(tile, r, cl, v);
-      w_row_terms<WF32>(v, acc);
+      for (int r = 0; r < rr; ++r) {     // rr is uniform over the CTA
+        float v[kTileCPT];
+        lds8<WF32>(sub, r, cl, v);
+        w_row_terms8<WF32>(v, acc);
+      }
+    }
+    // the warp is done with this buffer: it takes the rows two sub-tiles on
+    __syncthreads();
+    if (threadIdx.x == 0 && sb + 2 < nsub) {
+      ptx::mbar_arrive_expect_tx(&bar[buf], sub_bytes);
+      ptx::tma_load_2d(tile + buf * buf_bytes, map, &bar[buf], ct * kTileCols, static_cast<int>(r0) + (sb + 2) * kSubRows);
     }
   }
   double *out = a.part + static_cast<int64_t>(is_x ? chunk : a.nchunk_x + chunk) * a.K + c0;
 #pragma unroll
-  for (int i = 0; i < kColsPerThread; ++i)
+  for (int i = 0; i < kTileCPT; ++i)
     if (c0 + i < a.K) out[i] = acc[i];
 }
 
-constexpr int kFinCols = 32;       // columns per CTA
+constexpr int kFinCols = 16;       // columns per CTA
 constexpr int kFinThreads = 256;
-constexpr int kFinSlab = 128;      // chunk partials staged per pass (32 KB)
+constexpr int kFinSlab = 128;      // chunk partials staged per pass (16 KB)
+constexpr int kFinPer = kFinSlab * kFinCols / kFinThreads;
 
-// Stages the partials of 32 columns, kFinSlab chunks at a time, with every
-// thread's loads in flight; one warp then adds them in chunk order.
+// Stages the partials of 16 columns, kFinSlab chunks at a time, every
+// thread's loads in flight together; then thread (column, side) of the
+// first warp adds its side's chunks (X or W) in chunk order.
 __global__ void __launch_bounds__(kFinThreads) sens_finalize_kernel(SensArgs a, double *H, double *E, double *s) {
   pdl_wait();
   pdl_trigger();
   __shared__ double sp[kFinSlab][kFinCols];
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kFinCols;
   const int nch = a.nchunk_x + a.nchunk_w;
-  double sx = 0.0, se = 0.0;
+  const int col = threadIdx.x & (kFinCols - 1), side = (threadIdx.x >> 4) & 1;
+  double acc = 0.0;
   for (int s0 = 0; s0 < nch; s0 += kFinSlab) {
     const int ns = min(kFinSlab, nch - s0);
-    __syncthreads();
-#pragma unroll 4
-    for (int i = threadIdx.x; i < ns * kFinCols; i += kFinThreads) {
-      const int ch = i / kFinCols, col = i % kFinCols;
-      const int64_t c = c0 + col;
-      sp[ch][col] = c < a.K ? a.part[static_cast<int64_t>(s0 + ch) * a.K + c] : 0.0;
+    double v[kFinPer];
+#pragma unroll
+    for (int u = 0; u < kFinPer; ++u) {
+      const int i = threadIdx.x + u * kFinThreads, ch = i / kFinCols, cc = i % kFinCols;
+      const int64_t c = c0 + cc;
+      v[u] = ch < ns && c < a.K ? a.part[static_cast<int64_t>(s0 + ch) * a.K + c] : 0.0;
+    }
+    __syncthreads();                                   // the previous slab has been summed
+#pragma unroll
+    for (int u = 0; u < kFinPer; ++u) {
+      const int i = threadIdx.x + u * kFinThreads;
+      sp[i / kFinCols][i % kFinCols] = v[u];
     }
     __syncthreads();
-    if (threadIdx.x < kFinCols) {
-      for (int ch = 0; ch < ns; ++ch) {
-        const double v = sp[ch][threadIdx.x];
-        if (s0 + ch < a.nchunk_x) sx = __dadd_rn(sx, v);
-        else se = __dadd_rn(se, v);
-      }
+    if (threadIdx.x < 2 * kFinCols) {
+      const int lo = side ? a.nchunk_x : 0, hi = side ? nch : a.nchunk_x;
+      const int b0 = max(lo, s0) - s0, b1 = min(hi, s0 + ns) - s0;
+      for (int ch = b0; ch < b1; ++ch) acc = __dadd_rn(acc, sp[ch][col]);
     }
   }
-  const int64_t j = c0 + threadIdx.x;
-  if (threadIdx.x >= kFinCols || j >= a.K) return;
-  const double h = __ddiv_rn(__dmul_rn(2.0, sx), static_cast<double>(a.T));
+  if (threadIdx.x >= 2 * kFinCols) return;
+  const double se = __shfl_down_sync(0xffffffffu, acc, kFinCols);
+  const int64_t j = c0 + col;
+  if (side || j >= a.K) return;
+  const double h = __ddiv_rn(__dmul_rn(2.0, acc), static_cast<double>(a.T));
   H[j] = h;
   if (E) E[j] = se;
   s[j] = __dmul_rn(h, se);
@@ -375,17 +431,17 @@ extern "C" mxs_status mxs_sensitivity(const void *X, mxs_dtype xt, int64_t T, in
   const bool xf = xt == MXS_F32, wf = wt == MXS_F32;
   bool tiled = false;
   if (xvec && wvec) {
-    // TMA tiles: 64 rows x 256 columns per CTA
+    // TMA tiles: 64-row chunks x 256 columns per CTA, in 8-row sub-tiles
     CUtensorMap mx{}, mw{};
     int *status = device_status_word();
     const int64_t ctiles = (K + kTileCols - 1) / kTileCols;
     const int64_t ntiles = (a.nchunk_x + a.nchunk_w) * ctiles;
     if (status && ntiles < (1ll << 31) &&
         make_plain_map(&mx, xf ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                       static_cast<int>(dtype_size(xt)), X, K, T, ldx, kTileCols, kSumChunk) &&
+                       static_cast<int>(dtype_size(xt)), X, K, T, ldx, kTileCols, kSubRows) &&
         make_plain_map(&mw, wf ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                       static_cast<int>(dtype_size(wt)), W, K, N, ldw, kTileCols, kSumChunk)) {
-      const int smem = kSumChunk * kTileCols * ((xf || wf) ? 4 : 2);
+                       static_cast<int>(dtype_size(wt)), W, K, N, ldw, kTileCols, kSubRows)) {
+      const int smem = 2 * kSubRows * kTileCols * ((xf || wf) ? 4 : 2);
       const unsigned g = static_cast<unsigned>(ntiles);
       const int32_t ct = static_cast<int32_t>(ctiles);
       if (xf && wf) {

@@ -784,6 +784,7 @@ struct SmallArgs {
   int64_t w_spitch[3];
   __nv_bfloat16 *Y;
   int64_t ldy;
+  int32_t stage_w;       // the W rows' codes are copied into shared memory too
 };
 
 constexpr int kDecRows = 16;                 // W rows per CTA (two n-tiles of 8)
@@ -874,10 +875,12 @@ __device__ __forceinline__ void widen_frag(const uint32_t (&r)[DecSeg<G>::kRaw],
 }
 
 // Shared-memory image of one CTA: per segment g, the activations' packed
-// code rows (M rows at the source pitch), their scale rows, and the scale
-// rows of the CTA's 16 W rows (rows past N repeat row N-1).
+// code rows (M rows at the source pitch), their scale rows, the scale rows
+// of the CTA's 16 W rows (rows past N repeat row N-1) and, when they fit,
+// the 16 W rows' packed codes, so that every byte the CTA reads is in
+// flight from its first instruction.
 struct DecSmem {
-  int32_t a_code[3], a_scale[3], w_scale[3];
+  int32_t a_code[3], a_scale[3], w_scale[3], w_code[3];
   int32_t bytes;
 };
 
@@ -896,13 +899,17 @@ __host__ __device__ inline DecSmem dec_smem_plan(const SmallArgs &a) {
     p.w_scale[g] = off;
     off += a.nb[g] ? static_cast<int32_t>(kDecRows * a.w_spitch[g]) : 0;
   }
+  for (int g = 0; g < 3; ++g) {
+    p.w_code[g] = off;
+    off += a.stage_w && a.nb[g] ? static_cast<int32_t>(kDecRows * a.w_cpitch[g]) : 0;
+  }
   p.bytes = off;
   return p;
 }
 
 // The blocks of segment G: warp w takes every 8th, kU per round with their
 // W loads in flight together.
-template <int G>
+template <int G, bool SW>
 __device__ __forceinline__ void dec_segment(const SmallArgs &a, const uint8_t *smem, const DecSmem &sp, int n0,
                                             float (&acc)[2][4]) {
   constexpr int MB = G == 0 ? 8 : (G == 1 ? 6 : 4);
@@ -915,7 +922,9 @@ __device__ __forceinline__ void dec_segment(const SmallArgs &a, const uint8_t *s
   // this lane's rows: W rows n0 + 8j + gid (loads), activation rows gid, gid + 8
   const uint8_t *wrow[2];
 #pragma unroll
-  for (int j = 0; j < 2; ++j) wrow[j] = wc + static_cast<int64_t>(min(n0 + 8 * j + gid, a.N - 1)) * a.w_cpitch[G];
+  for (int j = 0; j < 2; ++j)
+    wrow[j] = SW ? smem + sp.w_code[G] + (8 * j + gid) * a.w_cpitch[G]
+                 : wc + static_cast<int64_t>(min(n0 + 8 * j + gid, a.N - 1)) * a.w_cpitch[G];
   const bool a_lo = gid < a.M, a_hi = gid + 8 < a.M;   // rows past M read as zero
   const uint8_t *arow_lo = smem + sp.a_code[G] + (a_lo ? gid : 0) * a.a_cpitch[G];
   const uint8_t *arow_hi = smem + sp.a_code[G] + (a_hi ? gid + 8 : 0) * a.a_cpitch[G];
@@ -928,7 +937,7 @@ __device__ __forceinline__ void dec_segment(const SmallArgs &a, const uint8_t *s
       const int bb = b0 + kDecWarps * u;
       if (bb < nbg) {
 #pragma unroll
-        for (int j = 0; j < 2; ++j) load_frag_raw<G, false>(wrow[j] + bb * BB, tig, raw[u][j]);
+        for (int j = 0; j < 2; ++j) load_frag_raw<G, SW>(wrow[j] + bb * BB, tig, raw[u][j]);
       }
     }
 #pragma unroll
@@ -995,10 +1004,14 @@ __global__ void __launch_bounds__(kDecThreads) gemm_small_kernel(SmallArgs a, in
         ptx::bulk_load(smem + sp.a_scale[g] + r * a.a_spitch[g], a.a_scales[g] + r * a.a_spitch[g],
                        static_cast<uint32_t>(a.a_spitch[g]), &bar);
       }
-      for (int r = lane; r < kDecRows; r += 32)
-        ptx::bulk_load(smem + sp.w_scale[g] + r * a.w_spitch[g],
-                       a.w_scales[g] + static_cast<int64_t>(min(n0 + r, a.N - 1)) * a.w_spitch[g],
+      for (int r = lane; r < kDecRows; r += 32) {
+        const int64_t wr = min(n0 + r, a.N - 1);
+        ptx::bulk_load(smem + sp.w_scale[g] + r * a.w_spitch[g], a.w_scales[g] + wr * a.w_spitch[g],
                        static_cast<uint32_t>(a.w_spitch[g]), &bar);
+        if (a.stage_w)
+          ptx::bulk_load(smem + sp.w_code[g] + r * a.w_cpitch[g], a.w_codes[g] + wr * a.w_cpitch[g],
+                         static_cast<uint32_t>(a.w_cpitch[g]), &bar);
+      }
     }
   }
   float acc[2][4];
@@ -1011,9 +1024,15 @@ __global__ void __launch_bounds__(kDecThreads) gemm_small_kernel(SmallArgs a, in
     if (threadIdx.x == 0) atomicExch(status, static_cast<int>(MXS_ERR_TIMEOUT));
     return;     // the copies are the wait that expired: nothing else is in flight
   }
-  dec_segment<0>(a, smem, sp, n0, acc);
-  dec_segment<1>(a, smem, sp, n0, acc);
-  dec_segment<2>(a, smem, sp, n0, acc);
+  if (a.stage_w) {
+    dec_segment<0, true>(a, smem, sp, n0, acc);
+    dec_segment<1, true>(a, smem, sp, n0, acc);
+    dec_segment<2, true>(a, smem, sp, n0, acc);
+  } else {
+    dec_segment<0, false>(a, smem, sp, n0, acc);
+    dec_segment<1, false>(a, smem, sp, n0, acc);
+    dec_segment<2, false>(a, smem, sp, n0, acc);
+  }
   // the warps' partial sums, added in warp order
   __syncthreads();
   float(*red)[16][kDecRows + 1] = reinterpret_cast<float(*)[16][kDecRows + 1]>(smem);
@@ -1062,6 +1081,8 @@ static SmallArgs small_args(const mxs_mxtensor *A, const mxs_mxtensor *W, void *
   }
   a.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
   a.ldy = ldy;
+  a.stage_w = 1;
+  if (small_smem_bytes(a) > kDecSmemCap) a.stage_w = 0;   // W codes stream from global memory instead
   return a;
 }
 

@@ -33,7 +33,7 @@ namespace mxs {
 constexpr int kRankCols = 32;                     // columns ranked per CTA
 constexpr int kRankParts = 16;                    // candidate slices per column
 constexpr int kRankThreads = kRankCols * kRankParts;
-constexpr int kRankTile = 2048;                   // candidates staged per pass
+constexpr int kRankTile = 4096;                   // candidates staged per pass (32 KB)
 constexpr int kRankSlice = kRankTile / kRankParts;
 
 // rank[j] = #{i : s_i > s_j, or s_i == s_j and i < j}.  Thread (part, c)
@@ -52,7 +52,21 @@ __global__ void __launch_bounds__(kRankThreads) rank_kernel(const double *s, int
   for (int64_t base = 0; base < K; base += kRankTile) {
     const int n = static_cast<int>(min(static_cast<int64_t>(kRankTile), K - base));
     __syncthreads();
-    for (int i = threadIdx.x; i < n; i += kRankThreads) tile[i] = s[base + i];
+    {
+      // every thread's loads in flight together, then the stores
+      constexpr int kPer = kRankTile / kRankThreads;
+      double v[kPer];
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int i = threadIdx.x + u * kRankThreads;
+        v[u] = i < n ? s[base + i] : 0.0;
+      }
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int i = threadIdx.x + u * kRankThreads;
+        if (i < n) tile[i] = v[u];
+      }
+    }
     __syncthreads();
     const int i0 = part * kRankSlice, i1 = min(i0 + kRankSlice, n);
     if (base + i1 <= j) {
@@ -112,9 +126,18 @@ __global__ void __launch_bounds__(kPermThreads) perm_kernel(const int32_t *rank,
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t ipt = (K + kPermThreads - 1) / kPermThreads;
   const int64_t j0 = min(K, threadIdx.x * ipt), j1 = min(K, j0 + ipt);
+  // up to kPermKeep ranks per thread stay in registers for the second pass
+  constexpr int kPermKeep = 8;
+  int32_t kept[kPermKeep];
+#pragma unroll
+  for (int u = 0; u < kPermKeep; ++u) kept[u] = j0 + u < j1 ? rank[j0 + u] : 0;
   unsigned long long cnt = 0;
-#pragma unroll 4
-  for (int64_t j = j0; j < j1; ++j) {
+#pragma unroll
+  for (int u = 0; u < kPermKeep; ++u) {
+    const int64_t r = kept[u];
+    if (j0 + u < j1) cnt += r < n8 ? 1ull : (r < n8 + n6 ? (1ull << 32) : 0ull);
+  }
+  for (int64_t j = j0 + kPermKeep; j < j1; ++j) {
     const int64_t r = rank[j];
     cnt += r < n8 ? 1ull : (r < n8 + n6 ? (1ull << 32) : 0ull);
   }
@@ -140,7 +163,11 @@ __global__ void __launch_bounds__(kPermThreads) perm_kernel(const int32_t *rank,
   int64_t c0 = static_cast<int64_t>(before & 0xFFFFFFFFull), c1 = static_cast<int64_t>(before >> 32);
   int64_t c2 = j0 - c0 - c1;
   for (int64_t j = j0; j < j1; ++j) {
-    const int64_t r = rank[j];
+    int64_t r = 0;
+#pragma unroll
+    for (int u = 0; u < kPermKeep; ++u)
+      if (j == j0 + u) r = kept[u];
+    if (j >= j0 + kPermKeep) r = rank[j];
     int64_t slot;
     if (r < n8) slot = c0++;
     else if (r < n8 + n6) slot = n8 + c1++;

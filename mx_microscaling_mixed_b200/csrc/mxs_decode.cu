@@ -1,0 +1,376 @@
+// mxs_decode.cu -- mxs_gemm for a handful of activation rows (decode).
+//
+// MXSens (arXiv 2607.17733), technical summary §2.3 and §4: the mixed
+// 4/6/8-bit MXINT linear layer; at decode the product is bound by the bytes
+// of the packed weights, which this path reads once.
+#include <algorithm>
+
+#include "mxs_decode.cuh"
+#include "mxs_ptx.cuh"
+
+namespace mxs {
+
+// ------------------------------------------------------ small-M decode path
+//
+// For a handful of activation rows the GEMM is bound by the bytes of W, so
+// W is read packed, once, and never expanded in memory.  Within one
+// 32-position block both operands share one E8M0 scale each, so the block's
+// contribution is an integer dot product times an exact power of two:
+//   sum_t qa_t qw_t * 2^(ea - m + 2) * 2^(ew - m + 2).
+// Every code is widened to a signed byte holding code * 2^(8-m) (the code
+// in the top bits of the byte: a mask, no sign extension), so one 32-column
+// block of either operand is 32 int8 values and the block's integer dot
+// product is exactly one tensor-core mma.sync m16n8k32 (s8 x s8 -> s32),
+// 16 activation rows x 8 W rows.  |sum| < 2^22, so the int32 converts
+// exactly, and the scale 2^(ea-6) * 2^(ew-6) is exact; only the fp32
+// accumulation over blocks (and the final bf16 rounding) rounds.  The block
+// scaling forbids accumulating across blocks inside the tensor core, which
+// is why the block-sized warp-level MMA is used here rather than tcgen05.
+//
+// Each CTA owns 16 W rows (two n-tiles of 8); its eight warps split the K
+// blocks of each segment (warp w takes blocks w, w+8, ...).  One warp
+// bulk-copies (TMA) the activations' packed code and scale rows and the 16 W
+// rows' packed code and scale rows into shared memory, so every byte the CTA
+// needs is in flight at once; every lane then builds, per block, its A and
+// B fragments from the shared copies, widening only the two 4-code groups a
+// fragment holds.  When the W rows do not fit beside the activations, their
+// codes stream from global memory instead (no L1 allocation, several blocks
+// in flight).  The warps' partial sums are added in shared memory in warp
+// order.  Calls whose packed activation rows do not fit in shared memory
+// take the tensor-core path.
+struct SmallArgs {
+  int32_t M, N;
+  int32_t nb[3];
+  int32_t nb_total;
+  const uint8_t *a_codes[3];
+  int64_t a_cpitch[3];
+  const uint8_t *a_scales[3];
+  int64_t a_spitch[3];
+  const uint8_t *w_codes[3];
+  int64_t w_cpitch[3];
+  const uint8_t *w_scales[3];
+  int64_t w_spitch[3];
+  __nv_bfloat16 *Y;
+  int64_t ldy;
+  int32_t stage_w;       // the W rows' codes are copied into shared memory too
+};
+
+constexpr int kDecRows = 16;                 // W rows per CTA (two n-tiles of 8)
+constexpr int kDecMaxM = 16;                 // activation rows: the MMA's 16 rows
+constexpr int kDecWarps = 8;                 // K slots
+constexpr int kDecThreads = kDecWarps * 32;
+
+__device__ __forceinline__ void small_locate(const SmallArgs &a, int gb, int &g, int &b) {
+  if (gb < a.nb[0]) { g = 0; b = gb; }
+  else if (gb < a.nb[0] + a.nb[1]) { g = 1; b = gb - a.nb[0]; }
+  else { g = 2; b = gb - a.nb[0] - a.nb[1]; }
+}
+
+// Four 4-bit codes (16 bits, code i in nibble i) -> four bytes code << 4.
+__device__ __forceinline__ uint32_t widen4(uint32_t x16) {
+  const uint32_t p = __byte_perm(x16, 0, 0x1100);       // bytes b0 b0 b1 b1
+  return ((p << 4) & 0x00F000F0u) | (p & 0xF000F000u);
+}
+// Four 6-bit codes (24 bits, code i at bits 6i) -> four bytes code << 2.
+__device__ __forceinline__ uint32_t widen6(uint32_t v) {
+  return ((v << 2) & 0xFCu) | ((v << 4) & 0xFC00u) | ((v << 6) & 0xFC0000u) | ((v << 8) & 0xFC000000u);
+}
+
+__device__ __forceinline__ void mma_s8_16x8x32(const uint4 &a, uint32_t b0, uint32_t b1, int (&c)[4]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%10, %11, %12, %13};"
+      : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1), "r"(0), "r"(0), "r"(0), "r"(0));
+}
+
+__device__ __forceinline__ uint32_t ld_stream_u16(const uint8_t *p) {
+  unsigned short v;
+  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_stream_u32(const uint8_t *p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
+// Per segment: raw words one lane loads for its B fragment of one W block,
+// and how many blocks a warp keeps in flight.
+template <int G> struct DecSeg;
+template <> struct DecSeg<0> { static constexpr int kRaw = 2, kU = 4; };   // 8-bit: words t, 4+t
+template <> struct DecSeg<1> { static constexpr int kRaw = 4, kU = 4; };   // 6-bit: two word pairs
+template <> struct DecSeg<2> { static constexpr int kRaw = 2, kU = 8; };   // 4-bit: two 16-bit groups
+
+__device__ __forceinline__ uint32_t lds_u16(const uint8_t *p) { return *reinterpret_cast<const unsigned short *>(p); }
+__device__ __forceinline__ uint32_t lds_u32(const uint8_t *p) { return *reinterpret_cast<const uint32_t *>(p); }
+
+// The words of block c (packed, m-bit) that lane-in-group t needs for its
+// fragment: code groups t and 4+t (codes 4t..4t+3 and 16+4t..16+4t+3).
+// SMEM: c points into shared memory (activations), else into global memory
+// (W, streaming loads).
+template <int G, bool SMEM>
+__device__ __forceinline__ void load_frag_raw(const uint8_t *c, int t, uint32_t (&r)[DecSeg<G>::kRaw]) {
+  if constexpr (G == 2) {
+    r[0] = SMEM ? lds_u16(c + 2 * t) : ld_stream_u16(c + 2 * t);
+    r[1] = SMEM ? lds_u16(c + 8 + 2 * t) : ld_stream_u16(c + 8 + 2 * t);
+  } else if constexpr (G == 0) {
+    r[0] = SMEM ? lds_u32(c + 4 * t) : ld_stream_u32(c + 4 * t);
+    r[1] = SMEM ? lds_u32(c + 16 + 4 * t) : ld_stream_u32(c + 16 + 4 * t);
+  } else {
+    // group t: bytes 3t..3t+2, inside words (3t)/4 and (3t+2)/4
+    const int w0 = 4 * ((3 * t) >> 2), w1 = 4 * ((3 * t + 2) >> 2);
+    r[0] = SMEM ? lds_u32(c + w0) : ld_stream_u32(c + w0);
+    r[1] = SMEM ? lds_u32(c + w1) : ld_stream_u32(c + w1);
+    r[2] = SMEM ? lds_u32(c + 12 + w0) : ld_stream_u32(c + 12 + w0);
+    r[3] = SMEM ? lds_u32(c + 12 + w1) : ld_stream_u32(c + 12 + w1);
+  }
+}
+
+template <int G>
+__device__ __forceinline__ void widen_frag(const uint32_t (&r)[DecSeg<G>::kRaw], int t, uint32_t &b0, uint32_t &b1) {
+  if constexpr (G == 2) {
+    b0 = widen4(r[0]);
+    b1 = widen4(r[1]);
+  } else if constexpr (G == 0) {
+    b0 = r[0];
+    b1 = r[1];
+  } else {
+    const int sh = (3 * t & 3) * 8;
+    b0 = widen6(__funnelshift_r(r[0], r[1], sh));
+    b1 = widen6(__funnelshift_r(r[2], r[3], sh));
+  }
+}
+
+// Shared-memory image of one CTA: per segment g, the activations' packed
+// code rows (M rows at the source pitch), their scale rows, the scale rows
+// of the CTA's 16 W rows (rows past N repeat row N-1) and, when they fit,
+// the 16 W rows' packed codes, so that every byte the CTA reads is in
+// flight from its first instruction.
+struct DecSmem {
+  int32_t a_code[3], a_scale[3], w_scale[3], w_code[3];
+  int32_t bytes;
+};
+
+__host__ __device__ inline DecSmem dec_smem_plan(const SmallArgs &a) {
+  DecSmem p{};
+  int32_t off = 0;
+  for (int g = 0; g < 3; ++g) {
+    p.a_code[g] = off;
+    off += a.nb[g] ? static_cast<int32_t>(a.M * a.a_cpitch[g]) : 0;
+  }
+  for (int g = 0; g < 3; ++g) {
+    p.a_scale[g] = off;
+    off += a.nb[g] ? static_cast<int32_t>(a.M * a.a_spitch[g]) : 0;
+  }
+  for (int g = 0; g < 3; ++g) {
+    p.w_scale[g] = off;
+    off += a.nb[g] ? static_cast<int32_t>(kDecRows * a.w_spitch[g]) : 0;
+  }
+  for (int g = 0; g < 3; ++g) {
+    p.w_code[g] = off;
+    off += a.stage_w && a.nb[g] ? static_cast<int32_t>(kDecRows * a.w_cpitch[g]) : 0;
+  }
+  p.bytes = off;
+  return p;
+}
+
+// The blocks of segment G: warp w takes every 8th, kU per round with their
+// W loads in flight together.
+template <int G, bool SW>
+__device__ __forceinline__ void dec_segment(const SmallArgs &a, const uint8_t *smem, const DecSmem &sp, int n0,
+                                            float (&acc)[2][4]) {
+  constexpr int MB = G == 0 ? 8 : (G == 1 ? 6 : 4);
+  constexpr int BB = kBlock * MB / 8;                 // bytes per packed block
+  constexpr int U = DecSeg<G>::kU, R = DecSeg<G>::kRaw;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int nbg = a.nb[G];
+  const uint8_t *wc = a.w_codes[G];
+  // this lane's rows: W rows n0 + 8j + gid (loads), activation rows gid, gid + 8
+  const uint8_t *wrow[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+    wrow[j] = SW ? smem + sp.w_code[G] + (8 * j + gid) * a.w_cpitch[G]
+                 : wc + static_cast<int64_t>(min(n0 + 8 * j + gid, a.N - 1)) * a.w_cpitch[G];
+  const bool a_lo = gid < a.M, a_hi = gid + 8 < a.M;   // rows past M read as zero
+  const uint8_t *arow_lo = smem + sp.a_code[G] + (a_lo ? gid : 0) * a.a_cpitch[G];
+  const uint8_t *arow_hi = smem + sp.a_code[G] + (a_hi ? gid + 8 : 0) * a.a_cpitch[G];
+  const uint8_t *asc = smem + sp.a_scale[G];
+  const uint8_t *wsc = smem + sp.w_scale[G];
+  for (int b0 = warp; b0 < nbg; b0 += kDecWarps * U) {
+    uint32_t raw[U][2][R];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int bb = b0 + kDecWarps * u;
+      if (bb < nbg) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) load_frag_raw<G, SW>(wrow[j] + bb * BB, tig, raw[u][j]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int bb = b0 + kDecWarps * u;
+      if (bb >= nbg) continue;
+      // A fragment: rows gid / gid+8, code groups tig / 4+tig
+      uint32_t ar[2][R];
+      load_frag_raw<G, true>(arow_lo + bb * BB, tig, ar[0]);
+      load_frag_raw<G, true>(arow_hi + bb * BB, tig, ar[1]);
+      uint4 af;
+      widen_frag<G>(ar[0], tig, af.x, af.z);
+      widen_frag<G>(ar[1], tig, af.y, af.w);
+      if (!a_lo) af.x = af.z = 0u;
+      if (!a_hi) af.y = af.w = 0u;
+      // bytes hold code * 2^(8-m): scale 2^(e-m+2) * 2^(m-8) = 2^(e-6)
+      const float fa_lo = pow2f(static_cast<int>(asc[(a_lo ? gid : 0) * a.a_spitch[G] + bb]) - 127 - 6);
+      const float fa_hi = pow2f(static_cast<int>(asc[(a_hi ? gid + 8 : 0) * a.a_spitch[G] + bb]) - 127 - 6);
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        uint32_t f0, f1;
+        widen_frag<G>(raw[u][j], tig, f0, f1);
+        int c[4];
+        mma_s8_16x8x32(af, f0, f1, c);
+        const float fw0 = pow2f(static_cast<int>(wsc[(8 * j + 2 * tig) * a.w_spitch[G] + bb]) - 127 - 6);
+        const float fw1 = pow2f(static_cast<int>(wsc[(8 * j + 2 * tig + 1) * a.w_spitch[G] + bb]) - 127 - 6);
+        acc[j][0] = fmaf(code_to_float(c[0]), fa_lo * fw0, acc[j][0]);
+        acc[j][1] = fmaf(code_to_float(c[1]), fa_lo * fw1, acc[j][1]);
+        acc[j][2] = fmaf(code_to_float(c[2]), fa_hi * fw0, acc[j][2]);
+        acc[j][3] = fmaf(code_to_float(c[3]), fa_hi * fw1, acc[j][3]);
+      }
+    }
+  }
+}
+
+constexpr long long kDecWaitLimit = 2000000000LL;    // cycles (~1 s)
+
+// One CTA: W rows n0 .. n0+15.  Thread 0 bulk-copies the activations' code
+// and scale rows and the 16 W rows' scale rows into shared memory; the warps
+// then run the three segments and add their partial sums in warp order.
+__global__ void __launch_bounds__(kDecThreads) gemm_small_kernel(SmallArgs a, int *status) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ __align__(8) uint64_t bar;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int n0 = blockIdx.x * kDecRows;
+  const DecSmem sp = dec_smem_plan(a);
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // copies: per segment, M activation code rows, M scale rows, 16 W scale rows
+    if (lane == 0) ptx::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(sp.bytes));
+    __syncwarp();
+    for (int g = 0; g < 3; ++g) {
+      if (!a.nb[g]) continue;
+      for (int r = lane; r < a.M; r += 32) {
+        ptx::bulk_load(smem + sp.a_code[g] + r * a.a_cpitch[g], a.a_codes[g] + r * a.a_cpitch[g],
+                       static_cast<uint32_t>(a.a_cpitch[g]), &bar);
+        ptx::bulk_load(smem + sp.a_scale[g] + r * a.a_spitch[g], a.a_scales[g] + r * a.a_spitch[g],
+                       static_cast<uint32_t>(a.a_spitch[g]), &bar);
+      }
+      for (int r = lane; r < kDecRows; r += 32) {
+        const int64_t wr = min(n0 + r, a.N - 1);
+        ptx::bulk_load(smem + sp.w_scale[g] + r * a.w_spitch[g], a.w_scales[g] + wr * a.w_spitch[g],
+                       static_cast<uint32_t>(a.w_spitch[g]), &bar);
+        if (a.stage_w)
+          ptx::bulk_load(smem + sp.w_code[g] + r * a.w_cpitch[g], a.w_codes[g] + wr * a.w_cpitch[g],
+                         static_cast<uint32_t>(a.w_cpitch[g]), &bar);
+      }
+    }
+  }
+  float acc[2][4];
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
+  const bool landed = ptx::mbar_wait_cycles(&bar, 0, kDecWaitLimit);
+  if (__syncthreads_or(!landed)) {                    // uniform: every thread leaves together
+    if (threadIdx.x == 0) atomicExch(status, static_cast<int>(MXS_ERR_TIMEOUT));
+    return;     // the copies are the wait that expired: nothing else is in flight
+  }
+  if (a.stage_w) {
+    dec_segment<0, true>(a, smem, sp, n0, acc);
+    dec_segment<1, true>(a, smem, sp, n0, acc);
+    dec_segment<2, true>(a, smem, sp, n0, acc);
+  } else {
+    dec_segment<0, false>(a, smem, sp, n0, acc);
+    dec_segment<1, false>(a, smem, sp, n0, acc);
+    dec_segment<2, false>(a, smem, sp, n0, acc);
+  }
+  // the warps' partial sums, added in warp order
+  __syncthreads();
+  float(*red)[16][kDecRows + 1] = reinterpret_cast<float(*)[16][kDecRows + 1]>(smem);
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    red[warp][gid][8 * j + 2 * tig] = acc[j][0];
+    red[warp][gid][8 * j + 2 * tig + 1] = acc[j][1];
+    red[warp][gid + 8][8 * j + 2 * tig] = acc[j][2];
+    red[warp][gid + 8][8 * j + 2 * tig + 1] = acc[j][3];
+  }
+  __syncthreads();
+  {
+    const int m = threadIdx.x >> 4, r = threadIdx.x & 15, n = n0 + r;
+    if (m < a.M && n < a.N) {
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) sum += red[w][m][r];
+      a.Y[static_cast<int64_t>(m) * a.ldy + n] = __float2bfloat16_rn(sum);
+    }
+  }
+}
+
+static int64_t small_smem_bytes(const SmallArgs &a) {
+  const int64_t red = static_cast<int64_t>(kDecWarps) * 16 * (kDecRows + 1) * 4;
+  return std::max<int64_t>(dec_smem_plan(a).bytes, red);
+}
+
+constexpr int64_t kDecSmemCap = 200 * 1024;
+
+static SmallArgs small_args(const mxs_mxtensor *A, const mxs_mxtensor *W, void *Y, int64_t ldy) {
+  SmallArgs a{};
+  a.M = static_cast<int32_t>(A->rows);
+  a.N = static_cast<int32_t>(W->rows);
+  a.nb_total = 0;
+  for (int g = 0; g < 3; ++g) {
+    a.nb[g] = static_cast<int32_t>(A->lay.seg[g].k_pad / kBlock);
+    a.nb_total += a.nb[g];
+    a.a_codes[g] = A->codes[g];
+    a.a_cpitch[g] = A->code_pitch[g];
+    a.a_scales[g] = A->scales[g];
+    a.a_spitch[g] = A->scale_pitch[g];
+    a.w_codes[g] = W->codes[g];
+    a.w_cpitch[g] = W->code_pitch[g];
+    a.w_scales[g] = W->scales[g];
+    a.w_spitch[g] = W->scale_pitch[g];
+  }
+  a.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
+  a.ldy = ldy;
+  a.stage_w = 1;
+  if (small_smem_bytes(a) > kDecSmemCap) a.stage_w = 0;   // W codes stream from global memory instead
+  return a;
+}
+
+// True when the decode path takes this call (up to 16 activation rows whose
+// packed rows fit in shared memory).
+bool small_fits(const mxs_mxtensor *A, const mxs_mxtensor *W) {
+  if (A->rows > kDecMaxM) return false;
+  return small_smem_bytes(small_args(A, W, nullptr, 0)) <= kDecSmemCap;
+}
+
+mxs_status gemm_small(const mxs_mxtensor *A, const mxs_mxtensor *W, void *Y, int64_t ldy, cudaStream_t cs) {
+  const SmallArgs a = small_args(A, W, Y, ldy);
+  int *status = device_status_word();
+  if (!status) return MXS_ERR_CUDA;
+  const int smem = static_cast<int>(small_smem_bytes(a));
+  if (!ensure_smem(gemm_small_kernel, smem)) return MXS_ERR_CUDA;
+  launch_pdl(gemm_small_kernel, dim3((a.N + kDecRows - 1) / kDecRows), dim3(kDecThreads), smem, cs, a, status);
+  count_launch();
+  return cuda_status(cudaGetLastError());
+}
+
+
+}  // namespace mxs

@@ -81,6 +81,12 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);
 }
 
+// Value of an integer |q| < 2^22 as an exact float: the integer rides in the
+// mantissa of 1.5*2^23 and is taken back out by a subtraction.
+__device__ __forceinline__ float code_to_float(int q) {
+  return __uint_as_float(static_cast<uint32_t>(0x4B400000 + q)) - 12582912.0f;
+}
+
 // Exact x * 2^k for the exponents the MXINT coder needs (k in [-126, 140]).
 // A single multiply by a normal power of two is exact unless the result is
 // subnormal, which only happens for values that round to code 0 anyway.

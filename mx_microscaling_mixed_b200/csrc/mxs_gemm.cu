@@ -342,6 +342,7 @@ constexpr int kP2TileBytes = kP2Rows * kSliceBytes;
 constexpr int kP2SfaBytes = kSfChunk;              // own 128 A rows x 4 blocks
 constexpr int kP2SfbBytes = 2 * kSfChunk;          // the pair's 256 N rows x 4 blocks
 constexpr int kP2EpiWarps = 8;
+constexpr int kP2EpiCols = 40;                      // Y columns per TMA store (3 per half tile)
 constexpr int kP2Threads = (2 + kP2EpiWarps) * 32;
 // cta_group::2, M = 256, N = 240
 constexpr uint32_t kIdesc2Bf16 = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kP2N >> 3) << 17) |
@@ -356,7 +357,11 @@ struct P2Smem {
   static constexpr int sfb_off = sfa_off + kP2Stages * kP2Sub * kP2SfaBytes;
   static constexpr int bar_off = sfb_off + kP2Stages * kP2Sub * kP2SfbBytes;
   // full[S], empty[S], acc_full[2], acc_empty[2], tmem slot, abort flag
-  static constexpr int bytes = bar_off + (2 * kP2Stages + 4) * 8 + 16;
+  static constexpr int bar_end = bar_off + (2 * kP2Stages + 4) * 8 + 16;
+  // per epilogue warp: a 32-row x 40-column bf16 piece of Y on its way out by TMA
+  static constexpr int epi_off = (bar_end + 127) / 128 * 128;
+  static constexpr int epi_bytes = 32 * kP2EpiCols * 2;
+  static constexpr int bytes = epi_off + kP2EpiWarps * epi_bytes;
 };
 constexpr int kP2SmemBytes = P2Smem::bytes + 1024;
 
@@ -368,12 +373,14 @@ struct P2Args {
   __nv_bfloat16 *Y;
   int64_t ldy;
   int32_t y_vec;
+  int32_t y_tma;         // Y leaves through the tensor map (16-byte aligned rows)
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA16, const __grid_constant__ CUtensorMap tmB16,
                     const __grid_constant__ CUtensorMap tmA8, const __grid_constant__ CUtensorMap tmB8,
-                    const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB, P2Args g) {
+                    const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
+                    const __grid_constant__ CUtensorMap tmY, P2Args g) {
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -409,8 +416,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
     ptx::tmem_relinquish2();
   }
   if (threadIdx.x == 32) {
-    const CUtensorMap *maps[6] = {&tmA16, &tmB16, &tmA8, &tmB8, &tmSFA, &tmSFB};
-    for (int i = 0; i < 6; ++i) asm volatile("prefetch.tensormap [%0];" ::"l"(maps[i]) : "memory");
+    const CUtensorMap *maps[7] = {&tmA16, &tmB16, &tmA8, &tmB8, &tmSFA, &tmSFB, &tmY};
+    for (int i = 0; i < 7; ++i) asm volatile("prefetch.tensormap [%0];" ::"l"(maps[i]) : "memory");
   }
   ptx::tc_fence_before();
   ptx::cluster_sync();
@@ -524,7 +531,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&acc_empty[buf]), 0));
       const int mt = t / g.n_tiles, nt = t - mt * g.n_tiles;
-      const int row = mt * 256 + static_cast<int>(rank) * kP2Rows + q * 32 + lane;
+      const int row0 = mt * 256 + static_cast<int>(rank) * kP2Rows + q * 32;
+      if (g.y_tma) {
+        // three 32 x 40 pieces per warp: bf16 rows into the warp's staging
+        // buffer (row = lane, 80 bytes), then one tensor store each; the
+        // store clips rows past M and columns past N
+        uint8_t *stg = smem + P2Smem::epi_off + (warp - 2) * P2Smem::epi_bytes;
+#pragma unroll
+        for (int pc = 0; pc < kP2N / 2 / kP2EpiCols; ++pc) {
+          uint32_t pk[kP2EpiCols / 2];
+#pragma unroll
+          for (int i = 0; i < kP2EpiCols / 2; ++i) {
+            const int col = kP2EpiCols * pc + 2 * i;
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[col >> 5][col & 31]),
+                                                      __uint_as_float(r[col >> 5][(col & 31) + 1]));
+            pk[i] = *reinterpret_cast<uint32_t *>(&b2);
+          }
+          if (lane == 0) ptx::bulk_wait_read_all();      // the previous piece has left the buffer
+          __syncwarp();
+          uint4 *dst = reinterpret_cast<uint4 *>(stg + lane * kP2EpiCols * 2);
+#pragma unroll
+          for (int j = 0; j < kP2EpiCols / 8; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) {
+            ptx::tma_store_2d(&tmY, stg, nt * kP2N + (kP2N / 2) * h + kP2EpiCols * pc, row0);
+            ptx::bulk_commit();
+          }
+        }
+        continue;
+      }
+      const int row = row0 + lane;
       if (row < g.M) {
         __nv_bfloat16 *yrow = g.Y + static_cast<int64_t>(row) * g.ldy;
 #pragma unroll
@@ -553,6 +590,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
     }
   }
 
+  // the tensor stores of Y are complete before the CTA leaves
+  if (warp >= 2 && lane == 0) ptx::bulk_wait_all();
   ptx::tc_fence_before();
   __syncthreads();
   ptx::cluster_sync();
@@ -990,10 +1029,13 @@ extern "C" mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, voi
     pa.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
     pa.ldy = ldy;
     pa.y_vec = y_vec;
+    CUtensorMap mY{};
+    pa.y_tma = y_vec && make_plain_map(&mY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, N, M, ldy, kP2EpiCols, 32);
     if (!ensure_smem(gemm_tc2_kernel, kP2SmemBytes)) return MXS_ERR_CUDA;
     const int tiles = pa.m_tiles * pa.n_tiles;
     const int pairs = std::max(1, std::min(tiles, nsm / 2));
-    launch_pdl(gemm_tc2_kernel, dim3(2 * pairs), dim3(kP2Threads), kP2SmemBytes, cs, mA16, mB16, mA8, mB8, mSFA, mSFB, pa);
+    launch_pdl(gemm_tc2_kernel, dim3(2 * pairs), dim3(kP2Threads), kP2SmemBytes, cs, mA16, mB16, mA8, mB8, mSFA, mSFB, mY,
+               pa);
     count_launch();
     return cuda_status(cudaGetLastError());
   }

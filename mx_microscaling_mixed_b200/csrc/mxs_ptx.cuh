@@ -120,6 +120,17 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
 
 // Waits on phase `parity` of *b for at most `limit` clock cycles; false when
 // the limit ran out.
+// Tensor store shared -> global (bulk group), and the group waits.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+               "r"(smem_addr(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the group's reads of shared memory are done (the source may be rewritten)
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// the group's writes are complete
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ bool mbar_wait_cycles(uint64_t *b, uint32_t parity, long long limit) {
   if (mbar_try_wait(b, parity)) return true;
   const long long t0 = clock64();

@@ -81,3 +81,22 @@ def test_infeasible_budget(c):
     with pytest.raises(c.MxsError) as e:
         c.mxs_allocate([s], [8], mode="budget", budget=(4, 1))
     assert e.value.status == 5
+
+
+def test_llama3_8b_stack_global_budget(c):
+    """The whole Llama-3-8B linear stack under one 4.5-bit budget: 32 layers x
+    (q, k, v, o 4096-wide inputs; gate, up 4096; down 14336), layer weights the
+    output widths' shares, one greedy across all 224 layers."""
+    rng = np.random.default_rng(8)
+    shapes = [(4096, 4096), (1024, 4096), (1024, 4096), (4096, 4096), (14336, 4096), (14336, 4096),
+              (4096, 14336)] * 32                      # (N, K) per layer
+    Ns = [n for n, _ in shapes]
+    # heavy-tailed sensitivities with per-layer scale, as outlier columns give
+    s_np = [rng.standard_t(3, k) ** 2 * float(rng.uniform(0.5, 2.0)) for _, k in shapes]
+    s_dev = [torch.from_numpy(x).cuda() for x in s_np]
+    gp, gc = c.mxs_allocate(s_dev, Ns, mode="budget", budget=(9, 2))
+    op, oc = oracle.allocate(s_np, Ns, mode="budget", budget=(9, 2))
+    _cmp(gp, gc, op, oc)
+    bits = sum(n * (8 * a + 6 * b + 4 * d) for n, (a, b, d) in zip(Ns, gc))
+    elems = sum(n * k for n, k in shapes)
+    assert bits <= 4.5 * elems                          # the budget holds across the stack

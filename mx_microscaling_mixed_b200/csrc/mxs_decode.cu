@@ -361,8 +361,164 @@ bool small_fits(const mxs_mxtensor *A, const mxs_mxtensor *W) {
   return small_smem_bytes(small_args(A, W, nullptr, 0)) <= kDecSmemCap;
 }
 
+// ------------------------------------------------------------- GEMV (M <= 4)
+//
+// With one to four activation rows the tensor core's 16-row MMA mostly
+// multiplies zeros, and each block's scaling dominates the instruction
+// count.  Here one warp takes one W row; each lane takes every 32nd block
+// of it, widens the block's codes to signed bytes (code * 2^(8-m), as
+// above) and forms the block's integer dot product with each activation row
+// by eight dp4a, exact in int32, then adds it times the exact scale
+// 2^(ea-6) * 2^(ew-6) to an fp32 sum; the lanes' sums are added by a
+// shuffle tree.  The activation rows are widened once per CTA into shared
+// memory (int8 bytes and float scales).  The dp4a issue rate bounds this
+// path at larger M, which is why it stops at four rows.
+constexpr int kGvMaxM = 4;
+constexpr int kGvThreads = 128;
+constexpr int kGvU = 2;                       // blocks per lane with W loads in flight together
+
+__host__ __device__ inline int64_t gemv_smem_bytes(int M, int nb_total) {
+  return static_cast<int64_t>(M) * nb_total * (kBlock + 4);
+}
+
+// The 8 words of one block widened to signed bytes from its raw packed words.
+template <int G>
+__device__ __forceinline__ void widen_block(const uint32_t (&w)[8], uint32_t (&o)[8]) {
+  if constexpr (G == 2) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      o[2 * j] = widen4(w[j] & 0xFFFFu);
+      o[2 * j + 1] = widen4(w[j] >> 16);
+    }
+  } else if constexpr (G == 1) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int pos = 24 * i, word = pos >> 5, off = pos & 31;
+      uint32_t v = w[word] >> off;
+      if (off > 8) v |= w[word + 1] << (32 - off);
+      o[i] = widen6(v);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = w[i];
+  }
+}
+
+__global__ void __launch_bounds__(kGvThreads) gemm_gemv_kernel(SmallArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int NB = a.nb_total, M = a.M;
+  uint8_t *aq = smem;                                                  // [M][NB][32] widened codes
+  float *as = reinterpret_cast<float *>(smem + static_cast<int64_t>(M) * NB * kBlock);   // [M][NB] scales
+  // activations: one thread per (row, block)
+  for (int i = threadIdx.x; i < M * NB; i += kGvThreads) {
+    const int m = i / NB, gb = i - m * NB;
+    int g, bb;
+    small_locate(a, gb, g, bb);
+    const int mb = seg_bits(g);
+    const uint8_t *c = a.a_codes[g] + m * a.a_cpitch[g] + static_cast<int64_t>(bb) * kBlock * mb / 8;
+    uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    for (int j = 0; j < mb; ++j) w[j] = *reinterpret_cast<const uint32_t *>(c + 4 * j);
+    uint32_t o[8];
+    if (g == 0) widen_block<0>(w, o);
+    else if (g == 1) widen_block<1>(w, o);
+    else widen_block<2>(w, o);
+    uint4 *dst = reinterpret_cast<uint4 *>(aq + static_cast<int64_t>(i) * kBlock);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    as[i] = pow2f(static_cast<int>(a.a_scales[g][m * a.a_spitch[g] + bb]) - 127 - 6);
+  }
+  __syncthreads();
+  const int nwarps = gridDim.x * (kGvThreads / 32);
+  for (int n = blockIdx.x * (kGvThreads / 32) + warp; n < a.N; n += nwarps) {
+    float acc[kGvMaxM] = {0.f, 0.f, 0.f, 0.f};
+    for (int b0 = lane; b0 < NB; b0 += 32 * kGvU) {
+      uint32_t raw[kGvU][8];
+      uint8_t sw[kGvU];
+      int gs[kGvU];
+#pragma unroll
+      for (int u = 0; u < kGvU; ++u) {
+        const int gb = b0 + 32 * u;
+        gs[u] = -1;
+        if (gb < NB) {
+          int g, bb;
+          small_locate(a, gb, g, bb);
+          gs[u] = g;
+          const uint8_t *c = a.w_codes[g] + static_cast<int64_t>(n) * a.w_cpitch[g] + static_cast<int64_t>(bb) * kBlock * seg_bits(g) / 8;
+          if (g == 2) {
+            const uint4 x = __ldg(reinterpret_cast<const uint4 *>(c));
+            raw[u][0] = x.x; raw[u][1] = x.y; raw[u][2] = x.z; raw[u][3] = x.w;
+          } else if (g == 1) {
+#pragma unroll
+            for (int j = 0; j < 3; ++j) {
+              const uint2 x = __ldg(reinterpret_cast<const uint2 *>(c) + j);
+              raw[u][2 * j] = x.x;
+              raw[u][2 * j + 1] = x.y;
+            }
+          } else {
+            const uint4 x0 = __ldg(reinterpret_cast<const uint4 *>(c)), x1 = __ldg(reinterpret_cast<const uint4 *>(c) + 1);
+            raw[u][0] = x0.x; raw[u][1] = x0.y; raw[u][2] = x0.z; raw[u][3] = x0.w;
+            raw[u][4] = x1.x; raw[u][5] = x1.y; raw[u][6] = x1.z; raw[u][7] = x1.w;
+          }
+          sw[u] = __ldg(a.w_scales[g] + static_cast<int64_t>(n) * a.w_spitch[g] + bb);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kGvU; ++u) {
+        if (gs[u] < 0) continue;
+        const int gb = b0 + 32 * u;
+        uint32_t wq[8];
+        if (gs[u] == 0) widen_block<0>(raw[u], wq);
+        else if (gs[u] == 1) widen_block<1>(raw[u], wq);
+        else widen_block<2>(raw[u], wq);
+        const float fw = pow2f(static_cast<int>(sw[u]) - 127 - 6);
+#pragma unroll
+        for (int m = 0; m < kGvMaxM; ++m) {
+          if (m >= M) break;
+          const uint4 *ap = reinterpret_cast<const uint4 *>(aq + (static_cast<int64_t>(m) * NB + gb) * kBlock);
+          const uint4 x0 = ap[0], x1 = ap[1];
+          int d = __dp4a(static_cast<int>(wq[0]), static_cast<int>(x0.x), 0);
+          d = __dp4a(static_cast<int>(wq[1]), static_cast<int>(x0.y), d);
+          d = __dp4a(static_cast<int>(wq[2]), static_cast<int>(x0.z), d);
+          d = __dp4a(static_cast<int>(wq[3]), static_cast<int>(x0.w), d);
+          d = __dp4a(static_cast<int>(wq[4]), static_cast<int>(x1.x), d);
+          d = __dp4a(static_cast<int>(wq[5]), static_cast<int>(x1.y), d);
+          d = __dp4a(static_cast<int>(wq[6]), static_cast<int>(x1.z), d);
+          d = __dp4a(static_cast<int>(wq[7]), static_cast<int>(x1.w), d);
+          acc[m] = fmaf(code_to_float(d), fw * as[m * NB + gb], acc[m]);
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < kGvMaxM; ++m) {
+      if (m >= M) break;
+      float v = acc[m];
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) a.Y[static_cast<int64_t>(m) * a.ldy + n] = __float2bfloat16_rn(v);
+    }
+  }
+}
+
 mxs_status gemm_small(const mxs_mxtensor *A, const mxs_mxtensor *W, void *Y, int64_t ldy, cudaStream_t cs) {
   const SmallArgs a = small_args(A, W, Y, ldy);
+  if (a.M <= kGvMaxM) {
+    const int64_t gsmem = gemv_smem_bytes(a.M, a.nb_total);
+    if (gsmem <= kDecSmemCap) {
+      int dev = 0, nsm = 148;
+      cudaGetDevice(&dev);
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+      const int rows_per_cta = kGvThreads / 32;
+      const int grid = static_cast<int>(std::min<int64_t>((a.N + rows_per_cta - 1) / rows_per_cta,
+                                                          static_cast<int64_t>(nsm) * 64));
+      if (!ensure_smem(gemm_gemv_kernel, static_cast<int>(std::max<int64_t>(gsmem, 16)))) return MXS_ERR_CUDA;
+      launch_pdl(gemm_gemv_kernel, dim3(grid), dim3(kGvThreads), static_cast<size_t>(std::max<int64_t>(gsmem, 16)), cs, a);
+      count_launch();
+      return cuda_status(cudaGetLastError());
+    }
+  }
   int *status = device_status_word();
   if (!status) return MXS_ERR_CUDA;
   const int smem = static_cast<int>(small_smem_bytes(a));

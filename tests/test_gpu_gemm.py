@@ -174,7 +174,7 @@ def test_gemm_small_m_extreme_codes(c):
 
 
 PAIR_SHAPES = [
-    # M >= 512 runs the 2-CTA pair kernel (256 x 256 tiles, persistent)
+    # M >= 512 runs the 2-CTA pair kernel (256 x 240 tiles, persistent)
     (512, 256, 4096, (32, 960, 3104)),
     (600, 700, 640, (32, 96, 512)),          # ragged M and N tiles
     (512, 512, 256, (256, 0, 0)),            # 8-bit only: bf16 MMAs only

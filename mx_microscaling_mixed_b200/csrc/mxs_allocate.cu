@@ -14,12 +14,12 @@
 // bits), stopping at the first group that does not fit.
 //
 // Device work: an all-pairs rank count (each CTA ranks 32 columns against
-// every candidate, 16 threads per column each taking a slice of every
+// every candidate, 32 threads per column each taking a slice of every
 // candidate tile staged in shared memory, partial counts added in shared
 // memory -- exact and order-free, no atomics), the group gains (one thread
-// sums one group in rank order), and a single-CTA stable compaction (a
-// block-wide scan of per-thread segment counts) that writes the permutation
-// segment by segment in ascending column order.  The integer budget
+// sums one group in rank order), and a stable compaction that writes the
+// permutation segment by segment in ascending column order (each CTA counts
+// the segments of all columns before its range, then scans its own).  The integer budget
 // arithmetic and the cross-layer greedy are a few hundred scalar steps and
 // run on the host side of the call; only the multi-layer greedy needs device
 // data (the group gains) and so a stream synchronisation.
@@ -31,7 +31,7 @@
 namespace mxs {
 
 constexpr int kRankCols = 32;                     // columns ranked per CTA
-constexpr int kRankParts = 16;                    // candidate slices per column
+constexpr int kRankParts = 32;                    // candidate slices per column
 constexpr int kRankThreads = kRankCols * kRankParts;
 constexpr int kRankTile = 4096;                   // candidates staged per pass (32 KB)
 constexpr int kRankSlice = kRankTile / kRankParts;
@@ -112,36 +112,54 @@ __global__ void group_gain_kernel(const double *s, const int32_t *order, int64_t
   gains[g] = sum;
 }
 
-constexpr int kPermThreads = 1024;
+// The permutation: a stable compaction by segment.  CTA c places columns
+// [256 c, 256 c + 256).  Its threads first count, over all columns before
+// the CTA's range, how many fall in segments 0 and 1 (two 32-bit fields of
+// a 64-bit word, loads batched 8 per thread, a block reduction); a block
+// scan over its own columns then gives each one its slot.  The permutation keeps
+// ascending column order inside each segment.
+constexpr int kPlaceCols = 256;
 
-// One CTA.  Thread t owns columns [t*ipt, (t+1)*ipt); pass 1 counts its
-// columns of segments 0 and 1 (two 32-bit fields of one 64-bit word), a
-// block-wide exclusive scan of those words gives every thread its starting
-// slot in each segment, pass 2 writes the permutation.
-__global__ void __launch_bounds__(kPermThreads) perm_kernel(const int32_t *rank, int64_t K, int64_t n8,
-                                                            int64_t n6, int32_t *perm) {
+__device__ __forceinline__ unsigned long long seg_word(int64_t r, int64_t n8, int64_t n6) {
+  return r < n8 ? 1ull : (r < n8 + n6 ? (1ull << 32) : 0ull);
+}
+
+__global__ void __launch_bounds__(kPlaceCols) perm_place_kernel(const int32_t *rank, int64_t K, int64_t n8,
+                                                               int64_t n6, int32_t *perm) {
   pdl_wait();
   pdl_trigger();
-  __shared__ unsigned long long warp_tot[kPermThreads / 32];
+  __shared__ unsigned long long warp_tot[kPlaceCols / 32];
+  __shared__ unsigned long long before_cta;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t ipt = (K + kPermThreads - 1) / kPermThreads;
-  const int64_t j0 = min(K, threadIdx.x * ipt), j1 = min(K, j0 + ipt);
-  // up to kPermKeep ranks per thread stay in registers for the second pass
-  constexpr int kPermKeep = 8;
-  int32_t kept[kPermKeep];
-#pragma unroll
-  for (int u = 0; u < kPermKeep; ++u) kept[u] = j0 + u < j1 ? rank[j0 + u] : 0;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kPlaceCols;
+  // segment counts over columns [0, c0)
   unsigned long long cnt = 0;
+  for (int64_t j0 = threadIdx.x; j0 < c0; j0 += 8 * kPlaceCols) {
+    int32_t r[8];
 #pragma unroll
-  for (int u = 0; u < kPermKeep; ++u) {
-    const int64_t r = kept[u];
-    if (j0 + u < j1) cnt += r < n8 ? 1ull : (r < n8 + n6 ? (1ull << 32) : 0ull);
+    for (int u = 0; u < 8; ++u) {
+      const int64_t j = j0 + static_cast<int64_t>(u) * kPlaceCols;
+      r[u] = j < c0 ? rank[j] : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (r[u] >= 0) cnt += seg_word(r[u], n8, n6);
   }
-  for (int64_t j = j0 + kPermKeep; j < j1; ++j) {
-    const int64_t r = rank[j];
-    cnt += r < n8 ? 1ull : (r < n8 + n6 ? (1ull << 32) : 0ull);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if (lane == 0) warp_tot[warp] = cnt;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long t = 0;
+    for (int w = 0; w < kPlaceCols / 32; ++w) t += warp_tot[w];
+    before_cta = t;
   }
-  unsigned long long inc = cnt;                    // inclusive warp scan
+  __syncthreads();
+  // this CTA's columns: an exclusive block scan of their segment words
+  const int64_t j = c0 + threadIdx.x;
+  const int64_t rj = j < K ? rank[j] : -1;
+  const unsigned long long mine = rj >= 0 ? seg_word(rj, n8, n6) : 0ull;
+  unsigned long long inc = mine;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const unsigned long long v = __shfl_up_sync(0xffffffffu, inc, o);
@@ -149,31 +167,16 @@ __global__ void __launch_bounds__(kPermThreads) perm_kernel(const int32_t *rank,
   }
   if (lane == 31) warp_tot[warp] = inc;
   __syncthreads();
-  if (warp == 0) {
-    unsigned long long w = warp_tot[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned long long v = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += v;
-    }
-    warp_tot[lane] = w;                            // inclusive over warps
-  }
-  __syncthreads();
-  const unsigned long long before = (warp ? warp_tot[warp - 1] : 0ull) + inc - cnt;
-  int64_t c0 = static_cast<int64_t>(before & 0xFFFFFFFFull), c1 = static_cast<int64_t>(before >> 32);
-  int64_t c2 = j0 - c0 - c1;
-  for (int64_t j = j0; j < j1; ++j) {
-    int64_t r = 0;
-#pragma unroll
-    for (int u = 0; u < kPermKeep; ++u)
-      if (j == j0 + u) r = kept[u];
-    if (j >= j0 + kPermKeep) r = rank[j];
-    int64_t slot;
-    if (r < n8) slot = c0++;
-    else if (r < n8 + n6) slot = n8 + c1++;
-    else slot = n8 + n6 + c2++;
-    perm[slot] = static_cast<int32_t>(j);
-  }
+  unsigned long long wbefore = 0;
+  for (int w = 0; w < warp; ++w) wbefore += warp_tot[w];
+  if (rj < 0) return;
+  const unsigned long long before = before_cta + wbefore + inc - mine;
+  const int64_t b0 = static_cast<int64_t>(before & 0xFFFFFFFFull), b1 = static_cast<int64_t>(before >> 32);
+  int64_t slot;
+  if (rj < n8) slot = b0;
+  else if (rj < n8 + n6) slot = n8 + b1;
+  else slot = n8 + n6 + (j - b0 - b1);
+  perm[slot] = static_cast<int32_t>(j);
 }
 
 struct LayerWs {
@@ -301,7 +304,8 @@ extern "C" mxs_status mxs_allocate(int32_t n_layers, const int64_t *K, const int
   }
 
   for (int l = 0; l < n_layers; ++l) {
-    launch_pdl(perm_kernel, dim3(1), dim3(kPermThreads), 0, cs, L[l].rank, K[l], n8[l], n6[l], perm[l]);
+    launch_pdl(perm_place_kernel, dim3(static_cast<unsigned>((K[l] + kPlaceCols - 1) / kPlaceCols)), dim3(kPlaceCols), 0,
+               cs, L[l].rank, K[l], n8[l], n6[l], perm[l]);
     count_launch();
     counts[3 * l + 0] = n8[l];
     counts[3 * l + 1] = n6[l];

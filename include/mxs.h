@@ -148,7 +148,8 @@ mxs_status mxs_mxtensor_bytes(int64_t rows, const mxs_layout *lay,
  * chunks of 64 from zero, in row order, and chunk sums are added in chunk
  * order; the result is bit-identical for any launch configuration.
  *   X (device): T x K, dtype xt, pitch ldx (elements); W (device): N x K,
- *   dtype wt, pitch ldw.  H, E, s (device): K doubles each (E may be NULL).
+ *   dtype wt, pitch ldw; all values finite (a NaN or Inf makes H, E and s
+ *   unspecified).  H, E, s (device): K doubles each (E may be NULL).
  *   ws (device, 256-byte aligned): mxs_sensitivity_workspace_bytes(T, N, K).
  * T, N >= 1, K >= 1. */
 mxs_status mxs_sensitivity_workspace_bytes(int64_t T, int64_t N, int64_t K, size_t *bytes);

@@ -337,7 +337,8 @@ constexpr int kP2N = 240;                          // output columns per pair ti
 constexpr int kP2BRows = kP2N / 2;                 // rows of B per CTA per stage
 constexpr int kP2AccCols = kP2N;                   // one accumulator buffer; two buffers at columns 0 and 240
 constexpr int kP2SfCol = 2 * kP2AccCols;           // scale slots from column 480: 2 x 12 columns
-constexpr int kP2SfSlots = 2;
+constexpr int kP2SfSlots = kP2Sub;                 // one scale slot per slice of a stage
+static_assert(kP2SfCol + kP2SfSlots * kSfSlotCols <= kTmemCols, "accumulators and scale slots fit in TMEM");
 constexpr int kP2TileBytes = kP2Rows * kSliceBytes;
 constexpr int kP2SfaBytes = kSfChunk;              // own 128 A rows x 4 blocks
 constexpr int kP2SfbBytes = 2 * kSfChunk;          // the pair's 256 N rows x 4 blocks
@@ -482,6 +483,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
           const bool wide = k < n16s;
           const int j0 = kP2Sub * (wide ? k : k - n16s);
           const int nsub = min(kP2Sub, (wide ? g.n16_stages : g.n8_stages) - j0);
+          if (!wide) {
+            // the stage's scale chunks first (one slot per slice), so the
+            // copies for a later slice are queued ahead of the earlier
+            // slice's MMAs; slots are reused only by later stages, behind
+            // these MMAs in the same issue order
+            for (int h = 0; h < nsub; ++h) {
+              const uint32_t sfa_s = ptx::smem_addr(smem + P2Smem::sfa_off + (s * kP2Sub + h) * kP2SfaBytes);
+              const uint32_t sfb_s = ptx::smem_addr(smem + P2Smem::sfb_off + (s * kP2Sub + h) * kP2SfbBytes);
+              const uint32_t slot = kSfSlotCols * static_cast<uint32_t>(h);
+              ptx::copy_sf_to_tmem2(tsfa + slot, ptx::desc_sf(sfa_s));
+              ptx::copy_sf_to_tmem2(tsfb + slot, ptx::desc_sf(sfb_s));
+              ptx::copy_sf_to_tmem2(tsfb + slot + 4, ptx::desc_sf(sfb_s + kSfChunk));
+            }
+          }
           for (int h = 0; h < nsub; ++h) {
             const uint32_t a_base = ptx::smem_addr(smem + P2Smem::a_off + (s * kP2Sub + h) * kP2TileBytes);
             const uint32_t b_base = ptx::smem_addr(smem + P2Smem::b_off + (s * kP2Sub + h) * kP2TileBytes);
@@ -491,12 +506,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
                 ptx::mma2_bf16(acc, ptx::desc_sw128(a_base + 32 * q), ptx::desc_sw128(b_base + 32 * q), kIdesc2Bf16,
                                (k > 0 || h > 0 || q > 0) ? 1u : 0u);
             } else {
-              const uint32_t sfa_s = ptx::smem_addr(smem + P2Smem::sfa_off + (s * kP2Sub + h) * kP2SfaBytes);
-              const uint32_t sfb_s = ptx::smem_addr(smem + P2Smem::sfb_off + (s * kP2Sub + h) * kP2SfbBytes);
-              const uint32_t slot = kSfSlotCols * static_cast<uint32_t>((kP2Sub * it + h) % kP2SfSlots);
-              ptx::copy_sf_to_tmem2(tsfa + slot, ptx::desc_sf(sfa_s));
-              ptx::copy_sf_to_tmem2(tsfb + slot, ptx::desc_sf(sfb_s));
-              ptx::copy_sf_to_tmem2(tsfb + slot + 4, ptx::desc_sf(sfb_s + kSfChunk));
+              const uint32_t slot = kSfSlotCols * static_cast<uint32_t>(h);
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 const uint32_t idesc = kIdesc2Mxf8 | (static_cast<uint32_t>(q) << 4) | (static_cast<uint32_t>(q) << 29);
@@ -629,7 +639,14 @@ struct StageArgs {
   int64_t k16, k4;
   int32_t nkg;          // k-groups of 4 blocks in the 4-bit segment
   int32_t start[5];     // item ranges (the last entry is the end)
+  uint32_t nbw_magic, nb4p_magic;   // floor(2^32 / d) + 1 for the divisions i / d (0: divide)
 };
+
+// i / d by multiply-high with magic = floor(2^32 / d) + 1, exact while
+// i * d < 2^32 (the host passes 0 when some item index breaks that).
+__device__ __forceinline__ int div_magic(int i, int d, uint32_t magic) {
+  return magic ? static_cast<int>(__umulhi(static_cast<uint32_t>(i), magic)) : i / d;
+}
 
 __device__ __forceinline__ int64_t sf_index(int64_t r, int64_t b, int32_t nrg) {
   return ((b >> 2) * nrg + (r >> 7)) * kSfChunk + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (b & 3);
@@ -704,76 +721,122 @@ __device__ __forceinline__ void wide6_words_fast(const uint32_t (&w)[6], uint8_t
   }
 }
 
-// 6/8-bit block -> 32 exact bf16 values, four 16-byte stores.
+// 32-byte store (one 256-bit access; p 32-byte aligned).
+__device__ __forceinline__ void st_global_32B(void *p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+               "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
+// 6/8-bit block -> 32 exact bf16 values, two 32-byte stores.
 template <int M>
 __device__ __forceinline__ void stage_wide_block(const uint8_t *c, uint8_t sbyte, __nv_bfloat16 *dst) {
   uint32_t pk[16];
   wide_block_words<M>(c, sbyte, pk);
-  uint4 *o = reinterpret_cast<uint4 *>(dst);
-  o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-  o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-  o[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
-  o[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+  const uint32_t lo[8] = {pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]};
+  const uint32_t hi[8] = {pk[8], pk[9], pk[10], pk[11], pk[12], pk[13], pk[14], pk[15]};
+  st_global_32B(dst, lo);
+  st_global_32B(dst + 16, hi);
+}
+
+constexpr int kStageU = 2;   // 32-item groups per warp round of the staging kernel
+
+// Eight 4-bit codes (one word, low nibble first) -> their eight E4M3 bytes
+// (q/4), in register byte permutes: the code's low three bits pick entry
+// n & 7 of an 8-byte table (t[0..1]: codes 0..7; t[2..3]: codes 8..15, the
+// negative ones), and a third permute takes, byte by byte, the second
+// table's pick where the code's bit 3 is set.
+// Byte permute; every selector nibble here has bit 3 clear (a plain pick).
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+__device__ __forceinline__ uint2 e4m3_of_nibbles(uint32_t x, const uint32_t (&t)[4]) {
+  const uint32_t lo3 = x & 0x77777777u;
+  const uint32_t pick = ((x >> 1) & 0x44444444u) | 0x32103210u;   // byte j: j, or j + 4 when bit 3 is set
+  const uint32_t p0 = prmt(t[0], t[1], lo3), n0 = prmt(t[2], t[3], lo3);
+  const uint32_t p1 = prmt(t[0], t[1], lo3 >> 16), n1 = prmt(t[2], t[3], lo3 >> 16);
+  return make_uint2(prmt(p0, n0, pick), prmt(p1, n1, pick >> 16));
 }
 
 // One thread per item, warps on consecutive items (consecutive blocks of a
 // row), so code loads and converted stores are contiguous across the warp.
-// 4-bit codes become E4M3 pairs through a 256-entry table (one byte = two
-// codes); a k-group's four scale bytes are gathered by shuffles and written
-// as one word of the tensor core's 512-byte chunk layout.
+// 4-bit codes become E4M3 bytes by register byte permutes; a k-group's four
+// scale bytes are gathered by shuffles and written as one word of the tensor
+// core's 512-byte chunk layout.
 __global__ void __launch_bounds__(256) gemm_stage_kernel(StageArgs a) {
   pdl_wait();
   pdl_trigger();
-  __shared__ uint16_t lut[256];                        // byte of two 4-bit codes -> their E4M3 pair (q/4)
-  {
-    const int b = threadIdx.x;
-    const int lo = (b & 0xF) >= 8 ? (b & 0xF) - 16 : (b & 0xF);
-    const int hi = (b >> 4) >= 8 ? (b >> 4) - 16 : (b >> 4);
-    lut[b] = static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(make_float2(0.25f * lo, 0.25f * hi), __NV_SATFINITE, __NV_E4M3));
-  }
-  __syncthreads();
+  // E4M3 of q/4 for the codes 0..15 (q = code, or code - 16 from 8 on), one
+  // byte each: 0, .25, .5, .75, 1, 1.25, 1.5, 1.75, -2, -1.75, ..., -.25
+  const uint32_t tab[4] = {0x34302800u, 0x3E3C3A38u, 0xBABCBEC0u, 0xA8B0B4B8u};
   const int lane = threadIdx.x & 31;
   const int nwarps = gridDim.x * (blockDim.x >> 5);
-  for (int base = (blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 32; base < a.start[4]; base += nwarps * 32) {
-    int rg = 0;                                        // range of this warp (uniform)
-    while (rg < 3 && base >= a.start[rg + 1]) ++rg;
-    const int i = base + lane - a.start[rg];
-    const bool in_range = base + lane < a.start[rg + 1];
-    const StageOperand &op = a.op[rg & 1];
-    if (rg < 2) {
-      const int row = i / a.nbw, b = i - row * a.nbw;
-      if (in_range && row < op.rows) {
-        const int g = b < a.nb[0] ? 0 : 1;
-        const int bb = g == 0 ? b : b - a.nb[0];
-        const uint8_t sbyte = op.scales[g][row * op.spitch[g] + bb];
-        __nv_bfloat16 *dst = op.x16 + static_cast<int64_t>(row) * a.k16 + static_cast<int64_t>(b) * kBlock;
-        if (g == 0) stage_wide_block<8>(op.codes[0] + row * op.cpitch[0] + static_cast<int64_t>(bb) * 32, sbyte, dst);
-        else stage_wide_block<6>(op.codes[1] + row * op.cpitch[1] + static_cast<int64_t>(bb) * 24, sbyte, dst);
-      }
-    } else {
-      const int row = i / a.nb4p, b = i - row * a.nb4p;     // row of the chunk grid
-      const int lr = row & 255, real = (row >> 8) * op.tile_rows + lr;   // the operand row it holds
-      uint32_t sb = 0x7Fu;                             // 2^0 for padding rows and blocks
-      if (in_range && lr < op.tile_rows && real < op.rows && b < a.nb[2]) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(op.codes[2] + real * op.cpitch[2] + static_cast<int64_t>(b) * 16);
-        sb = op.scales[2][real * op.spitch[2] + b];
-        const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-        uint32_t out[8];
+  // a warp takes kStageU groups of 32 items per round: the 4-bit groups'
+  // code and scale loads are all issued before any of them is converted
+  for (int base = (blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * (32 * kStageU); base < a.start[4];
+       base += nwarps * 32 * kStageU) {
+    int rg[kStageU], row[kStageU], b[kStageU], real[kStageU];
+    bool live[kStageU];
+    uint4 v[kStageU];
+    uint32_t sb[kStageU];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t x = in[j];
-          out[2 * j] = static_cast<uint32_t>(lut[x & 0xFF]) | (static_cast<uint32_t>(lut[(x >> 8) & 0xFF]) << 16);
-          out[2 * j + 1] = static_cast<uint32_t>(lut[(x >> 16) & 0xFF]) | (static_cast<uint32_t>(lut[x >> 24]) << 16);
+    for (int u = 0; u < kStageU; ++u) {
+      const int gb = base + 32 * u;                    // this group's first item (uniform)
+      rg[u] = 0;
+      while (rg[u] < 4 && gb >= a.start[rg[u] + 1]) ++rg[u];
+      sb[u] = 0x7Fu;                                   // 2^0 for padding rows and blocks
+      live[u] = false;
+      if (rg[u] >= 2 && rg[u] < 4) {
+        const StageOperand &op = a.op[rg[u] & 1];
+        const int i = gb + lane - a.start[rg[u]];
+        row[u] = div_magic(i, a.nb4p, a.nb4p_magic);    // row of the chunk grid
+        b[u] = i - row[u] * a.nb4p;
+        const int lr = row[u] & 255;
+        real[u] = (row[u] >> 8) * op.tile_rows + lr;   // the operand row it holds
+        live[u] = lr < op.tile_rows && real[u] < op.rows && b[u] < a.nb[2];
+        if (live[u]) {
+          v[u] = *reinterpret_cast<const uint4 *>(op.codes[2] + real[u] * op.cpitch[2] + static_cast<int64_t>(b[u]) * 16);
+          sb[u] = op.scales[2][real[u] * op.spitch[2] + b[u]];
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(op.x8 + static_cast<int64_t>(real) * a.k4 + static_cast<int64_t>(b) * kBlock);
-        dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-        dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
       }
-      // lanes 4j..4j+3 hold blocks 4k..4k+3 of one row (ranges and nb4p are multiples of 4)
-      sb |= __shfl_down_sync(0xffffffffu, sb, 1) << 8;
-      sb |= __shfl_down_sync(0xffffffffu, sb, 2) << 16;
-      if (in_range && (lane & 3) == 0)
-        *reinterpret_cast<uint32_t *>(op.sf + sf_index(row, b, op.nrg)) = sb;
+    }
+#pragma unroll
+    for (int u = 0; u < kStageU; ++u) {
+      if (rg[u] >= 4) break;                           // past the last range (uniform)
+      const int gb = base + 32 * u;
+      const StageOperand &op = a.op[rg[u] & 1];
+      if (rg[u] < 2) {
+        const int i = gb + lane - a.start[rg[u]];
+        const int r = div_magic(i, a.nbw, a.nbw_magic), bw = i - r * a.nbw;
+        if (r < op.rows) {
+          const int g = bw < a.nb[0] ? 0 : 1;
+          const int bb = g == 0 ? bw : bw - a.nb[0];
+          const uint8_t sbyte = op.scales[g][r * op.spitch[g] + bb];
+          __nv_bfloat16 *dst = op.x16 + static_cast<int64_t>(r) * a.k16 + static_cast<int64_t>(bw) * kBlock;
+          if (g == 0) stage_wide_block<8>(op.codes[0] + r * op.cpitch[0] + static_cast<int64_t>(bb) * 32, sbyte, dst);
+          else stage_wide_block<6>(op.codes[1] + r * op.cpitch[1] + static_cast<int64_t>(bb) * 24, sbyte, dst);
+        }
+      } else {
+        if (live[u]) {
+          const uint32_t in[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+          uint32_t out[8];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint2 e = e4m3_of_nibbles(in[j], tab);
+            out[2 * j] = e.x;
+            out[2 * j + 1] = e.y;
+          }
+          st_global_32B(op.x8 + static_cast<int64_t>(real[u]) * a.k4 + static_cast<int64_t>(b[u]) * kBlock, out);
+        }
+        // lanes 4j..4j+3 hold blocks 4k..4k+3 of one row (ranges and nb4p are multiples of 4)
+        uint32_t w = sb[u];
+        w |= __shfl_down_sync(0xffffffffu, w, 1) << 8;
+        w |= __shfl_down_sync(0xffffffffu, w, 2) << 16;
+        if ((lane & 3) == 0) *reinterpret_cast<uint32_t *>(op.sf + sf_index(row[u], b[u], op.nrg)) = w;
+      }
     }
   }
 }
@@ -982,6 +1045,13 @@ extern "C" mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, voi
     }
     if (at >= INT32_MAX) return MXS_ERR_SHAPE;
     sa.start[4] = static_cast<int32_t>(at);
+  }
+  {
+    auto magic = [](int64_t d, int64_t imax) -> uint32_t {
+      return d > 1 && imax * d < (1ll << 32) ? static_cast<uint32_t>((1ull << 32) / static_cast<uint64_t>(d) + 1) : 0u;
+    };
+    sa.nbw_magic = magic(sa.nbw, std::max(sa.start[2] - sa.start[0], 0));
+    sa.nb4p_magic = magic(sa.nb4p, std::max(sa.start[4] - sa.start[2], 0));
   }
   int dev = 0, nsm = 148;
   cudaGetDevice(&dev);

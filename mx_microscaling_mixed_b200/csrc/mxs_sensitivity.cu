@@ -79,40 +79,35 @@ __device__ __forceinline__ double pow2d(int k) {
 
 constexpr int kRowBatch = 8;   // rows loaded ahead per thread
 
-// Square of x as an fp64 term (one fp64 product; exact for fp32 or bf16 x).
-__device__ __forceinline__ double square_term(float x) {
-  const double d = static_cast<double>(x);
-  return __dmul_rn(d, d);
-}
+// acc + d^2 rounded once.  Every d here has at most 26 significant bits and
+// an exponent within fp32's range widened by a few bits, so d^2 is exact in
+// fp64 and the fused form equals the product rounded and then added.
+__device__ __forceinline__ double add_square(double acc, double d) { return __fma_rn(d, d, acc); }
 
-// (w - Q4(w))^2 as an fp64 term, Q4 the 4-bit code under the block exponent:
+// w - Q4(w) in fp64, Q4 the 4-bit code under the block exponent:
 // sc = 2^(2-e) (a normal float), step = 2^(e-2).  The code comes from
 // fma(w, sc, 1.5*2^23) (round half to even), clamped on its bit pattern; the
 // same pattern minus 1.5*2^23 is the code as a float.  For bf16 w the
 // difference w - q*step has <= 9 significant bits on the bf16 grid and is
-// exact in fp32; for fp32 w it is formed in fp64.  The square is one fp64
-// product.
+// exact in fp32; for fp32 w it is formed in fp64.
 template <bool F32>
-__device__ __forceinline__ double q4_err_term(float w, float sc, float step) {
+__device__ __forceinline__ double q4_err(float w, float sc, float step) {
   uint32_t x = __float_as_uint(fmaf(w, sc, 12582912.0f));
   x = min(max(x, 0x4B400000u - 7u), 0x4B400000u + 7u);
   const float qv = __fmul_rn(__uint_as_float(x) - 12582912.0f, step);     // exact
-  double d;
-  if constexpr (F32) d = __dsub_rn(static_cast<double>(w), static_cast<double>(qv));
-  else d = static_cast<double>(__fsub_rn(w, qv));
-  return __dmul_rn(d, d);
+  if constexpr (F32) return __dsub_rn(static_cast<double>(w), static_cast<double>(qv));
+  else return static_cast<double>(__fsub_rn(w, qv));
 }
 
-// The same term for a block whose maximum is below 2^-125, where 2^(2-e)
-// is not a normal float: the code is found on the input pre-scaled by 2^64
-// and the difference is formed in fp64.
-__device__ __forceinline__ double q4_err_term_tiny(float w, int e) {
+// The same difference for a block whose maximum is below 2^-125, where
+// 2^(2-e) is not a normal float: the code is found on the input pre-scaled
+// by 2^64 and the difference is formed in fp64.
+__device__ __forceinline__ double q4_err_tiny(float w, int e) {
   const float sc = __uint_as_float(static_cast<uint32_t>(2 - e - 64 + 127) << 23);
   uint32_t x = __float_as_uint(fmaf(w * 18446744073709551616.0f, sc, 12582912.0f));
   x = min(max(x, 0x4B400000u - 7u), 0x4B400000u + 7u);
   const double q = static_cast<double>(__uint_as_float(x) - 12582912.0f);
-  const double d = __dsub_rn(static_cast<double>(w), __dmul_rn(q, pow2d(e - 2)));
-  return __dmul_rn(d, d);
+  return __dsub_rn(static_cast<double>(w), __dmul_rn(q, pow2d(e - 2)));
 }
 
 template <bool XF32, bool WF32, bool XVEC, bool WVEC>
@@ -139,7 +134,7 @@ __global__ void __launch_bounds__(kSensThreads) sens_partial_kernel(SensArgs a) 
       for (int u = 0; u < kRowBatch; ++u) {
         if (t + u < r1) {
 #pragma unroll
-          for (int i = 0; i < kColsPerThread; ++i) acc[i] = __dadd_rn(acc[i], square_term(v[u][i]));
+          for (int i = 0; i < kColsPerThread; ++i) acc[i] = add_square(acc[i], static_cast<double>(v[u][i]));
         }
       }
     }
@@ -170,10 +165,10 @@ __global__ void __launch_bounds__(kSensThreads) sens_partial_kernel(SensArgs a) 
             const float sc = __uint_as_float(static_cast<uint32_t>(2 - e + 127) << 23);
             const float step = pow2f(e - 2);
 #pragma unroll
-            for (int i = 0; i < kColsPerThread; ++i) acc[i] = __dadd_rn(acc[i], q4_err_term<WF32>(v[u][i], sc, step));
+            for (int i = 0; i < kColsPerThread; ++i) acc[i] = add_square(acc[i], q4_err<WF32>(v[u][i], sc, step));
           } else {
 #pragma unroll
-            for (int i = 0; i < kColsPerThread; ++i) acc[i] = __dadd_rn(acc[i], q4_err_term_tiny(v[u][i], e));
+            for (int i = 0; i < kColsPerThread; ++i) acc[i] = add_square(acc[i], q4_err_tiny(v[u][i], e));
           }
         }
       }
@@ -191,45 +186,51 @@ constexpr int kTileCPT = 8;                           // columns per thread in t
 constexpr int kTileThreads = kTileCols / kTileCPT;
 constexpr long long kTileWaitLimit = 2000000000LL;    // cycles (~1 s)
 
-// Row r of a staged tile: this thread's 8 values.
-template <bool F32>
-__device__ __forceinline__ void lds8(const uint8_t *tile, int r, int cl, float (&v)[kTileCPT]) {
-  if constexpr (F32) {
-    const float4 *p = reinterpret_cast<const float4 *>(tile + (static_cast<int64_t>(r) * kTileCols + cl) * 4);
-    const float4 a = p[0], b = p[1];
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-  } else {
-    const uint4 a = *reinterpret_cast<const uint4 *>(tile + (static_cast<int64_t>(r) * kTileCols + cl) * 2);
-    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+// Row r of a staged fp32 tile: this thread's 8 values.
+__device__ __forceinline__ void lds_row_f32(const uint8_t *tile, int r, int cl, float (&v)[kTileCPT]) {
+  const float4 *p = reinterpret_cast<const float4 *>(tile + (static_cast<int64_t>(r) * kTileCols + cl) * 4);
+  const float4 a = p[0], b = p[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// Row r of a staged bf16 tile: this thread's 8 values as 4 packed words.
+__device__ __forceinline__ void lds_row_bf16(const uint8_t *tile, int r, int cl, uint32_t (&p)[kTileCPT / 2]) {
+  const uint4 a = *reinterpret_cast<const uint4 *>(tile + (static_cast<int64_t>(r) * kTileCols + cl) * 2);
+  p[0] = a.x; p[1] = a.y; p[2] = a.z; p[3] = a.w;
+}
+
+__device__ __forceinline__ void unpack_bf16(const uint32_t (&p)[kTileCPT / 2], float (&v)[kTileCPT]) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      v[2 * j] = __uint_as_float(w[j] << 16);
-      v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-    }
+  for (int j = 0; j < kTileCPT / 2; ++j) {
+    v[2 * j] = __uint_as_float(p[j] << 16);
+    v[2 * j + 1] = __uint_as_float(p[j] & 0xFFFF0000u);
   }
 }
 
-// (w - Q4(w))^2 for a bf16 w in the common case (block exponent e >= -125):
-// the code comes from fma(w, 2^(2-e), 1.5*2^23) clamped on its bit pattern;
-// w - q*2^(e-2) has <= 9 significant bits, so the fma that forms it is exact.
-__device__ __forceinline__ double q4_err_term_bf16(float w, float sc, float step) {
-  uint32_t x = __float_as_uint(fmaf(w, sc, 12582912.0f));
-  x = min(max(x, 0x4B400000u - 7u), 0x4B400000u + 7u);
-  const float d = fmaf(-(__uint_as_float(x) - 12582912.0f), step, w);
-  const double dd = static_cast<double>(d);
-  return __dmul_rn(dd, dd);
+// max(|a|, |b|) per bf16 half (the sign of the result is dropped by the caller).
+__device__ __forceinline__ uint32_t maxabs_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
-// One row of 8 W values: adds (w - Q4(w))^2 to acc under the 32-column
-// block's maximum (shared by the 4 lanes of the block).
+// w - Q4(w) for a bf16 w in the common case (block exponent e >= -125):
+// the code comes from fma(w, 2^(2-e), 1.5*2^23) clamped on its bit pattern;
+// w - q*2^(e-2) has <= 9 significant bits, so the fma that forms it is exact.
+__device__ __forceinline__ double q4_err_bf16(float w, float sc, float step) {
+  uint32_t x = __float_as_uint(fmaf(w, sc, 12582912.0f));
+  x = min(max(x, 0x4B400000u - 7u), 0x4B400000u + 7u);
+  return static_cast<double>(fmaf(-(__uint_as_float(x) - 12582912.0f), step, w));
+}
+
+// One row of this thread's W values: adds (w - Q4(w))^2 to acc under the
+// 32-column block's exponent e (the block spans the 4 lanes that share it;
+// `ab` is this lane's largest magnitude as fp32 bits).
 template <bool F32>
-__device__ __forceinline__ void w_row_terms8(const float (&v)[kTileCPT], double (&acc)[kTileCPT]) {
-  uint32_t ab = 0;
+__device__ __forceinline__ void w_row_terms(const float (&v)[kTileCPT], uint32_t ab, double (&acc)[kTileCPT]) {
 #pragma unroll
-  for (int i = 0; i < kTileCPT; ++i) ab = max(ab, __float_as_uint(v[i]) & 0x7FFFFFFFu);
-  ab = max(ab, __shfl_xor_sync(0xffffffffu, ab, 1));
-  ab = max(ab, __shfl_xor_sync(0xffffffffu, ab, 2));
+  for (int m = 1; m < 32 / kTileCPT; m <<= 1) ab = max(ab, __shfl_xor_sync(0xffffffffu, ab, m));
   const int ef = static_cast<int>(ab >> 23);
   const int e = ef == 0 ? -127 : ef - 127;
   if (e >= -125) {
@@ -237,20 +238,21 @@ __device__ __forceinline__ void w_row_terms8(const float (&v)[kTileCPT], double 
     const float step = pow2f(e - 2);
 #pragma unroll
     for (int i = 0; i < kTileCPT; ++i) {
-      if constexpr (F32) acc[i] = __dadd_rn(acc[i], q4_err_term<true>(v[i], sc, step));
-      else acc[i] = __dadd_rn(acc[i], q4_err_term_bf16(v[i], sc, step));
+      if constexpr (F32) acc[i] = add_square(acc[i], q4_err<true>(v[i], sc, step));
+      else acc[i] = add_square(acc[i], q4_err_bf16(v[i], sc, step));
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < kTileCPT; ++i) acc[i] = __dadd_rn(acc[i], q4_err_term_tiny(v[i], e));
+    for (int i = 0; i < kTileCPT; ++i) acc[i] = add_square(acc[i], q4_err_tiny(v[i], e));
   }
 }
 
 // Tiles in launch order: all X tiles (chunk-major), then all W tiles.  A
-// tile (one 64-row chunk x 256 columns) streams through two shared-memory
+// tile (one 64-row chunk x 256 columns) streams through kSubBufs shared-memory
 // buffers of kSubRows rows, so the next rows load while these are summed
 // and a CTA needs little shared memory: many CTAs share an SM.
 constexpr int kSubRows = 8;
+constexpr int kSubBufs = 2;       // sub-tiles in flight per CTA
 
 template <bool XF32, bool WF32>
 __global__ void __launch_bounds__(kTileThreads)
@@ -259,7 +261,7 @@ __global__ void __launch_bounds__(kTileThreads)
   pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(128) uint8_t tile[];
-  __shared__ __align__(8) uint64_t bar[2];
+  __shared__ __align__(8) uint64_t bar[kSubBufs];
   const int nx = a.nchunk_x * ctiles;
   const bool is_x = static_cast<int>(blockIdx.x) < nx;
   const int t = is_x ? blockIdx.x : blockIdx.x - nx;
@@ -272,13 +274,12 @@ __global__ void __launch_bounds__(kTileThreads)
   const int rows = static_cast<int>(min(static_cast<int64_t>(kSumChunk), (is_x ? a.T : a.N) - r0));
   const int nsub = (rows + kSubRows - 1) / kSubRows;
   if (threadIdx.x == 0) {
-    ptx::mbar_init(&bar[0], 1);
-    ptx::mbar_init(&bar[1], 1);
+    for (int b = 0; b < kSubBufs; ++b) ptx::mbar_init(&bar[b], 1);
     ptx::fence_mbar_init();
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    for (int b = 0; b < 2 && b < nsub; ++b) {
+    for (int b = 0; b < kSubBufs && b < nsub; ++b) {
       ptx::mbar_arrive_expect_tx(&bar[b], sub_bytes);
       ptx::tma_load_2d(tile + b * buf_bytes, map, &bar[b], ct * kTileCols, static_cast<int>(r0) + b * kSubRows);
     }
@@ -289,12 +290,13 @@ __global__ void __launch_bounds__(kTileThreads)
 #pragma unroll
   for (int i = 0; i < kTileCPT; ++i) acc[i] = 0.0;
   for (int sb = 0; sb < nsub; ++sb) {
-    const int buf = sb & 1;
-    if (!ptx::mbar_wait_cycles(&bar[buf], (sb >> 1) & 1, kTileWaitLimit)) {
-      // the other buffer's load, if any, lands before the CTA exits
+    const int buf = sb % kSubBufs;
+    if (!ptx::mbar_wait_cycles(&bar[buf], (sb / kSubBufs) & 1, kTileWaitLimit)) {
+      // the other buffers' loads, if any, land before the CTA exits
       if (threadIdx.x == 0) {
         atomicExch(status, static_cast<int>(MXS_ERR_TIMEOUT));
-        if (sb + 1 < nsub) ptx::mbar_wait_cycles(&bar[buf ^ 1], ((sb + 1) >> 1) & 1, kTileWaitLimit);
+        for (int b = sb + 1; b < sb + kSubBufs && b < nsub; ++b)
+          ptx::mbar_wait_cycles(&bar[b % kSubBufs], (b / kSubBufs) & 1, kTileWaitLimit);
       }
       return;
     }
@@ -304,23 +306,42 @@ __global__ void __launch_bounds__(kTileThreads)
 #pragma unroll 8
       for (int r = 0; r < rr; ++r) {
         float v[kTileCPT];
-        lds8<XF32>(sub, r, cl, v);
+        if constexpr (XF32) {
+          lds_row_f32(sub, r, cl, v);
+        } else {
+          uint32_t p[kTileCPT / 2];
+          lds_row_bf16(sub, r, cl, p);
+          unpack_bf16(p, v);
+        }
 #pragma unroll
-        for (int i = 0; i < kTileCPT; ++i) acc[i] = __dadd_rn(acc[i], square_term(v[i]));
+        for (int i = 0; i < kTileCPT; ++i) acc[i] = add_square(acc[i], static_cast<double>(v[i]));
       }
     } else {
 #pragma unroll 4
       for (int r = 0; r < rr; ++r) {     // rr is uniform over the CTA
         float v[kTileCPT];
-        lds8<WF32>(sub, r, cl, v);
-        w_row_terms8<WF32>(v, acc);
+        uint32_t ab;
+        if constexpr (WF32) {
+          lds_row_f32(sub, r, cl, v);
+          ab = 0;
+#pragma unroll
+          for (int i = 0; i < kTileCPT; ++i) ab = max(ab, __float_as_uint(v[i]) & 0x7FFFFFFFu);
+        } else {
+          uint32_t p[kTileCPT / 2];
+          lds_row_bf16(sub, r, cl, p);
+          unpack_bf16(p, v);
+          const uint32_t m = maxabs_bf16x2(maxabs_bf16x2(p[0], p[1]), maxabs_bf16x2(p[2], p[3])) & 0x7FFF7FFFu;
+          ab = max(m << 16, m & 0xFFFF0000u);      // the larger half, as fp32 bits
+        }
+        w_row_terms<WF32>(v, ab, acc);
       }
     }
-    // the warp is done with this buffer: it takes the rows two sub-tiles on
+    // the warp is done with this buffer: it takes the rows kSubBufs sub-tiles on
     __syncthreads();
-    if (threadIdx.x == 0 && sb + 2 < nsub) {
+    if (threadIdx.x == 0 && sb + kSubBufs < nsub) {
       ptx::mbar_arrive_expect_tx(&bar[buf], sub_bytes);
-      ptx::tma_load_2d(tile + buf * buf_bytes, map, &bar[buf], ct * kTileCols, static_cast<int>(r0) + (sb + 2) * kSubRows);
+      ptx::tma_load_2d(tile + buf * buf_bytes, map, &bar[buf], ct * kTileCols,
+                       static_cast<int>(r0) + (sb + kSubBufs) * kSubRows);
     }
   }
   double *out = a.part + static_cast<int64_t>(is_x ? chunk : a.nchunk_x + chunk) * a.K + c0;
@@ -441,7 +462,7 @@ extern "C" mxs_status mxs_sensitivity(const void *X, mxs_dtype xt, int64_t T, in
                        static_cast<int>(dtype_size(xt)), X, K, T, ldx, kTileCols, kSubRows) &&
         make_plain_map(&mw, wf ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                        static_cast<int>(dtype_size(wt)), W, K, N, ldw, kTileCols, kSubRows)) {
-      const int smem = 2 * kSubRows * kTileCols * ((xf || wf) ? 4 : 2);
+      const int smem = kSubBufs * kSubRows * kTileCols * ((xf || wf) ? 4 : 2);
       const unsigned g = static_cast<unsigned>(ntiles);
       const int32_t ct = static_cast<int32_t>(ctiles);
       if (xf && wf) {

@@ -243,9 +243,14 @@ __device__ __forceinline__ void dec_segment(const SmallArgs &a, const uint8_t *s
 
 constexpr long long kDecWaitLimit = 2000000000LL;    // cycles (~1 s)
 
-// One CTA: W rows n0 .. n0+15.  Thread 0 bulk-copies the activations' code
-// and scale rows and the 16 W rows' scale rows into shared memory; the warps
-// then run the three segments and add their partial sums in warp order.
+// One CTA: W rows n0 .. n0+15.  Rows of a packed segment lie at a fixed
+// pitch, so the activations' code rows, their scale rows and the CTA's W
+// scale (and, when staged, code) rows are each one contiguous range: one
+// thread bulk-copies them into shared memory with one copy per range (a
+// dozen copies, not one per row, which the copy engine would take one by
+// one); W rows past N are not copied and only feed outputs that are never
+// stored.  The warps then run the three segments and add their partial sums
+// in warp order.
 __global__ void __launch_bounds__(kDecThreads) gemm_small_kernel(SmallArgs a, int *status) {
   pdl_wait();
   pdl_trigger();
@@ -260,26 +265,24 @@ __global__ void __launch_bounds__(kDecThreads) gemm_small_kernel(SmallArgs a, in
     ptx::fence_mbar_init();
   }
   __syncthreads();
-  if (warp == 0) {
-    // copies: per segment, M activation code rows, M scale rows, 16 W scale rows
-    if (lane == 0) ptx::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(sp.bytes));
-    __syncwarp();
+  if (threadIdx.x == 0) {
+    const int wrows = min(kDecRows, a.N - n0);        // W rows of this CTA that exist
+    uint32_t bytes = 0;
     for (int g = 0; g < 3; ++g) {
       if (!a.nb[g]) continue;
-      for (int r = lane; r < a.M; r += 32) {
-        ptx::bulk_load(smem + sp.a_code[g] + r * a.a_cpitch[g], a.a_codes[g] + r * a.a_cpitch[g],
-                       static_cast<uint32_t>(a.a_cpitch[g]), &bar);
-        ptx::bulk_load(smem + sp.a_scale[g] + r * a.a_spitch[g], a.a_scales[g] + r * a.a_spitch[g],
-                       static_cast<uint32_t>(a.a_spitch[g]), &bar);
-      }
-      for (int r = lane; r < kDecRows; r += 32) {
-        const int64_t wr = min(n0 + r, a.N - 1);
-        ptx::bulk_load(smem + sp.w_scale[g] + r * a.w_spitch[g], a.w_scales[g] + wr * a.w_spitch[g],
-                       static_cast<uint32_t>(a.w_spitch[g]), &bar);
-        if (a.stage_w)
-          ptx::bulk_load(smem + sp.w_code[g] + r * a.w_cpitch[g], a.w_codes[g] + wr * a.w_cpitch[g],
-                         static_cast<uint32_t>(a.w_cpitch[g]), &bar);
-      }
+      bytes += static_cast<uint32_t>(a.M * (a.a_cpitch[g] + a.a_spitch[g]) + wrows * a.w_spitch[g]);
+      if (a.stage_w) bytes += static_cast<uint32_t>(wrows * a.w_cpitch[g]);
+    }
+    ptx::mbar_arrive_expect_tx(&bar, bytes);
+    for (int g = 0; g < 3; ++g) {
+      if (!a.nb[g]) continue;
+      ptx::bulk_load(smem + sp.a_code[g], a.a_codes[g], static_cast<uint32_t>(a.M * a.a_cpitch[g]), &bar);
+      ptx::bulk_load(smem + sp.a_scale[g], a.a_scales[g], static_cast<uint32_t>(a.M * a.a_spitch[g]), &bar);
+      ptx::bulk_load(smem + sp.w_scale[g], a.w_scales[g] + static_cast<int64_t>(n0) * a.w_spitch[g],
+                     static_cast<uint32_t>(wrows * a.w_spitch[g]), &bar);
+      if (a.stage_w)
+        ptx::bulk_load(smem + sp.w_code[g], a.w_codes[g] + static_cast<int64_t>(n0) * a.w_cpitch[g],
+                       static_cast<uint32_t>(wrows * a.w_cpitch[g]), &bar);
     }
   }
   float acc[2][4];

@@ -249,40 +249,45 @@ constexpr long long kDecWaitLimit = 2000000000LL;    // cycles (~1 s)
 // thread bulk-copies them into shared memory with one copy per range (a
 // dozen copies, not one per row, which the copy engine would take one by
 // one); W rows past N are not copied and only feed outputs that are never
-// stored.  The warps then run the three segments and add their partial sums
-// in warp order.
+// stored.  The copies complete on two barriers: the scale rows with the 8-
+// and 6-bit codes, then the 4-bit codes, so the warps run the 8- and 6-bit
+// segments while the 4-bit codes are still landing.  Then they add their
+// partial sums in warp order.
 __global__ void __launch_bounds__(kDecThreads) gemm_small_kernel(SmallArgs a, int *status) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ __align__(8) uint64_t bar;
+  __shared__ __align__(8) uint64_t bar[2];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gid = lane >> 2, tig = lane & 3;
   const int n0 = blockIdx.x * kDecRows;
   const DecSmem sp = dec_smem_plan(a);
   if (threadIdx.x == 0) {
-    ptx::mbar_init(&bar, 1);
+    ptx::mbar_init(&bar[0], 1);
+    ptx::mbar_init(&bar[1], 1);
     ptx::fence_mbar_init();
   }
   __syncthreads();
   if (threadIdx.x == 0) {
     const int wrows = min(kDecRows, a.N - n0);        // W rows of this CTA that exist
-    uint32_t bytes = 0;
+    uint32_t bytes[2] = {0u, 0u};
     for (int g = 0; g < 3; ++g) {
       if (!a.nb[g]) continue;
-      bytes += static_cast<uint32_t>(a.M * (a.a_cpitch[g] + a.a_spitch[g]) + wrows * a.w_spitch[g]);
-      if (a.stage_w) bytes += static_cast<uint32_t>(wrows * a.w_cpitch[g]);
+      bytes[0] += static_cast<uint32_t>(a.M * a.a_spitch[g] + wrows * a.w_spitch[g]);
+      bytes[g == 2] += static_cast<uint32_t>(a.M * a.a_cpitch[g] + (a.stage_w ? wrows * a.w_cpitch[g] : 0));
     }
-    ptx::mbar_arrive_expect_tx(&bar, bytes);
+    ptx::mbar_arrive_expect_tx(&bar[0], bytes[0]);
+    ptx::mbar_arrive_expect_tx(&bar[1], bytes[1]);
     for (int g = 0; g < 3; ++g) {
       if (!a.nb[g]) continue;
-      ptx::bulk_load(smem + sp.a_code[g], a.a_codes[g], static_cast<uint32_t>(a.M * a.a_cpitch[g]), &bar);
-      ptx::bulk_load(smem + sp.a_scale[g], a.a_scales[g], static_cast<uint32_t>(a.M * a.a_spitch[g]), &bar);
+      uint64_t *cb = &bar[g == 2];
+      ptx::bulk_load(smem + sp.a_scale[g], a.a_scales[g], static_cast<uint32_t>(a.M * a.a_spitch[g]), &bar[0]);
       ptx::bulk_load(smem + sp.w_scale[g], a.w_scales[g] + static_cast<int64_t>(n0) * a.w_spitch[g],
-                     static_cast<uint32_t>(wrows * a.w_spitch[g]), &bar);
+                     static_cast<uint32_t>(wrows * a.w_spitch[g]), &bar[0]);
+      ptx::bulk_load(smem + sp.a_code[g], a.a_codes[g], static_cast<uint32_t>(a.M * a.a_cpitch[g]), cb);
       if (a.stage_w)
         ptx::bulk_load(smem + sp.w_code[g], a.w_codes[g] + static_cast<int64_t>(n0) * a.w_cpitch[g],
-                       static_cast<uint32_t>(wrows * a.w_cpitch[g]), &bar);
+                       static_cast<uint32_t>(wrows * a.w_cpitch[g]), cb);
     }
   }
   float acc[2][4];
@@ -290,18 +295,26 @@ __global__ void __launch_bounds__(kDecThreads) gemm_small_kernel(SmallArgs a, in
   for (int j = 0; j < 2; ++j)
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
-  const bool landed = ptx::mbar_wait_cycles(&bar, 0, kDecWaitLimit);
-  if (__syncthreads_or(!landed)) {                    // uniform: every thread leaves together
-    if (threadIdx.x == 0) atomicExch(status, static_cast<int>(MXS_ERR_TIMEOUT));
-    return;     // the copies are the wait that expired: nothing else is in flight
-  }
+  auto part = [&](int c) -> bool {
+    const bool landed = ptx::mbar_wait_cycles(&bar[c], 0, kDecWaitLimit);
+    if (!__syncthreads_or(!landed)) return true;
+    if (threadIdx.x == 0) {
+      atomicExch(status, static_cast<int>(MXS_ERR_TIMEOUT));
+      if (c == 0) ptx::mbar_wait_cycles(&bar[1], 0, kDecWaitLimit);
+    }
+    return false;
+  };
   if (a.stage_w) {
+    if (!part(0)) return;
     dec_segment<0, true>(a, smem, sp, n0, acc);
     dec_segment<1, true>(a, smem, sp, n0, acc);
+    if (!part(1)) return;
     dec_segment<2, true>(a, smem, sp, n0, acc);
   } else {
+    if (!part(0)) return;
     dec_segment<0, false>(a, smem, sp, n0, acc);
     dec_segment<1, false>(a, smem, sp, n0, acc);
+    if (!part(1)) return;
     dec_segment<2, false>(a, smem, sp, n0, acc);
   }
   // the warps' partial sums, added in warp order

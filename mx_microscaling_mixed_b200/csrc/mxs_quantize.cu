@@ -621,29 +621,36 @@ __device__ __forceinline__ void encode2_store(const uint32_t (&v)[kBlock], uint8
     for (int t = 0; t < kBlock; ++t) r[t] = fma_bf16x2(minabs_bf16x2(v[t], c2), s2, 0x43404340u);
     *s0 = static_cast<uint8_t>(ef0);
     if (has1) *s1 = static_cast<uint8_t>(ef1);
-    // x0[j] / x1[j]: the low bytes of positions 4j..4j+3 of row 0 / row 1
-    uint32_t x0[8], x1[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t A = __byte_perm(r[4 * j], r[4 * j + 1], 0x6240);
-      const uint32_t B = __byte_perm(r[4 * j + 2], r[4 * j + 3], 0x6240);
-      x0[j] = __byte_perm(A, B, 0x5410);
-      x1[j] = __byte_perm(A, B, 0x7632);
-    }
     if constexpr (M == 4) {
+      // a lane's low nibble is the code (0x40 + q).  Word pair (r[2i], r[2i+1])
+      // -> t: byte 0 = row 0's codes of positions 2i, 2i+1 (low nibble first),
+      // byte 2 = row 1's, by one select of r[2i]'s low nibbles against
+      // r[2i+1] shifted up a nibble; bytes 1 and 3 are never read
       uint32_t w0[4], w1[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint32_t a0 = (x0[2 * j] & 0x0F0F0F0Fu) | ((x0[2 * j] >> 4) & 0xF0F0F0F0u);
-        const uint32_t b0 = (x0[2 * j + 1] & 0x0F0F0F0Fu) | ((x0[2 * j + 1] >> 4) & 0xF0F0F0F0u);
-        w0[j] = __byte_perm(a0, b0, 0x6420);
-        const uint32_t a1 = (x1[2 * j] & 0x0F0F0F0Fu) | ((x1[2 * j] >> 4) & 0xF0F0F0F0u);
-        const uint32_t b1 = (x1[2 * j + 1] & 0x0F0F0F0Fu) | ((x1[2 * j + 1] >> 4) & 0xF0F0F0F0u);
-        w1[j] = __byte_perm(a1, b1, 0x6420);
+        uint32_t t[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t a = r[8 * j + 2 * k], b = r[8 * j + 2 * k + 1] << 4;
+          t[k] = (a & 0x000F000Fu) | (b & 0xFFF0FFF0u);
+        }
+        const uint32_t u0 = __byte_perm(t[0], t[1], 0x6240), u1 = __byte_perm(t[2], t[3], 0x6240);
+        w0[j] = __byte_perm(u0, u1, 0x5410);      // row 0, positions 8j .. 8j+7
+        w1[j] = __byte_perm(u0, u1, 0x7632);      // row 1
       }
       *reinterpret_cast<uint4 *>(c0) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
       if (has1) *reinterpret_cast<uint4 *>(c1) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
     } else {
+      // x0[j] / x1[j]: the low bytes of positions 4j..4j+3 of row 0 / row 1
+      uint32_t x0[8], x1[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t A = __byte_perm(r[4 * j], r[4 * j + 1], 0x6240);
+        const uint32_t B = __byte_perm(r[4 * j + 2], r[4 * j + 3], 0x6240);
+        x0[j] = __byte_perm(A, B, 0x5410);
+        x1[j] = __byte_perm(A, B, 0x7632);
+      }
       uint32_t u0[8], u1[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {

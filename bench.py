@@ -198,6 +198,24 @@ class Path:
             fn()
 
 
+def max_over_ranks(t: float, world: int, device) -> float:
+    """The job's time for a per-rank time t: the slowest rank's (a MAX
+    all-reduce over the process group, which every rank joins)."""
+    if world == 1:
+        return t
+    import torch
+    import torch.distributed as dist
+    tt = torch.tensor([t], device=device, dtype=torch.float64)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def job_tflops(flops_per_rank_step: float, steps: int, world: int, job_s: float) -> float:
+    """Whole-job throughput: the work of every rank (each runs its own replica
+    of the workload: weak scaling) over the slowest rank's time."""
+    return world * flops_per_rank_step * steps / job_s / 1e12
+
+
 def traffic_from_profile(pk_name: str):
     """dram bytes per launch recorded in profiles/, if the kernel source is unchanged since."""
     prof = os.path.join(ROOT, "profiles", pk_name)
@@ -294,12 +312,8 @@ def run_gpu(args, rank, world, local_rank):
     launches = launches_per_step * args.steps
     c.mxs_sync()
     step_ms = [s.elapsed_time(e) for s, e in step_ev]
-    total_s = sum(step_ms) * 1e-3
-    if world > 1:
-        tt = torch.tensor([total_s], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_s = float(tt.item())
-    value = world * path.gemm_flops * args.steps / total_s / 1e12
+    total_s = max_over_ranks(sum(step_ms) * 1e-3, world, dev)
+    value = job_tflops(path.gemm_flops, args.steps, world, total_s)
     best = {name: min(s.elapsed_time(e) for s, e in evs) * 1e-3 for name, evs in rec.items()}
     per_call = {name: max(best[name] - best[""], 0.0) / CALL_REPS for name, _ in calls}
     call_sum = sum(per_call.values())
@@ -394,13 +408,8 @@ def run_e2e(path, args, dev, world):
         torch.cuda.synchronize()
         if i:
             ms.append(s.elapsed_time(e))
-    t = sum(ms) / len(ms) * 1e-3
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([t], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t = float(tt.item())
-    return {"value": world * path.gemm_flops / t / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+    t = max_over_ranks(sum(ms) / len(ms) * 1e-3, world, dev)
+    return {"value": job_tflops(path.gemm_flops, 1, world, t), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": t * 1e3}
 
 

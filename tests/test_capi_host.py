@@ -115,3 +115,34 @@ def test_quantize_argument_checks(capi):
     assert capi._lib.mxs_quantize_act(1 << 20, 7, 8, 64, ctypes.byref(t), None) == 4
     # ld < K
     assert capi._lib.mxs_quantize_weight(1 << 20, 0, 8, 32, ctypes.byref(t), None) == 2
+
+
+def test_sensitivity_argument_checks(capi):
+    f = capi._lib.mxs_sensitivity
+    X, W, H, E, S = 1 << 20, 1 << 24, 1 << 26, 1 << 27, 1 << 28
+    need = ctypes.c_size_t(0)
+    assert capi._lib.mxs_sensitivity_workspace_bytes(128, 256, 512, ctypes.byref(need)) == 0
+    ws, big = 1 << 30, need.value
+    # NULL input -> MXS_ERR_ARG
+    assert f(None, 1, 128, 512, 512, W, 1, 256, 512, H, E, S, ws, big, None) == 1
+    # T < 1 -> MXS_ERR_ARG
+    assert f(X, 1, 0, 512, 512, W, 1, 256, 512, H, E, S, ws, big, None) == 1
+    # unknown dtype -> MXS_ERR_DTYPE
+    assert f(X, 9, 128, 512, 512, W, 1, 256, 512, H, E, S, ws, big, None) == 4
+    # pitch below K -> MXS_ERR_SHAPE
+    assert f(X, 1, 128, 512, 511, W, 1, 256, 512, H, E, S, ws, big, None) == 2
+    assert f(X, 1, 128, 512, 512, W, 1, 256, 500, H, E, S, ws, big, None) == 2
+    # more 64-row chunks than one launch takes -> MXS_ERR_SHAPE
+    assert f(X, 1, 64 * 65536, 512, 512, W, 1, 256, 512, H, E, S, ws, 1 << 62, None) == 2
+    # workspace missing, misaligned or short -> MXS_ERR_WORKSPACE
+    assert f(X, 1, 128, 512, 512, W, 1, 256, 512, H, E, S, None, big, None) == 9
+    assert f(X, 1, 128, 512, 512, W, 1, 256, 512, H, E, S, ws + 64, big, None) == 9
+    assert f(X, 1, 128, 512, 512, W, 1, 256, 512, H, E, S, ws, big - 8, None) == 9
+
+
+def test_gemm_empty_product_needs_no_device(capi):
+    lay = capi.mxs_layout_make(256, (32, 64, 160))
+    A0 = _fake_tensor(capi, 0, lay)
+    W = _fake_tensor(capi, 300, lay)
+    # M = 0: nothing to compute, MXS_OK before any device work
+    assert capi._lib.mxs_gemm(ctypes.byref(A0), ctypes.byref(W), 1 << 24, 300, None, 0, None) == 0

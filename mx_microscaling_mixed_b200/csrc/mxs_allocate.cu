@@ -209,6 +209,20 @@ extern "C" mxs_status mxs_allocate_workspace_bytes(int32_t n_layers, const int64
   return MXS_OK;
 }
 
+// Budget mode: the bit budget (num/den bits per weight over all layers)
+// times den, and what the 4-bit columns plus the fixed 8-bit block already
+// use of it.  Infeasible when used > cap.
+static void budget_base(int32_t n_layers, const int64_t *K, const int64_t *N, const mxs_budget &B, __int128 &cap,
+                        __int128 &used) {
+  cap = 0;
+  used = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    const int64_t n8 = std::min<int64_t>(B.fixed8, K[l]);
+    cap += static_cast<__int128>(B.num) * N[l] * K[l];
+    used += static_cast<__int128>(B.den) * N[l] * (4 * K[l] + 4 * n8);
+  }
+}
+
 extern "C" mxs_status mxs_allocate(int32_t n_layers, const int64_t *K, const int64_t *N,
                                    const double *const *s, const double *layer_w,
                                    const mxs_budget *budget, int32_t *const *perm,
@@ -223,6 +237,9 @@ extern "C" mxs_status mxs_allocate(int32_t n_layers, const int64_t *K, const int
     if (B.p8_den <= 0 || B.p6_den <= 0 || B.p8_num < 0 || B.p6_num < 0) return MXS_ERR_ARG;
   } else if (B.mode == MXS_ALLOC_BUDGET) {
     if (B.den <= 0 || B.num < 0 || B.fixed8 < 0) return MXS_ERR_ARG;
+    __int128 cap, used;
+    budget_base(n_layers, K, N, B, cap, used);
+    if (used > cap) return MXS_ERR_BUDGET;           // before any launch
   } else {
     return MXS_ERR_ARG;
   }
@@ -252,13 +269,9 @@ extern "C" mxs_status mxs_allocate(int32_t n_layers, const int64_t *K, const int
       n6[l] = std::min(round_half_up_frac(B.p6_num, B.p6_den, K[l]), K[l] - n8[l]);
     }
   } else {
-    __int128 cap = 0, used = 0;
-    for (int l = 0; l < n_layers; ++l) {
-      n8[l] = std::min(B.fixed8, K[l]);
-      cap += static_cast<__int128>(B.num) * N[l] * K[l];
-      used += static_cast<__int128>(B.den) * N[l] * (4 * K[l] + 4 * n8[l]);
-    }
-    if (used > cap) return MXS_ERR_BUDGET;
+    __int128 cap, used;
+    budget_base(n_layers, K, N, B, cap, used);     // feasible: checked above
+    for (int l = 0; l < n_layers; ++l) n8[l] = std::min(B.fixed8, K[l]);
     std::vector<std::vector<double>> gains(n_layers);
     if (n_layers > 1) {
       for (int l = 0; l < n_layers; ++l) {

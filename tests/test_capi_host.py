@@ -146,3 +146,30 @@ def test_gemm_empty_product_needs_no_device(capi):
     W = _fake_tensor(capi, 300, lay)
     # M = 0: nothing to compute, MXS_OK before any device work
     assert capi._lib.mxs_gemm(ctypes.byref(A0), ctypes.byref(W), 1 << 24, 300, None, 0, None) == 0
+
+
+def _alloc_call(capi, K, N, budget, ws=1 << 30, ws_bytes=1 << 40):
+    n = len(K)
+    Ks, Ns = (ctypes.c_int64 * n)(*K), (ctypes.c_int64 * n)(*N)
+    s = (ctypes.c_void_p * n)(*[(1 << 20) + 65536 * i for i in range(n)])
+    perm = (ctypes.c_void_p * n)(*[(1 << 24) + 65536 * i for i in range(n)])
+    counts = (ctypes.c_int64 * (3 * n))()
+    return capi._lib.mxs_allocate(n, Ks, Ns, s, None, ctypes.byref(budget), perm, counts, ws, ws_bytes, None)
+
+
+def test_allocate_argument_and_budget_checks(capi):
+    # budget mode: 4.0 bits on average cannot carry the fixed 32-column 8-bit
+    # block -> MXS_ERR_BUDGET, decided on the host before any launch
+    b = capi.BudgetC(mode=1, num=4, den=1, fixed8=32)
+    assert _alloc_call(capi, [4096], [4096], b) == 5
+    assert _alloc_call(capi, [4096, 14336], [4096, 4096], b) == 5
+    # a bad mode or denominator -> MXS_ERR_ARG
+    assert _alloc_call(capi, [4096], [4096], capi.BudgetC(mode=7, num=9, den=2, fixed8=32)) == 1
+    assert _alloc_call(capi, [4096], [4096], capi.BudgetC(mode=1, num=9, den=0, fixed8=32)) == 1
+    assert _alloc_call(capi, [4096], [4096], capi.BudgetC(mode=0, p8_num=1, p8_den=0, p6_num=0, p6_den=1)) == 1
+    # K < 1 -> MXS_ERR_ARG
+    assert _alloc_call(capi, [0], [4096], capi.BudgetC(mode=1, num=9, den=2, fixed8=32)) == 1
+    # feasible budget, workspace missing or short -> MXS_ERR_WORKSPACE
+    ok = capi.BudgetC(mode=1, num=9, den=2, fixed8=32)
+    assert _alloc_call(capi, [4096], [4096], ok, ws=None) == 9
+    assert _alloc_call(capi, [4096], [4096], ok, ws_bytes=16) == 9

@@ -1057,8 +1057,12 @@ extern "C" mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, voi
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   const int sgrid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((sa.start[4] + 255) / 256, static_cast<int64_t>(nsm) * 8)));
-  launch_pdl(gemm_stage_kernel, dim3(sgrid), dim3(256), 0, cs, sa);
-  count_launch();
+  // the staging kernel goes out right before the tensor-core kernel, after
+  // every host step that can fail: a failed call launches nothing
+  auto launch_stage = [&]() {
+    launch_pdl(gemm_stage_kernel, dim3(sgrid), dim3(256), 0, cs, sa);
+    count_launch();
+  };
 
   CUtensorMap mA16{}, mB16{}, mA8{}, mB8{};
   if (p.k16 > 0) {
@@ -1104,6 +1108,7 @@ extern "C" mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, voi
     if (!ensure_smem(gemm_tc2_kernel, kP2SmemBytes)) return MXS_ERR_CUDA;
     const int tiles = pa.m_tiles * pa.n_tiles;
     const int pairs = std::max(1, std::min(tiles, nsm / 2));
+    launch_stage();
     launch_pdl(gemm_tc2_kernel, dim3(2 * pairs), dim3(kP2Threads), kP2SmemBytes, cs, mA16, mB16, mA8, mB8, mSFA, mSFB, mY,
                pa);
     count_launch();
@@ -1123,6 +1128,7 @@ extern "C" mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, voi
   ga.y_vec = y_vec;
   if (!ensure_smem(gemm_tc_kernel, kGemmSmemBytes)) return MXS_ERR_CUDA;
   dim3 grid(static_cast<unsigned>((N + kBN - 1) / kBN), static_cast<unsigned>((M + kBM - 1) / kBM));
+  launch_stage();
   launch_pdl(gemm_tc_kernel, dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, cs, mA16, mB16, mA8, mB8, ga);
   count_launch();
   return cuda_status(cudaGetLastError());

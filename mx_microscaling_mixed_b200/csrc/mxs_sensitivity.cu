@@ -8,10 +8,12 @@
 //
 // Rounding order (pinned so that every launch shape gives the same bits):
 // rows are cut into chunks of 64; a chunk is summed from zero in row order in
-// fp64; chunk sums are then added in chunk order.  Each term is one fp64
-// product (a square of an fp32/bf16 value, exact; or of the exact fp64
-// difference W - Q4(W)), formed and added with explicit round-to-nearest
-// intrinsics so that no fused multiply-add can change the result.
+// fp64; chunk sums are then added in chunk order.  Each term is the square
+// of an fp32/bf16 value or of the exact difference W - Q4(W); both have at
+// most 26 significant bits, so the square is exact in fp64 and one fused
+// multiply-add adds it with a single rounding, the same bits as a rounded
+// product followed by a rounded add.  The remaining operations use explicit
+// round-to-nearest intrinsics, so no contraction can change the result.
 //
 // Two launches.  (1) Chunk partials: one CTA (one warp) per 64-row chunk x
 // 256-column tile of X or of W; one thread streams the chunk through two

@@ -173,3 +173,39 @@ def test_allocate_argument_and_budget_checks(capi):
     ok = capi.BudgetC(mode=1, num=9, den=2, fixed8=32)
     assert _alloc_call(capi, [4096], [4096], ok, ws=None) == 9
     assert _alloc_call(capi, [4096], [4096], ok, ws_bytes=16) == 9
+
+
+def test_host_checks_survive_random_arguments(capi):
+    """Random shapes, pitches and pointers return a status and never crash the
+    process.  Some combinations pass every host check and would reach a
+    launch on fake pointers, so this runs only where no CUDA device exists
+    (the device check then fails first)."""
+    import random
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("would launch kernels on fake pointers where a device exists")
+    rng = random.Random(1234)
+    valid = set(range(10))
+    for _ in range(400):
+        K = rng.choice([0, 1, 31, 32, 33, 256, 4096, 1 << 20])
+        counts = [rng.choice([0, 1, 32, 64, K]) for _ in range(2)]
+        counts.append(K - sum(counts))
+        try:
+            lay = capi.mxs_layout_make(K, counts)
+        except Exception:
+            continue
+        for rows in (0, 1, 16, 2048):
+            t = _fake_tensor(capi, rows, lay, base=rng.choice([1 << 20, (1 << 20) + 8]))
+            if rng.random() < 0.3:
+                t.code_pitch[rng.randrange(3)] = rng.choice([1, 15, 17, 1 << 40])
+            w = _fake_tensor(capi, rng.choice([1, 300, 4096]), lay)
+            need = ctypes.c_size_t(0)
+            assert capi._lib.mxs_gemm_workspace_bytes(ctypes.byref(t), ctypes.byref(w), ctypes.byref(need)) in valid
+            assert capi._lib.mxs_gemm(ctypes.byref(t), ctypes.byref(w), rng.choice([None, 1 << 24]),
+                                      rng.choice([0, 1, 4096]), rng.choice([None, 1 << 30, (1 << 30) + 4]),
+                                      rng.choice([0, 1 << 40]), None) in valid
+            dt = rng.choice([0, 1, 2, -1])
+            ld = rng.choice([0, K, K + 1, 1 << 33])
+            assert capi._lib.mxs_quantize_act(rng.choice([None, 1 << 20, (1 << 20) + 2]), dt, rows, ld,
+                                              ctypes.byref(t), None) in valid
+            assert capi._lib.mxs_quantize_weight(1 << 20, dt, rows, ld, ctypes.byref(t), None) in valid

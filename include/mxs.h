@@ -168,6 +168,10 @@ mxs_status mxs_sensitivity(const void *X, mxs_dtype xt, int64_t T, int64_t K, in
  *   before any launch.  No memory is allocated.
  *   The first call on a device looks up the array's address (with that
  *   device current); make one call on each device before any stream capture.
+ *   A device reset (cudaDeviceReset) moves the array: the first call after
+ *   it looks the address up again, so it too belongs outside any capture.
+ *   Argument checks and return codes are those of mxs_sensitivity; they run
+ *   before the device is touched.
  *   Every call shares the one array: calls that overlap on the GPU (other
  *   streams, other host threads) race on it and must be serialised by the
  *   caller.  Nothing in the array needs to start at zero.

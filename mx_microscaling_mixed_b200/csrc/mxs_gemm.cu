@@ -923,17 +923,24 @@ bool make_plain_map(CUtensorMap *m, CUtensorMapDataType dt, int esize, const voi
 }
 
 int *device_status_word() {
-  static int *addr[64] = {};
+  struct Entry {
+    unsigned long long ctx;
+    int *addr;
+  };
+  static Entry cache[64] = {};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  const unsigned long long ctx = current_context_id();
+  if (!ctx || cache[dev].ctx != ctx || !cache[dev].addr) {
+    // first use on this device, or its context was reset since: the
+    // symbol's address belongs to the current context's module
     void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
-    addr[dev] = static_cast<int *>(p);
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess || !p) return nullptr;
+    cache[dev] = Entry{current_context_id(), static_cast<int *>(p)};
   }
-  return addr[dev];
+  return cache[dev].addr;
 }
 
 // 2-D byte map with 128-byte rows, no swizzle: the scale-chunk arrays seen as

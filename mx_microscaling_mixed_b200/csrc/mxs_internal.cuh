@@ -31,6 +31,13 @@ inline bool dtype_ok(mxs_dtype t) { return t == MXS_F32 || t == MXS_BF16; }
 // Checks that the current device is a compute-capability 10.x part.
 mxs_status check_device();
 
+// Unique id of the CUDA context current on this thread (the driver's
+// context id, unique for the life of the process), or 0 when no context is
+// current yet.  Per-device caches of device addresses and kernel attributes
+// are keyed by it, so that a device reset (which destroys the context and
+// with it every module's device addresses) invalidates them.
+unsigned long long current_context_id();
+
 // Validates a layout against its own invariants (host only).
 mxs_status check_layout(const mxs_layout *lay);
 

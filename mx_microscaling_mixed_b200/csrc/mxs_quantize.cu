@@ -48,27 +48,53 @@ void count_launch(int n) {
   g_launches += n;
 }
 
+unsigned long long current_context_id() {
+  typedef CUresult (*GetCurrentFn)(CUcontext *);
+  typedef CUresult (*GetIdFn)(CUcontext, unsigned long long *);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(p);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
 bool ensure_smem_impl(const void *kernel, int bytes) {
   struct Entry {
     const void *fn;
-    int dev;
+    unsigned long long ctx;
     int bytes;
   };
   static Entry table[256];
   static int used = 0;
   static std::mutex mu;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return false;
   std::lock_guard<std::mutex> lk(mu);
-  for (int i = 0; i < used; ++i)
-    if (table[i].fn == kernel && table[i].dev == dev && table[i].bytes >= bytes) return true;
+  unsigned long long ctx = current_context_id();
+  if (ctx)
+    for (int i = 0; i < used; ++i)
+      if (table[i].fn == kernel && table[i].ctx == ctx && table[i].bytes >= bytes) return true;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  ctx = current_context_id();   // the call above made the context current if it was not
+  if (!ctx) return true;
   for (int i = 0; i < used; ++i)
-    if (table[i].fn == kernel && table[i].dev == dev) {
+    if (table[i].fn == kernel && table[i].ctx == ctx) {
       table[i].bytes = bytes;
       return true;
     }
-  if (used < 256) table[used++] = Entry{kernel, dev, bytes};
+  if (used < 256) table[used++] = Entry{kernel, ctx, bytes};
   return true;
 }
 

@@ -505,21 +505,28 @@ namespace mxs {
 constexpr size_t kNoAllocScratchBytes = MXS_NOALLOC_SCRATCH_BYTES;   // 16 MiB: 2 Mi chunk partials
 __device__ __align__(256) uint8_t g_sens_scratch[kNoAllocScratchBytes];
 
-// Address of the scratch array on the current device, looked up once per
-// device (with that device current) and kept.
+// Address of the scratch array in the current device's context.  It is
+// looked up once per device with that device current, and again only when
+// the context has changed since (a device reset destroys the context, and
+// the module's arrays move with the new one).
 static mxs_status sens_scratch(void **ptr) {
-  static void *addr[64] = {};
+  struct Entry {
+    unsigned long long ctx;
+    void *addr;
+  };
+  static Entry cache[64] = {};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MXS_ERR_CUDA;
   if (dev < 0 || dev >= 64) return MXS_ERR_DEVICE;
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  const unsigned long long ctx = current_context_id();
+  if (!ctx || cache[dev].ctx != ctx || !cache[dev].addr) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_sens_scratch) != cudaSuccess || !p) return MXS_ERR_CUDA;
-    addr[dev] = p;
+    cache[dev] = Entry{current_context_id(), p};
   }
-  *ptr = addr[dev];
+  *ptr = cache[dev].addr;
   return MXS_OK;
 }
 
@@ -528,6 +535,12 @@ static mxs_status sens_scratch(void **ptr) {
 extern "C" mxs_status mxs_sensitivity_noalloc(const void *X, mxs_dtype xt, int64_t T, int64_t K, int64_t ldx,
                                               const void *W, mxs_dtype wt, int64_t N, int64_t ldw,
                                               double *H, double *E, double *s, void *stream) {
+  // the same argument checks as mxs_sensitivity, in the same order, before
+  // anything touches the device
+  if (!X || !W || !H || !s || T < 1 || N < 1 || K < 1) return MXS_ERR_ARG;
+  if (!dtype_ok(xt) || !dtype_ok(wt)) return MXS_ERR_DTYPE;
+  if (ldx < K || ldw < K) return MXS_ERR_SHAPE;
+  if (chunks(T) + chunks(N) > 65535) return MXS_ERR_SHAPE;
   size_t need = 0;
   mxs_status st = mxs_sensitivity_workspace_bytes(T, N, K, &need);
   if (st != MXS_OK) return st;

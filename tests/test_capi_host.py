@@ -1,11 +1,19 @@
 """Host-only checks of the C ABI: the library loads, exports every entry point
 declared in include/mxs.h, and rejects bad arguments before any launch.
-No call here touches a GPU."""
+No call here touches a GPU.  The argument checks pass made-up device
+addresses, which the library must reject on the host; they run only where no
+CUDA device exists, so that a check that stopped rejecting could never reach
+a launch on a real GPU (tests/test_gpu_argchecks.py repeats the checks that
+can be made with real buffers)."""
 import ctypes
 import os
 import re
 
 import pytest
+import torch
+
+fake_pointers = pytest.mark.skipif(torch.cuda.is_available(),
+                                   reason="passes made-up device addresses: CPU hosts only")
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "mxs.h")
@@ -83,6 +91,7 @@ def _fake_tensor(capi, rows, lay, base=1 << 20):
     return t
 
 
+@fake_pointers
 def test_gemm_argument_checks(capi):
     lay = capi.mxs_layout_make(256, (32, 64, 160))
     A = _fake_tensor(capi, 100, lay)
@@ -106,6 +115,7 @@ def test_gemm_argument_checks(capi):
     assert capi._lib.mxs_gemm(ctypes.byref(A), ctypes.byref(W), 1 << 24, 299, 1 << 26, 1 << 30, None) == 2
 
 
+@fake_pointers
 def test_quantize_argument_checks(capi):
     lay = capi.mxs_layout_make(64, (0, 0, 64))
     t = _fake_tensor(capi, 8, lay)
@@ -117,6 +127,7 @@ def test_quantize_argument_checks(capi):
     assert capi._lib.mxs_quantize_weight(1 << 20, 0, 8, 32, ctypes.byref(t), None) == 2
 
 
+@fake_pointers
 def test_sensitivity_argument_checks(capi):
     f = capi._lib.mxs_sensitivity
     X, W, H, E, S = 1 << 20, 1 << 24, 1 << 26, 1 << 27, 1 << 28
@@ -140,6 +151,7 @@ def test_sensitivity_argument_checks(capi):
     assert f(X, 1, 128, 512, 512, W, 1, 256, 512, H, E, S, ws, big - 8, None) == 9
 
 
+@fake_pointers
 def test_gemm_empty_product_needs_no_device(capi):
     lay = capi.mxs_layout_make(256, (32, 64, 160))
     A0 = _fake_tensor(capi, 0, lay)
@@ -157,6 +169,7 @@ def _alloc_call(capi, K, N, budget, ws=1 << 30, ws_bytes=1 << 40):
     return capi._lib.mxs_allocate(n, Ks, Ns, s, None, ctypes.byref(budget), perm, counts, ws, ws_bytes, None)
 
 
+@fake_pointers
 def test_allocate_argument_and_budget_checks(capi):
     # budget mode: 4.0 bits on average cannot carry the fixed 32-column 8-bit
     # block -> MXS_ERR_BUDGET, decided on the host before any launch
@@ -175,15 +188,13 @@ def test_allocate_argument_and_budget_checks(capi):
     assert _alloc_call(capi, [4096], [4096], ok, ws_bytes=16) == 9
 
 
+@fake_pointers
 def test_host_checks_survive_random_arguments(capi):
     """Random shapes, pitches and pointers return a status and never crash the
     process.  Some combinations pass every host check and would reach a
     launch on fake pointers, so this runs only where no CUDA device exists
     (the device check then fails first)."""
     import random
-    import torch
-    if torch.cuda.is_available():
-        pytest.skip("would launch kernels on fake pointers where a device exists")
     rng = random.Random(1234)
     valid = set(range(10))
     for _ in range(400):
@@ -209,3 +220,24 @@ def test_host_checks_survive_random_arguments(capi):
             assert capi._lib.mxs_quantize_act(rng.choice([None, 1 << 20, (1 << 20) + 2]), dt, rows, ld,
                                               ctypes.byref(t), None) in valid
             assert capi._lib.mxs_quantize_weight(1 << 20, dt, rows, ld, ctypes.byref(t), None) in valid
+
+
+@fake_pointers
+def test_noalloc_argument_checks(capi):
+    """mxs_sensitivity_noalloc returns the codes of mxs_sensitivity and rejects
+    shapes beyond its fixed scratch, all before touching the device."""
+    f = capi._lib.mxs_sensitivity_noalloc
+    X, W, H, E, S = 1 << 20, 1 << 24, 1 << 26, 1 << 27, 1 << 28
+    assert f(None, 1, 128, 512, 512, W, 1, 256, 512, H, E, S, None) == 1
+    assert f(X, 1, 128, 512, 512, W, 1, 256, 512, None, E, S, None) == 1
+    assert f(X, 9, 128, 512, 512, W, 1, 256, 512, H, E, S, None) == 4
+    assert f(X, 1, 128, 512, 511, W, 1, 256, 512, H, E, S, None) == 2
+    # (ceil(T/64) + ceil(N/64)) * K * 8 bytes > 16 MiB -> MXS_ERR_WORKSPACE
+    T, N, K = 64, 64 * 1024, 4096
+    assert capi.mxs_sensitivity_workspace_bytes(T, N, K) > capi.NOALLOC_SCRATCH_BYTES
+    launches = capi.mxs_launch_count()
+    assert f(X, 1, T, K, K, W, 1, N, K, H, E, S, None) == 9
+    # the Llama-2-70B MLP shapes exceed it too; the Llama-3-8B down projection fits
+    assert capi.mxs_sensitivity_workspace_bytes(2048, 28672, 8192) > capi.NOALLOC_SCRATCH_BYTES
+    assert capi.mxs_sensitivity_workspace_bytes(2048, 4096, 14336) <= capi.NOALLOC_SCRATCH_BYTES
+    assert capi.mxs_launch_count() == launches

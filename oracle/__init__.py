@@ -78,6 +78,8 @@ def _declare(L):
     L.orc_dequantize_rows.restype = None
     L.orc_gemm.argtypes = [_I64, _I64, _P, _P, _P, _P, _P, _P, _I64, _P, _I64, _P]
     L.orc_gemm.restype = None
+    L.orc_attn_decode.argtypes = [_P, _I64, _I64, _P, _P, _P, _P, _I64, _I64, ctypes.c_double, _P]
+    L.orc_attn_decode.restype = None
 
 
 def _ptr(a: np.ndarray):
@@ -245,3 +247,20 @@ def gemm(a_codes, a_scales, w_codes, w_scales, counts, rows=None, cols=None):
     lib().orc_gemm(M, N, _ptr(counts), *[ctypes.cast(p, ctypes.c_void_p) for p in ptrs],
                    _ptr(rows), rows.size, _ptr(cols), cols.size, _ptr(Y))
     return Y
+
+
+# ------------------------------------------------- decode attention (KV4)
+def attn_decode(q, k_codes, k_scales, v_codes, v_scales, T: int, n_kvh: int, sm_scale: float) -> np.ndarray:
+    """fp64 output (n_qh x d) of one decode step of grouped-query attention
+    over MXINT4 K/V caches given as compact codes (T*n_kvh x d/2 bytes) and
+    scales (T*n_kvh x d/32 bytes), rows token-major."""
+    q = _f64(q)
+    n_qh, d = q.shape
+    assert d % BLOCK == 0 and n_qh % n_kvh == 0
+    arrs = [np.ascontiguousarray(np.asarray(a, dtype=np.uint8)) for a in (k_codes, k_scales, v_codes, v_scales)]
+    for a, w in zip(arrs, (d // 2, d // BLOCK, d // 2, d // BLOCK)):
+        assert a.shape == (T * n_kvh, w), (a.shape, T, n_kvh, w)
+    out = np.zeros((n_qh, d))
+    lib().orc_attn_decode(_ptr(q), n_qh, d, *[_ptr(a) for a in arrs], int(T), int(n_kvh), float(sm_scale),
+                          _ptr(out))
+    return out

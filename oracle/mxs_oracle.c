@@ -468,3 +468,69 @@ void orc_gemm(int64_t M, int64_t N, const int64_t *counts,
     free(a);
     free(w);
 }
+
+/* ------------------------------------------------------------------------ */
+/* Decode-step attention over the 4-bit MXINT K/V cache                     */
+/* ------------------------------------------------------------------------ */
+
+/* One decoding step of grouped-query attention whose key and value caches
+ * are kept as MXINT4: the uniform 4-bit layout {0, 0, d}, blocks of 32 along
+ * the head dimension, one E8M0 byte per block [TS §4: the W4A4KV4 setting
+ * quantises the K/V cache to 4 bits; RV Validation: A4W4KV4 against
+ * A4W4KV16].  The pages do not spell out the attention arithmetic; it is the
+ * textbook scaled dot-product attention of one query token, read on the
+ * decoded cache:
+ *   query head h uses kv head g = h / (n_qh / n_kvh);
+ *   cache row t * n_kvh + g holds token t of kv head g (a [T][n_kvh][d]
+ *   cache flattened token-major);
+ *   s_t = sm_scale * sum_d q[h][d] * deq(K)[t n_kvh + g][d]
+ *   p_t = exp(s_t - max_u s_u) / sum_u exp(s_u - max_u s_u)
+ *   out[h][d] = sum_t p_t * deq(V)[t n_kvh + g][d]
+ * fp64 throughout; every sum runs in index order.  q is n_qh x d (row-major),
+ * the caches are compact (rows x d/2 code bytes, rows x d/32 scale bytes),
+ * out is n_qh x d. */
+void orc_attn_decode(const double *q, int64_t n_qh, int64_t d,
+                     const uint8_t *k_codes, const uint8_t *k_scales,
+                     const uint8_t *v_codes, const uint8_t *v_scales,
+                     int64_t T, int64_t n_kvh, double sm_scale, double *out)
+{
+    const int64_t counts[3] = {0, 0, d};
+    const int64_t rows = T * n_kvh;
+    const int64_t rep = n_qh / n_kvh;
+    double *kd = (double *)malloc(sizeof(double) * (size_t)(rows * d + 1));
+    double *vd = (double *)malloc(sizeof(double) * (size_t)(rows * d + 1));
+    double *s = (double *)malloc(sizeof(double) * (size_t)(T + 1));
+    const uint8_t *c[3], *sc[3];
+    c[0] = c[1] = sc[0] = sc[1] = NULL;
+    c[2] = k_codes;
+    sc[2] = k_scales;
+    orc_dequantize_rows(rows, counts, c, sc, kd);
+    c[2] = v_codes;
+    sc[2] = v_scales;
+    orc_dequantize_rows(rows, counts, c, sc, vd);
+    for (int64_t h = 0; h < n_qh; ++h) {
+        const int64_t g = h / rep;
+        double smax = -INFINITY;
+        for (int64_t t = 0; t < T; ++t) {
+            const double *k = kd + (t * n_kvh + g) * d;
+            double dot = 0.0;
+            for (int64_t i = 0; i < d; ++i) dot = dot + q[h * d + i] * k[i];
+            s[t] = sm_scale * dot;
+            if (s[t] > smax) smax = s[t];
+        }
+        double denom = 0.0;
+        for (int64_t t = 0; t < T; ++t) {
+            s[t] = exp(s[t] - smax);
+            denom = denom + s[t];
+        }
+        for (int64_t i = 0; i < d; ++i) out[h * d + i] = 0.0;
+        for (int64_t t = 0; t < T; ++t) {
+            const double p = s[t] / denom;
+            const double *v = vd + (t * n_kvh + g) * d;
+            for (int64_t i = 0; i < d; ++i) out[h * d + i] = out[h * d + i] + p * v[i];
+        }
+    }
+    free(kd);
+    free(vd);
+    free(s);
+}

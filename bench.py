@@ -1,21 +1,29 @@
 #!/usr/bin/env python
 """Benchmark of the MXSens mixed-width MXINT hot path on B200.
 
-One STEP is one pass of the whole path over one synthetic Llama-3-8B-shaped
-attention projection (W 4096x4096 bf16 with 3% Student-t(3) columns,
-calibration X 2048x4096 bf16 with 8 outlier channels x50, average budget 4.5
-bits) plus the K/V cache of the stack workload (8192 tokens x 8 heads x 128,
-K and V):
-  sensitivity(X, W) -> allocate (budget 4.5) -> quantize W ->
-  for M in (2048, 16, 1): quantize A_M -> gemm(A_M, W)  ->  quantize K, V.
-`value` = GEMM FLOPs of the step (2 M N K_real summed over the three M) per
-second of whole-step time, all ranks; the per-kernel numbers and the roofline
-of the dominant kernel are reported beside it.
+One STEP is one pass of the whole path over one batch of synthetic
+Llama-3-8B-shaped layers (every call through the C ABI):
+  attention projection  W 4096x4096 (3% Student-t(3) columns), calibration
+                        X 2048x4096 (8 outlier channels x50), GEMM M in
+                        {2048, 16, 1};
+  MLP gate/up           W 14336x4096, X as above, GEMM M in {8192, 16, 1};
+  MLP down              W 4096x14336, X and A Laplace(0, 0.1) with 0.5%
+                        spikes x100, GEMM M in {8192, 16, 1};
+each: sensitivity(X, W) -> allocate (budget 4.5 bits) -> quantize W ->
+for each M: quantize A_M -> gemm(A_M, W); then the K/V cache of the stack
+workload (8192 tokens x 8 kv heads x 128, K and V) is quantised to MXINT4
+and one decode step of attention (32 query heads) reads it.
+`value` = the step's GEMM FLOPs (2 M N K summed over all GEMMs) per second of
+whole-step time, summed over ranks; the per-call numbers, the roofline of the
+dominant kernel, the mixed-width overhead against uniform MXINT4 and the
+average-bit budget sweep are reported beside it.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
-`--impl reference` times the CPU oracle (plain single-threaded C, fp64) on the
-host cores instead, on a bounded row sample of the same workload per step.
+With --gpus N > 1 and no torchrun environment, the script relaunches itself
+under torch.distributed.run with N processes (one per GPU).  `--impl
+reference` times the CPU oracle (plain single-threaded C, fp64) on the host
+cores instead, on a bounded row sample of the same workload per step.
 """
 from __future__ import annotations
 
@@ -23,8 +31,11 @@ import argparse
 import hashlib
 import json
 import os
+import platform
 import re
+import socket
 import statistics
+import subprocess
 import sys
 import threading
 import time
@@ -32,15 +43,21 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-M_LIST = (2048, 16, 1)
-N_OUT, K_IN, T_CAL = 4096, 4096, 2048
-KV_SHAPE = (8192, 8, 128)
+T_CAL = 2048
 BUDGET = (9, 2)
 SEED = 2000
-CALL_REPS, CALL_TRIALS = 10, 5   # per-call timing: calls per graph, replays per graph
+KV_SHAPE = (8192, 8, 128)          # tokens, kv heads, head dim
+N_QH = 32                          # query heads of the decode step
+CALL_REPS, CALL_TRIALS = 10, 5     # per-call timing: calls per graph, replays per graph
 METRIC = "mxs_gemm TFLOP/s (% of roofline); MXINT quantize GB/s (% of HBM peak)"
-WORKLOAD = ("llama3-8b attention projection: W 4096x4096 bf16 (3% t3 columns), calib X 2048x4096 bf16 "
-            "(8 channels x50), budget 4.5 bits, GEMM M in {2048,16,1}; + K/V cache 8192x8x128 bf16 x2")
+# (name, N, K, calibration/activation kind, M values)
+LAYERS = (("attn", 4096, 4096, "gauss", (2048, 16, 1)),
+          ("mlp_up", 14336, 4096, "gauss", (8192, 16, 1)),
+          ("mlp_down", 4096, 14336, "laplace", (8192, 16, 1)))
+WORKLOAD = ("llama3-8b layer: attention projection W 4096x4096 (M 2048/16/1), MLP gate/up W 14336x4096 and "
+            "down W 4096x14336 (M 8192/16/1), bf16, calib X 2048 rows, budget 4.5 bits each; K/V cache "
+            "8192x8x128 bf16 x2 to MXINT4 + one decode-attention step (32 query heads)")
+SWEEP_BUDGETS = ((7, 2), (129, 32), (17, 4), (9, 2), (5, 1), (23, 4))     # 3.5 ... 5.75 average bits
 
 
 def peaks():
@@ -71,6 +88,25 @@ def gemm_roofline_s(M, N, counts, pk):
     t_c = 2.0 * M * N * n4 / (pk["fp8_tflops"] * 1e12) + 2.0 * M * N * (n8 + n6) / (pk["bf16_tflops"] * 1e12)
     byts = layout_bytes(M, counts, 0) + layout_bytes(N, counts, 0) + M * N * 2
     return max(t_c, byts / (pk["hbm_gbs"] * 1e9))
+
+
+def attn_bytes(T, n_kvh, n_qh, d=128):
+    """Algorithmic bytes of one decode-attention call: packed K and V (codes
+    and one scale byte per 32 values), the bf16 query and the fp32 output."""
+    cache = T * n_kvh * (d // 2 + d // 32)
+    return 2 * cache + n_qh * d * 2 + n_qh * d * 4
+
+
+def host_info():
+    model = platform.processor() or ""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"host_cores": os.cpu_count(), "cpu_model": model}
 
 
 # --------------------------------------------------------------------- clocks
@@ -124,78 +160,121 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ GPU arm
+def _layer_inputs(inputs, dev, seed, name, N, K, kind, Ms):
+    W = inputs.attn_weight(dev, seed, N, K)
+    if kind == "gauss":
+        X = inputs.gaussian_acts(dev, seed + 1, T_CAL, K)
+        A = {M: inputs.gaussian_acts(dev, seed + 2 + M, M, K) for M in Ms}
+    else:
+        X = inputs.laplace_acts(dev, seed + 1, T_CAL, K)
+        A = {M: inputs.laplace_acts(dev, seed + 2 + M, M, K) for M in Ms}
+    return W, X, A
+
+
+class Layer:
+    """One linear layer of the step: its inputs, quantised tensors and calls."""
+
+    def __init__(self, c, inputs, dev, seed, name, N, K, kind, Ms):
+        import torch
+        self.c, self.name, self.N, self.K, self.Ms = c, name, N, K, Ms
+        self.W, self.X, self.A = _layer_inputs(inputs, dev, seed, name, N, K, kind, Ms)
+        self.sens_ws = torch.empty(c.mxs_sensitivity_workspace_bytes(T_CAL, N, K) + 1024, dtype=torch.uint8, device=dev)
+        self.H = torch.empty(K, dtype=torch.float64, device=dev)
+        self.E, self.s = torch.empty_like(self.H), torch.empty_like(self.H)
+        self.perm = torch.empty(K, dtype=torch.int32, device=dev)
+        self.alloc_ws = torch.empty(1 << 20, dtype=torch.uint8, device=dev)
+        c.mxs_sensitivity(self.X, self.W, workspace=self.sens_ws, out=(self.H, self.E, self.s))
+        _, counts = c.mxs_allocate([self.s], [N], mode="budget", budget=BUDGET, perms=[self.perm],
+                                   workspace=self.alloc_ws)
+        self.counts = counts[0]
+        self.lay = c.mxs_layout_make(K, self.counts, self.perm)
+        self.Wq = c.mxtensor_empty(N, self.lay, dev)
+        self.Aq = {M: c.mxtensor_empty(M, self.lay, dev) for M in Ms}
+        self.Y = {M: torch.empty(M, N, dtype=torch.bfloat16, device=dev) for M in Ms}
+        c.mxs_quantize_weight(self.W, self.Wq)
+        for M in Ms:
+            c.mxs_quantize_act(self.A[M], self.Aq[M])
+        gws = max(c.mxs_gemm_workspace_bytes(self.Aq[M], self.Wq) for M in Ms)
+        self.gemm_ws = torch.empty(gws + 1024, dtype=torch.uint8, device=dev)
+
+    def work(self):
+        n = self.name
+        w = {f"{n}.mxs_sensitivity": ("GB/s", (T_CAL + self.N) * self.K * 2),
+             f"{n}.mxs_allocate": ("GB/s", self.K * 8 + self.K * 4),
+             f"{n}.mxs_quantize_weight": ("GB/s", layout_bytes(self.N, self.counts, 2))}
+        for M in self.Ms:
+            w[f"{n}.mxs_quantize_act_M{M}"] = ("GB/s", layout_bytes(M, self.counts, 2))
+            w[f"{n}.mxs_gemm_M{M}"] = ("TFLOP/s", 2 * M * self.N * self.K)
+        return w
+
+    def calls(self):
+        c, n = self.c, self.name
+
+        def alloc():
+            _, counts = c.mxs_allocate([self.s], [self.N], mode="budget", budget=BUDGET, perms=[self.perm],
+                                       workspace=self.alloc_ws)
+            assert counts[0] == self.counts
+        out = [(f"{n}.mxs_sensitivity", lambda: c.mxs_sensitivity(self.X, self.W, workspace=self.sens_ws,
+                                                                    out=(self.H, self.E, self.s))),
+               (f"{n}.mxs_allocate", alloc),
+               (f"{n}.mxs_quantize_weight", lambda: c.mxs_quantize_weight(self.W, self.Wq))]
+        for M in self.Ms:
+            out.append((f"{n}.mxs_quantize_act_M{M}", lambda M=M: c.mxs_quantize_act(self.A[M], self.Aq[M])))
+            out.append((f"{n}.mxs_gemm_M{M}", lambda M=M: c.mxs_gemm(self.Aq[M], self.Wq, Y=self.Y[M],
+                                                                     workspace=self.gemm_ws)))
+        return out
+
+
 class Path:
     """Device buffers and the step of the hot path (all kernels through the C ABI)."""
 
     def __init__(self, dev, seed):
+        import math
         import torch
         from mx_microscaling_mixed_b200 import capi, inputs
         self.torch, self.c = torch, capi
-        self.W = inputs.attn_weight(dev, seed, N_OUT, K_IN)
-        self.X = inputs.gaussian_acts(dev, seed + 1, T_CAL, K_IN)
-        self.A = {M: inputs.gaussian_acts(dev, seed + 2 + M, M, K_IN) for M in M_LIST}
-        self.KV = [inputs.kv_cache(dev, seed + 10 + i, *KV_SHAPE).reshape(-1, KV_SHAPE[2]) for i in range(2)]
         c = capi
-        self.sens_ws = torch.empty(c.mxs_sensitivity_workspace_bytes(T_CAL, N_OUT, K_IN) + 1024,
-                                   dtype=torch.uint8, device=dev)
-        self.H = torch.empty(K_IN, dtype=torch.float64, device=dev)
-        self.E, self.s = torch.empty_like(self.H), torch.empty_like(self.H)
-        self.perm = torch.empty(K_IN, dtype=torch.int32, device=dev)
-        self.alloc_ws = torch.empty(1 << 20, dtype=torch.uint8, device=dev)
-        c.mxs_sensitivity(self.X, self.W, workspace=self.sens_ws, out=(self.H, self.E, self.s))
-        _, counts = c.mxs_allocate([self.s], [N_OUT], mode="budget", budget=BUDGET, perms=[self.perm],
-                                   workspace=self.alloc_ws)
-        self.counts = counts[0]
-        self.lay = c.mxs_layout_make(K_IN, self.counts, self.perm)
-        self.Wq = c.mxtensor_empty(N_OUT, self.lay, dev)
-        self.Aq = {M: c.mxtensor_empty(M, self.lay, dev) for M in M_LIST}
-        self.kv_lay = c.mxs_layout_make(KV_SHAPE[2], (0, 0, KV_SHAPE[2]))
+        self.layers = [Layer(c, inputs, dev, seed + 100 * i, *spec) for i, spec in enumerate(LAYERS)]
+        T, H, D = KV_SHAPE
+        self.KV = [inputs.kv_cache(dev, seed + 10 + i, T, H, D).reshape(-1, D) for i in range(2)]
+        self.q = inputs.random_matrix(N_QH, D, device=dev, seed=seed + 20, dtype=torch.bfloat16, outlier_frac=0.0)
+        self.kv_lay = c.mxs_layout_make(D, (0, 0, D))
         self.KVq = [c.mxtensor_empty(kv.shape[0], self.kv_lay, dev) for kv in self.KV]
-        self.Y = {M: torch.empty(M, N_OUT, dtype=torch.bfloat16, device=dev) for M in M_LIST}
-        c.mxs_quantize_weight(self.W, self.Wq)
-        for M in M_LIST:
-            c.mxs_quantize_act(self.A[M], self.Aq[M])
-        gws = max(c.mxs_gemm_workspace_bytes(self.Aq[M], self.Wq) for M in M_LIST)
-        self.gemm_ws = torch.empty(gws + 1024, dtype=torch.uint8, device=dev)
+        self.attn_out = torch.empty(N_QH, D, dtype=torch.float32, device=dev)
+        self.attn_ws = torch.empty(c.mxs_attn_decode_workspace_bytes(T, N_QH, H, D) + 1024, dtype=torch.uint8,
+                                   device=dev)
+        self.sm_scale = 1.0 / math.sqrt(D)
+        for i in range(2):
+            c.mxs_quantize_act(self.KV[i], self.KVq[i])
         self.flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
         self.flush_small = self.flush[: 256 << 20]          # per-call timing: twice the L2
         # algorithmic bytes / FLOPs per launch of each timed call
-        n8, n6, n4 = self.counts
-        self.work = {
-            "mxs_sensitivity": ("GB/s", (T_CAL + N_OUT) * K_IN * 2),
-            "mxs_allocate": ("GB/s", K_IN * 8 + K_IN * 4),
-            "mxs_quantize_weight": ("GB/s", layout_bytes(N_OUT, self.counts, 2)),
-            "mxs_quantize_kv0": ("GB/s", layout_bytes(KV_SHAPE[0] * KV_SHAPE[1], (0, 0, KV_SHAPE[2]), 2)),
-            "mxs_quantize_kv1": ("GB/s", layout_bytes(KV_SHAPE[0] * KV_SHAPE[1], (0, 0, KV_SHAPE[2]), 2)),
-        }
-        for M in M_LIST:
-            self.work[f"mxs_quantize_act_M{M}"] = ("GB/s", layout_bytes(M, self.counts, 2))
-            self.work[f"mxs_gemm_M{M}"] = ("TFLOP/s", 2 * M * N_OUT * K_IN)
-        self.gemm_flops = sum(2 * M * N_OUT * K_IN for M in M_LIST)
+        self.work = {}
+        for L in self.layers:
+            self.work.update(L.work())
+        for i in range(2):
+            self.work[f"kv.mxs_quantize_act_{'KV'[i]}"] = ("GB/s", layout_bytes(T * H, (0, 0, D), 2))
+        self.work["kv.mxs_attn_decode"] = ("GB/s", attn_bytes(T, H, N_QH, D))
+        self.gemm_flops = sum(2 * M * L.N * L.K for L in self.layers for M in L.Ms)
 
     def calls(self):
         """The step as (name, call) pairs in order; each call is one C-ABI entry point."""
         c = self.c
-
-        def alloc():
-            _, counts = c.mxs_allocate([self.s], [N_OUT], mode="budget", budget=BUDGET, perms=[self.perm],
-                                       workspace=self.alloc_ws)
-            assert counts[0] == self.counts
-        out = [("mxs_sensitivity", lambda: c.mxs_sensitivity(self.X, self.W, workspace=self.sens_ws,
-                                                               out=(self.H, self.E, self.s))),
-               ("mxs_allocate", alloc),
-               ("mxs_quantize_weight", lambda: c.mxs_quantize_weight(self.W, self.Wq))]
-        for M in M_LIST:
-            out.append((f"mxs_quantize_act_M{M}", lambda M=M: c.mxs_quantize_act(self.A[M], self.Aq[M])))
-            out.append((f"mxs_gemm_M{M}", lambda M=M: c.mxs_gemm(self.Aq[M], self.Wq, Y=self.Y[M],
-                                                                 workspace=self.gemm_ws)))
+        out = []
+        for L in self.layers:
+            out += L.calls()
         for i in range(2):
-            out.append((f"mxs_quantize_kv{i}", lambda i=i: c.mxs_quantize_act(self.KV[i], self.KVq[i])))
+            out.append((f"kv.mxs_quantize_act_{'KV'[i]}", lambda i=i: c.mxs_quantize_act(self.KV[i], self.KVq[i])))
+        T, H, _ = KV_SHAPE
+        out.append(("kv.mxs_attn_decode", lambda: c.mxs_attn_decode(self.q, self.KVq[0], self.KVq[1], T, H,
+                                                                     self.sm_scale, out=self.attn_out,
+                                                                     workspace=self.attn_ws)))
         return out
 
-    def step(self):
-        for _, fn in self.calls():
-            fn()
+    def gemm_spec(self, name):
+        layer, call = name.split(".", 1)
+        L = next(x for x in self.layers if x.name == layer)
+        return int(call.split("M")[-1]), L.N, L.counts
 
 
 def max_over_ranks(t: float, world: int, device) -> float:
@@ -216,8 +295,10 @@ def job_tflops(flops_per_rank_step: float, steps: int, world: int, job_s: float)
     return world * flops_per_rank_step * steps / job_s / 1e12
 
 
-def traffic_from_profile(pk_name: str):
-    """dram bytes per launch recorded in profiles/, if the kernel source is unchanged since."""
+def traffic_from_profile(pk_name: str, per_units: float = 1.0):
+    """dram bytes per launch recorded in profiles/, if the GEMM source is
+    unchanged since the capture; scaled by `per_units` (units of the bench
+    launch per unit of the captured one) when the capture was a smaller case."""
     prof = os.path.join(ROOT, "profiles", pk_name)
     try:
         text = open(prof).read()
@@ -230,7 +311,17 @@ def traffic_from_profile(pk_name: str):
     src = os.path.join(ROOT, "mx_microscaling_mixed_b200", "csrc", "mxs_gemm.cu")
     if hashlib.sha256(open(src, "rb").read()).hexdigest() != h.group(1):
         return None
-    return float(m.group(1))
+    return float(m.group(1)) * per_units
+
+
+def _graph_timer(torch, cap):
+    def timed(g):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        g.replay()
+        e.record()
+        return s, e
+    return timed
 
 
 def run_gpu(args, rank, world, local_rank):
@@ -245,7 +336,8 @@ def run_gpu(args, rank, world, local_rank):
     pk = peaks()
     for _ in range(args.warmup):
         path.flush.zero_()
-        path.step()
+        for _, fn in path.calls():
+            fn()
     c.mxs_sync()
 
     def barrier():
@@ -286,13 +378,7 @@ def run_gpu(args, rank, world, local_rank):
         for _, g in graphs:
             g.replay()
     c.mxs_sync()
-
-    def timed(g):
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s.record()
-        g.replay()
-        e.record()
-        return s, e
+    timed = _graph_timer(torch, cap)
 
     rec = {}
     step_ev = []
@@ -317,27 +403,34 @@ def run_gpu(args, rank, world, local_rank):
     best = {name: min(s.elapsed_time(e) for s, e in evs) * 1e-3 for name, evs in rec.items()}
     per_call = {name: max(best[name] - best[""], 0.0) / CALL_REPS for name, _ in calls}
     call_sum = sum(per_call.values())
+    del graphs, g_flush
 
     kernels = {}
     for name, per in per_call.items():
         unit, work = path.work[name]
-        ach = work / per / (1e12 if unit == "TFLOP/s" else 1e9)
+        ach = work / per / (1e12 if unit == "TFLOP/s" else 1e9) if per > 0 else None
         kd = {"us": per * 1e6, "achieved": ach, "unit": unit, "share": per / call_sum}
         if unit == "GB/s":
-            kd["frac_hbm"] = ach / pk["hbm_gbs"]
-            kd["frac_nominal_8tbs"] = ach / 8000.0
+            kd["frac_hbm"] = ach / pk["hbm_gbs"] if ach else None
+            kd["frac_nominal_8tbs"] = ach / 8000.0 if ach else None
         else:
-            M = int(name.split("M")[-1])
-            rt = gemm_roofline_s(M, N_OUT, path.counts, pk)
+            M, N, counts = path.gemm_spec(name)
+            rt = gemm_roofline_s(M, N, counts, pk)
             kd["roofline_us"] = rt * 1e6
-            kd["frac"] = rt / per
+            kd["frac"] = rt / per if per > 0 else None
+            kd["bound"] = "hbm" if rt == (layout_bytes(M, counts, 0) + layout_bytes(N, counts, 0) + M * N * 2) / (
+                pk["hbm_gbs"] * 1e9) else "tensor"
         kernels[name] = kd
-    # the dominant kernel: the prefill GEMM
-    g = kernels["mxs_gemm_M2048"]
+    # the dominant kernel: the GEMM call with the largest share of the step
+    dom = max((n for n in kernels if ".mxs_gemm_M" in n), key=lambda n: kernels[n]["us"])
+    g = kernels[dom]
+    M, N, counts = path.gemm_spec(dom)
+    K = sum(counts)
     rt = g["roofline_us"] * 1e-6
-    roof = {"kernel": "mxs_gemm M=2048 (one call: gemm_stage_kernel + gemm_tc2_kernel)", "bound": "tensor",
-            "achieved": g["achieved"], "peak": 2 * 2048 * N_OUT * K_IN / rt / 1e12, "unit": "TFLOP/s",
-            "frac": g["frac"], "traffic": traffic_from_profile("gemm_attn_prefill_M2048.md"),
+    roof = {"kernel": f"{dom} (one call: gemm_stage_kernel + gemm_tc2_kernel), M={M} N={N} K={K}",
+            "bound": "tensor", "achieved": g["achieved"], "peak": 2 * M * N * K / rt / 1e12, "unit": "TFLOP/s",
+            "frac": g["frac"],
+            "traffic": traffic_from_profile("gemm_mlp_prefill_M8192.md") if dom.startswith("mlp_up") else None,
             "peak_basis": f"4-bit segment at 2x measured bf16 ({pk['fp8_tflops']:.0f} TFLOP/s, no measured fp8), "
                           f"6/8-bit at measured bf16 ({pk['bf16_tflops']:.0f}); of {pk['source']}"}
 
@@ -347,8 +440,9 @@ def run_gpu(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": total_s / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "mxint4/6/8 codes; e4m3+bf16 MMA, f32 acc",
         "data": "synthetic (seeded; shapes and outlier structure of the workload)",
-        "config": {"workload": WORKLOAD, "counts_n8_n6_n4": list(path.counts), "l2": "flushed between steps "
-                   "(512 MB write outside the step events)", "parallelism": f"replicas x{world} (no data-path collective)",
+        "config": {"workload": WORKLOAD, "counts_n8_n6_n4": {L.name: list(L.counts) for L in path.layers},
+                   "l2": "flushed between steps (512 MB write outside the step events)",
+                   "parallelism": f"replicas x{world} (no data-path collective)",
                    "timing": "step = one CUDA graph of all C-ABI calls, replayed per step between CUDA events; "
                              f"kernels{{}}: per call, (graph of {CALL_REPS} x [L2 flush, call]) - (graph of "
                              f"{CALL_REPS} flushes), best of {CALL_TRIALS} replays each, / {CALL_REPS}; cold L2 per call",
@@ -356,6 +450,9 @@ def run_gpu(args, rank, world, local_rank):
         "roofline": roof, "kernels": kernels, "e2e": e2e, "gpu_launches": launches,
         "clocks": clocks.summary(), "wall_s_timed_region": wall,
     }
+    if not args.no_extras:
+        line["mixed_overhead"] = run_mixed_overhead(c, dev, path, torch)
+        line["budget_sweep"] = run_budget_sweep(c, dev, path, torch, pk)
     return line
 
 
@@ -363,22 +460,33 @@ def run_e2e(path, args, dev, world):
     """Same metric through the C ABI with pinned host buffers: H2D of the
     step's inputs and D2H of its outputs inside the timed region.  The copies
     run on their own streams in the order the step consumes the inputs; each
-    call waits only for the inputs it reads, and each GEMM's output leaves as
-    soon as it is written, so transfers overlap the kernels."""
+    call waits only for the inputs it reads, and each output leaves as soon as
+    it is written, so transfers overlap the kernels."""
     import torch
-    host = {"X": path.X.cpu().pin_memory(), "W": path.W.cpu().pin_memory(),
-            **{f"A{M}": path.A[M].cpu().pin_memory() for M in M_LIST},
-            **{f"KV{i}": path.KV[i].cpu().pin_memory() for i in range(2)}}
-    dst = {"X": path.X, "W": path.W, **{f"A{M}": path.A[M] for M in M_LIST},
-           **{f"KV{i}": path.KV[i] for i in range(2)}}
-    outs = {M: torch.empty(path.Y[M].shape, dtype=torch.bfloat16).pin_memory() for M in M_LIST}
+    dst = {}
+    needs = {}
+    for L in path.layers:
+        dst[f"{L.name}.X"], dst[f"{L.name}.W"] = L.X, L.W
+        needs[f"{L.name}.mxs_sensitivity"] = (f"{L.name}.X", f"{L.name}.W")
+        needs[f"{L.name}.mxs_quantize_weight"] = (f"{L.name}.W",)
+        for M in L.Ms:
+            dst[f"{L.name}.A{M}"] = L.A[M]
+            needs[f"{L.name}.mxs_quantize_act_M{M}"] = (f"{L.name}.A{M}",)
+    for i in range(2):
+        dst[f"kv.{'KV'[i]}"] = path.KV[i]
+        needs[f"kv.mxs_quantize_act_{'KV'[i]}"] = (f"kv.{'KV'[i]}",)
+    dst["kv.q"] = path.q
+    needs["kv.mxs_attn_decode"] = ("kv.q",)
+    host = {k: v.cpu().pin_memory() for k, v in dst.items()}
+    outs = {}
+    for L in path.layers:
+        for M in L.Ms:
+            outs[f"{L.name}.mxs_gemm_M{M}"] = (L.Y[M], torch.empty(L.Y[M].shape, dtype=L.Y[M].dtype).pin_memory())
+    outs["kv.mxs_attn_decode"] = (path.attn_out, torch.empty(path.attn_out.shape, dtype=torch.float32).pin_memory())
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = sum(t.numel() * t.element_size() for t in outs.values())
-    # inputs each call reads (the rest read only device results of earlier calls)
-    needs = {"mxs_sensitivity": ("X", "W"), "mxs_quantize_weight": ("W",),
-             **{f"mxs_quantize_act_M{M}": (f"A{M}",) for M in M_LIST},
-             **{f"mxs_quantize_kv{i}": (f"KV{i}",) for i in range(2)}}
+    d2h = sum(h.numel() * h.element_size() for _, h in outs.values())
     calls = path.calls()
+    order = list(dst)                                   # the order the step consumes them
     main = torch.cuda.current_stream()
     up, down = torch.cuda.Stream(), torch.cuda.Stream()
     steps = max(3, min(args.steps, 10))
@@ -389,7 +497,7 @@ def run_e2e(path, args, dev, world):
         up.wait_stream(main)
         landed = {}
         with torch.cuda.stream(up):
-            for k in ("X", "W", *[f"A{M}" for M in M_LIST], "KV0", "KV1"):
+            for k in order:
                 dst[k].copy_(host[k], non_blocking=True)
                 landed[k] = torch.cuda.Event()
                 landed[k].record(up)
@@ -397,11 +505,10 @@ def run_e2e(path, args, dev, world):
             for k in needs.get(name, ()):
                 main.wait_event(landed[k])
             fn()
-            if name.startswith("mxs_gemm_M"):
-                M = int(name[len("mxs_gemm_M"):])
+            if name in outs:
                 down.wait_stream(main)
                 with torch.cuda.stream(down):
-                    outs[M].copy_(path.Y[M], non_blocking=True)
+                    outs[name][1].copy_(outs[name][0], non_blocking=True)
         main.wait_stream(down)
         main.wait_stream(up)
         e.record(main)
@@ -413,55 +520,151 @@ def run_e2e(path, args, dev, world):
             "d2h_bytes_per_step": d2h, "ms_per_step": t * 1e3}
 
 
+def _time_call(torch, call, flush, reps):
+    """Median of `reps` CUDA-graph replays of one call, each after an L2 flush."""
+    for _ in range(3):
+        call()
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    with torch.cuda.graph(g, stream=cap):
+        call()
+    ev = []
+    for _ in range(reps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        ev.append((e0, e1))
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
+
+
+def run_mixed_overhead(c, dev, path, torch, reps=30):
+    """What the wider blocks cost: mxs_gemm on each layer's weight under
+    uniform MXINT4, the 32 fixed 8-bit columns alone (4 + 4*32/K bits) and the
+    4.5-bit budget, at every M of the layer ([TS §4] estimates ~3% latency at
+    ~4.03 bits)."""
+    out = {"unit": "us", "reps": reps, "timing": "median of CUDA-graph replays, L2 flushed before each",
+           "layers": {}}
+    for L in path.layers:
+        layouts = {"uniform4": ((0, 0, L.K), torch.arange(L.K, dtype=torch.int32, device=dev)),
+                   "fixed8_only": None, "b4.5": (L.counts, L.perm)}
+        perms, counts = c.mxs_allocate([L.s], [L.N], mode="budget", budget=(4 * L.K + 128, L.K))
+        layouts["fixed8_only"] = (counts[0], perms[0])
+        row = {"counts": {k: list(v[0]) for k, v in layouts.items()}, "us": {}, "overhead": {}}
+        for M in L.Ms:
+            for lname, (cnt, perm) in layouts.items():
+                lay = c.mxs_layout_make(L.K, cnt, perm)
+                Wq, Aq = c.mxtensor_empty(L.N, lay, dev), c.mxtensor_empty(M, lay, dev)
+                c.mxs_quantize_weight(L.W, Wq)
+                c.mxs_quantize_act(L.A[M], Aq)
+                ws = torch.empty(c.mxs_gemm_workspace_bytes(Aq, Wq) + 1024, dtype=torch.uint8, device=dev)
+                Y = torch.empty(M, L.N, dtype=torch.bfloat16, device=dev)
+                row["us"][f"M{M}/{lname}"] = _time_call(torch, lambda: c.mxs_gemm(Aq, Wq, Y=Y, workspace=ws),
+                                                        path.flush, reps)
+                del Wq, Aq, ws, Y
+            base = row["us"][f"M{M}/uniform4"]
+            for lname in ("fixed8_only", "b4.5"):
+                row["overhead"][f"M{M}/{lname}"] = row["us"][f"M{M}/{lname}"] / base - 1.0
+        out["layers"][L.name] = row
+    c.mxs_sync()
+    return out
+
+
+def run_budget_sweep(c, dev, path, torch, pk, reps=20):
+    """Average-bit budget sweep ([TS §4] ablation, ~3.28 to 5.75 bits): the
+    allocation's counts and the prefill mxs_gemm time of each layer at each
+    budget; budgets below what the fixed 8-bit block costs are infeasible."""
+    out = {"unit": "us", "reps": reps, "budgets": [f"{n}/{d}" for n, d in SWEEP_BUDGETS], "layers": {}}
+    for L in path.layers:
+        M = L.Ms[0]
+        rows = []
+        for num, den in SWEEP_BUDGETS:
+            r = {"budget_bits": num / den}
+            try:
+                perms, counts = c.mxs_allocate([L.s], [L.N], mode="budget", budget=(num, den))
+            except c.MxsError as e:
+                r["status"] = c.mxs_status_str(e.status).split(":")[0]
+                rows.append(r)
+                continue
+            cnt = counts[0]
+            lay = c.mxs_layout_make(L.K, cnt, perms[0])
+            Wq, Aq = c.mxtensor_empty(L.N, lay, dev), c.mxtensor_empty(M, lay, dev)
+            c.mxs_quantize_weight(L.W, Wq)
+            c.mxs_quantize_act(L.A[M], Aq)
+            ws = torch.empty(c.mxs_gemm_workspace_bytes(Aq, Wq) + 1024, dtype=torch.uint8, device=dev)
+            Y = torch.empty(M, L.N, dtype=torch.bfloat16, device=dev)
+            us = _time_call(torch, lambda: c.mxs_gemm(Aq, Wq, Y=Y, workspace=ws), path.flush, reps)
+            n8, n6, n4 = cnt
+            r.update({"counts": list(cnt), "achieved_bits": (8 * n8 + 6 * n6 + 4 * n4) / L.K,
+                      f"gemm_M{M}_us": us, "tflops": 2 * M * L.N * L.K / us / 1e6,
+                      "roofline_frac": gemm_roofline_s(M, L.N, cnt, pk) / (us * 1e-6)})
+            rows.append(r)
+            del Wq, Aq, ws, Y
+        out["layers"][L.name] = {"M": M, "rows": rows}
+    c.mxs_sync()
+    return out
+
+
 # ----------------------------------------------------------- oracle (CPU) arm
 class OraclePath:
     """The CPU oracle on a row sample of the same workload.  Every piece of the
     step is linear in the rows it processes, so a sample of fraction f is timed
-    and scaled by 1/f (allocation, which sorts one vector, runs in full)."""
+    and scaled by 1/f (allocation, which sorts one vector, runs in full; the
+    attention step runs on a token prefix of the cache)."""
 
-    def __init__(self, seed):
+    def __init__(self, seed, frac_hint=1.0 / 16):
         import numpy as np
         import torch
         import oracle
         from mx_microscaling_mixed_b200 import inputs
         self.np, self.o = np, oracle
         f64 = lambda t: t.float().numpy().astype(np.float64)
-        self.W = f64(inputs.attn_weight("cpu", seed, N_OUT, K_IN))
-        self.X = f64(inputs.gaussian_acts("cpu", seed + 1, T_CAL, K_IN))
-        self.A = {M: f64(inputs.gaussian_acts("cpu", seed + 2 + M, M, K_IN)) for M in M_LIST}
-        self.KV = [f64(inputs.kv_cache("cpu", seed + 10 + i, *KV_SHAPE).reshape(-1, KV_SHAPE[2])) for i in range(2)]
-        self.gemm_flops = sum(2 * M * N_OUT * K_IN for M in M_LIST)
-        _, _, s = oracle.sensitivity(self.X[:256], self.W[:256])
-        self.perm, self.counts = None, None
+        self.layers = []
+        for i, (name, N, K, kind, Ms) in enumerate(LAYERS):
+            # the draws of the GPU arm, of which a sample of fraction <= 1/8 uses the leading rows
+            W, X, A = _layer_inputs(inputs, "cpu", seed + 100 * i, name, N, K, kind, Ms)
+            self.layers.append((name, N, K, Ms, f64(W[: N // 8]), f64(X[: T_CAL // 8]),
+                                {M: f64(A[M][: max(1, M // 8)]) for M in Ms}))
+        T, H, D = KV_SHAPE
+        self.KV = [f64(inputs.kv_cache("cpu", seed + 10 + i, T // 8, H, D).reshape(-1, D)) for i in range(2)]
+        self.q = f64(inputs.random_matrix(N_QH, D, device="cpu", seed=seed + 20, dtype=torch.bfloat16,
+                                          outlier_frac=0.0))
+        self.gemm_flops = sum(2 * M * N * K for _, N, K, Ms, *_ in self.layers for M in Ms)
 
     def step(self, frac):
-        o, np = self.o, self.np
+        o = self.o
         rows = lambda n: max(1, int(round(n * frac)))
         t = {}
-        tx, tw = rows(T_CAL), rows(N_OUT)
-        t0 = time.perf_counter()
-        _, _, s = o.sensitivity(self.X[:tx], self.W[:tw])
-        t["sensitivity"] = (time.perf_counter() - t0) * ((T_CAL + N_OUT) / (tx + tw))
-        t0 = time.perf_counter()
-        perms, counts = o.allocate([s], [N_OUT], mode="budget", budget=BUDGET)
-        t["allocate"] = time.perf_counter() - t0
-        perm, counts = perms[0], counts[0]
-        t0 = time.perf_counter()
-        wc, ws = o.quantize_rows(self.W[:tw], perm, counts)
-        t["quantize_weight"] = (time.perf_counter() - t0) * N_OUT / tw
-        for M in M_LIST:
-            m = rows(M)
+        for name, N, K, Ms, W, X, A in self.layers:
+            tx, tw = rows(T_CAL), rows(N)
             t0 = time.perf_counter()
-            ac, as_ = o.quantize_rows(self.A[M][:m], perm, counts)
-            t[f"quantize_act_M{M}"] = (time.perf_counter() - t0) * M / m
+            _, _, s = o.sensitivity(X[:tx], W[:tw])
+            t[f"{name}.sensitivity"] = (time.perf_counter() - t0) * ((T_CAL + N) / (tx + tw))
             t0 = time.perf_counter()
-            o.gemm(ac, as_, wc, ws, counts)                   # m x tw block of Y
-            t[f"gemm_M{M}"] = (time.perf_counter() - t0) * (M * N_OUT) / (m * tw)
-        n_kv = rows(KV_SHAPE[0] * KV_SHAPE[1])
+            perms, counts = o.allocate([s], [N], mode="budget", budget=BUDGET)
+            t[f"{name}.allocate"] = time.perf_counter() - t0
+            perm, counts = perms[0], counts[0]
+            t0 = time.perf_counter()
+            wc, ws = o.quantize_rows(W[:tw], perm, counts)
+            t[f"{name}.quantize_weight"] = (time.perf_counter() - t0) * N / tw
+            for M in Ms:
+                m = rows(M)
+                t0 = time.perf_counter()
+                ac, as_ = o.quantize_rows(A[M][:m], perm, counts)
+                t[f"{name}.quantize_act_M{M}"] = (time.perf_counter() - t0) * M / m
+                t0 = time.perf_counter()
+                o.gemm(ac, as_, wc, ws, counts)                   # m x tw block of Y
+                t[f"{name}.gemm_M{M}"] = (time.perf_counter() - t0) * (M * N) / (m * tw)
+        T, H, D = KV_SHAPE
+        n_tok = rows(T)
         t0 = time.perf_counter()
-        for kv in self.KV:
-            o.quantize_rows(kv[:n_kv], None, (0, 0, KV_SHAPE[2]))
-        t["quantize_kv"] = (time.perf_counter() - t0) * (KV_SHAPE[0] * KV_SHAPE[1]) / n_kv
+        kv = [o.quantize_rows(x[: n_tok * H], None, (0, 0, D)) for x in self.KV]
+        t["kv.quantize"] = (time.perf_counter() - t0) * T / n_tok
+        t0 = time.perf_counter()
+        o.attn_decode(self.q, kv[0][0][2], kv[0][1][2], kv[1][0][2], kv[1][1][2], n_tok, H, 1.0 / D ** 0.5)
+        t["kv.attn_decode"] = (time.perf_counter() - t0) * T / n_tok
         return sum(t.values()), t
 
 
@@ -469,11 +672,11 @@ def run_reference(args, world):
     """The oracle as the reference arm: rank 0 only, host cores."""
     op = OraclePath(SEED)
     budget_s = 150.0 / max(1, args.steps + args.warmup)
-    frac = 1.0 / 64
+    frac = 1.0 / 256
     t_probe = time.perf_counter()
     op.step(frac)
     dt = time.perf_counter() - t_probe
-    frac = max(1.0 / 512, min(1.0 / 8, frac * budget_s / max(dt, 1e-3)))
+    frac = max(1.0 / 2048, min(1.0 / 8, frac * budget_s / max(dt, 1e-3)))
     for _ in range(args.warmup):
         op.step(frac)
     est = []
@@ -481,84 +684,66 @@ def run_reference(args, world):
         est.append(op.step(frac)[0])
     per_step = statistics.mean(est)
     value = op.gemm_flops / per_step / 1e12
-    sample = (f"row fraction {frac:.5f} of every piece (X, W, A, K/V rows; GEMM on the sampled A x W block), "
-              f"time scaled by 1/fraction; allocation in full; single thread")
+    sample = (f"row fraction {frac:.5f} of every piece (X, W, A, K/V rows; GEMM on the sampled A x W block; "
+              f"attention on a token prefix), time scaled by 1/fraction; allocation in full; single thread")
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
             "config": {"workload": WORKLOAD},
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": sample,
+                             **host_info()},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
 def cpu_baseline():
     """The oracle timed once on ~10-30 s of host work (rank 0, N=1 only)."""
     op = OraclePath(SEED)
-    frac = 1.0 / 32
+    frac = 1.0 / 128
     total, parts = op.step(frac)
     return {"value": op.gemm_flops / total / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
             "sample": f"row fraction {frac:.4f} of each piece of one step (sensitivity, quantisers, a "
-                      f"{frac:.4f}-row x {frac:.4f}-row block of each GEMM), scaled by 1/fraction; allocation "
-                      f"in full; single-threaded C, fp64",
-            "ms_per_step_extrapolated": total * 1e3,
+                      f"{frac:.4f}-row x {frac:.4f}-row block of each GEMM, attention on a {frac:.4f} token prefix),"
+                      f" scaled by 1/fraction; allocation in full; single-threaded C, fp64",
+            "ms_per_step_extrapolated": total * 1e3, **host_info(),
             "parts_s": {k: round(v, 4) for k, v in parts.items()}}
 
 
-def run_mixed_overhead(args):
-    """Time mxs_gemm on one weight under three layouts -- uniform MXINT4, the
-    32 fixed 8-bit columns alone (budget 4.03125 bits) and the 4.5-bit budget
-    -- to measure what the wider blocks cost (the pages estimate ~3% at
-    ~4.03 bits).  CUDA-graph replays of one call, L2 flushed before each,
-    CUDA events around each replay."""
+# ------------------------------------------------------------ multi-process
+def _free_port() -> int:
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def spawn_ranks(n: int, argv) -> int:
+    """Relaunch this script under torch.distributed.run with n processes on
+    this node (rendezvous on 127.0.0.1) and return its exit status; rank 0
+    prints the JSON line."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={_free_port()}", os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
+def probe_ranks(world, rank):
+    """Launch check only (no GPU work): every rank joins the process group
+    and contributes its rank; rank 0 prints what it saw."""
+    import datetime
     import torch
-    from mx_microscaling_mixed_b200 import build
-    build.build()
-    from mx_microscaling_mixed_b200 import capi as c, inputs
-    dev = torch.device("cuda", 0)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-    reps = max(10, min(args.steps, 100))
-    out = {"metric": "mxs_gemm time by layout", "unit": "us", "reps": reps, "shapes": []}
-    for (N, K) in ((4096, 4096), (14336, 4096)):
-        W = inputs.attn_weight(dev, SEED, N, K)
-        X = inputs.gaussian_acts(dev, SEED + 1, T_CAL, K)
-        _, _, s = c.mxs_sensitivity(X, W)
-        layouts = {"uniform4": ((0, 0, K), torch.arange(K, dtype=torch.int32, device=dev))}
-        for name, budget in (("b4.03125", (129, 32)), ("b4.5", (9, 2))):
-            perms, counts = c.mxs_allocate([s], [N], mode="budget", budget=budget)
-            layouts[name] = (counts[0], perms[0])
-        row = {"N": N, "K": K, "counts": {k: list(v[0]) for k, v in layouts.items()}, "us": {}}
-        for M in M_LIST:
-            A = inputs.gaussian_acts(dev, SEED + 2 + M, M, K)
-            for name, (counts, perm) in layouts.items():
-                lay = c.mxs_layout_make(K, counts, perm)
-                Wq, Aq = c.mxtensor_empty(N, lay, dev), c.mxtensor_empty(M, lay, dev)
-                c.mxs_quantize_weight(W, Wq)
-                c.mxs_quantize_act(A, Aq)
-                ws = torch.empty(c.mxs_gemm_workspace_bytes(Aq, Wq) + 1024, dtype=torch.uint8, device=dev)
-                Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-                call = lambda: c.mxs_gemm(Aq, Wq, Y=Y, workspace=ws)
-                for _ in range(3):
-                    call()
-                g = torch.cuda.CUDAGraph()
-                cap = torch.cuda.Stream()
-                with torch.cuda.graph(g, stream=cap):
-                    call()
-                ms = []
-                for _ in range(reps):
-                    flush.zero_()
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    e0.record()
-                    g.replay()
-                    e1.record()
-                    ms.append((e0, e1))
-                torch.cuda.synchronize()
-                row["us"][f"M{M}/{name}"] = statistics.median(a.elapsed_time(b) for a, b in ms) * 1e3
-            base = row["us"][f"M{M}/uniform4"]
-            for name in ("b4.03125", "b4.5"):
-                row["us"][f"M{M}/{name}/overhead"] = row["us"][f"M{M}/{name}"] / base - 1.0
-        out["shapes"].append(row)
-    c.mxs_sync()
-    return out
+    import torch.distributed as dist
+    backend = "nccl" if torch.cuda.is_available() else "gloo"
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0"))) if backend == "nccl" else torch.device("cpu")
+    if backend == "nccl":
+        torch.cuda.set_device(dev)
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
+    t = torch.zeros(world, dtype=torch.float64, device=dev)
+    t[rank] = rank + 1
+    dist.all_reduce(t)
+    job = max_over_ranks(0.1 * (rank + 1), world, dev)
+    if rank == 0:
+        print(json.dumps({"probe": "ranks", "n_gpus": world, "backend": backend,
+                          "ranks_seen": [int(x) - 1 for x in t.tolist()], "max_over_ranks": job}), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
 
 
 def main():
@@ -568,16 +753,18 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mixed-overhead", action="store_true",
-                    help="time mxs_gemm under uniform-4-bit vs mixed layouts and exit")
+    ap.add_argument("--no-extras", action="store_true", help="skip the mixed-overhead table and the budget sweep")
+    ap.add_argument("--probe-ranks", action="store_true", help="launch check: join the process group and exit")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(spawn_ranks(args.gpus, sys.argv[1:]))
     rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.gpus == 1 else 1)))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.mixed_overhead:
-        print(json.dumps(run_mixed_overhead(args)), flush=True)
+    if args.probe_ranks:
+        probe_ranks(world, rank)
         return
     if args.impl == "reference":
         if rank == 0:

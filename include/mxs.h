@@ -6,7 +6,8 @@
  * and section the operation comes from:
  *   [TS]  gist.science technical summary ("Technische Samenvatting") §1-§5;
  *   [ABS] the paper's abstract (insight.artgrammer.co.kr);
- *   [RP]  researchpod.app summary.
+ *   [RP]  researchpod.app summary;
+ *   [RV]  romaanj.github.io review.
  * The pages publish no formula beyond H = X^T X, no bit layout and no API;
  * the fixed readings used by this library are stated at each entry point.
  *
@@ -248,6 +249,32 @@ mxs_status mxs_dequantize(const mxs_mxtensor *in, float *out, int64_t ldo, void 
 mxs_status mxs_gemm_workspace_bytes(const mxs_mxtensor *A, const mxs_mxtensor *W, size_t *bytes);
 mxs_status mxs_gemm(const mxs_mxtensor *A, const mxs_mxtensor *W, void *Y, int64_t ldy,
                     void *ws, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * mxs_attn_decode -- one decode step of grouped-query attention that reads
+ * the 4-bit MXINT K/V cache directly.  [TS §4: the W4A4KV4 setting keeps the
+ * K/V cache in 4-bit MXINT; RV Validation: A4W4KV4 against A4W4KV16.]  The
+ * pages give no attention formula; this is scaled dot-product attention of
+ * one query token on the decoded cache:
+ *   query head h reads kv head g = h / (n_qh / n_kvh);
+ *   s_t = sm_scale * sum_d q[h][d] * deq(K)[t*n_kvh + g][d]      (t < T)
+ *   p = softmax(s);   out[h][d] = sum_t p_t * deq(V)[t*n_kvh + g][d]
+ *   q (device): n_qh x 128 bf16, pitch ldq (elements; 16-byte aligned rows);
+ *   K, V: the caches as mxs_quantize_act writes them with the identity
+ *   layout {0, 0, 128}: T*n_kvh rows, row t*n_kvh + g = token t of kv head g
+ *   (a [T][n_kvh][128] cache flattened token-major), one 4-bit segment;
+ *   out (device): n_qh x 128 fp32, pitch ldo (elements).
+ *   Head dimension 128; n_qh a multiple of n_kvh with n_qh / n_kvh <= 8;
+ *   T >= 1; block scale bytes <= 249 (values below 2^122).
+ *   ws (device, 256-byte aligned): mxs_attn_decode_workspace_bytes(...), the
+ *   per-split partial results (the call splits the tokens over CTAs and
+ *   merges the splits in a second kernel).
+ * Decoded cache values are exact; the dot products accumulate in fp32, the
+ * softmax weights enter the output product with 16 significant bits. */
+mxs_status mxs_attn_decode_workspace_bytes(int64_t T, int64_t n_qh, int64_t n_kvh, int64_t d, size_t *bytes);
+mxs_status mxs_attn_decode(const void *q, int64_t n_qh, int64_t ldq, const mxs_mxtensor *K, const mxs_mxtensor *V,
+                           int64_t T, int64_t n_kvh, float sm_scale, float *out, int64_t ldo,
+                           void *ws, size_t ws_bytes, void *stream);
 
 #ifdef __cplusplus
 }

@@ -84,12 +84,15 @@ _sig("mxs_quantize_act", [_P, _ST, _I64, _I64, ctypes.POINTER(MXTensorC), _P])
 _sig("mxs_dequantize", [ctypes.POINTER(MXTensorC), _P, _I64, _P])
 _sig("mxs_gemm_workspace_bytes", [ctypes.POINTER(MXTensorC), ctypes.POINTER(MXTensorC), ctypes.POINTER(_SZ)])
 _sig("mxs_gemm", [ctypes.POINTER(MXTensorC), ctypes.POINTER(MXTensorC), _P, _I64, _P, _SZ, _P])
+_sig("mxs_attn_decode_workspace_bytes", [_I64, _I64, _I64, _I64, ctypes.POINTER(_SZ)])
+_sig("mxs_attn_decode", [_P, _I64, _I64, ctypes.POINTER(MXTensorC), ctypes.POINTER(MXTensorC), _I64, _I64,
+                         ctypes.c_float, _P, _I64, _P, _SZ, _P])
 
 EXPORTS = ["mxs_status_str", "mxs_launch_count", "mxs_sync", "mxs_layout_make", "mxs_mxtensor_bytes",
            "mxs_sensitivity_workspace_bytes", "mxs_sensitivity", "mxs_sensitivity_noalloc",
            "mxs_allocate_workspace_bytes",
            "mxs_allocate", "mxs_quantize_weight", "mxs_quantize_act", "mxs_dequantize",
-           "mxs_gemm_workspace_bytes", "mxs_gemm"]
+           "mxs_gemm_workspace_bytes", "mxs_gemm", "mxs_attn_decode_workspace_bytes", "mxs_attn_decode"]
 
 
 def _check(st: int, where: str):
@@ -316,6 +319,32 @@ def mxs_gemm(A: MXTensor, W: MXTensor, Y: Optional[torch.Tensor] = None, workspa
     _check(_lib.mxs_gemm(ctypes.byref(A.c), ctypes.byref(W.c), Y.data_ptr(), Y.stride(0), _aligned_ptr(ws), need,
                          _stream(stream)), "mxs_gemm")
     return Y
+
+
+# -------------------------------------------------------- decode attention
+def mxs_attn_decode_workspace_bytes(T: int, n_qh: int, n_kvh: int, d: int = 128) -> int:
+    need = _SZ(0)
+    _check(_lib.mxs_attn_decode_workspace_bytes(T, n_qh, n_kvh, d, ctypes.byref(need)),
+           "mxs_attn_decode_workspace_bytes")
+    return need.value
+
+
+def mxs_attn_decode(q: torch.Tensor, K: MXTensor, V: MXTensor, T: int, n_kvh: int, sm_scale: float,
+                    out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """fp32 (n_qh x 128) output of one decode step of grouped-query attention
+    over the MXINT4 K/V caches K and V (T*n_kvh rows each, token-major)."""
+    if q.dtype != torch.bfloat16:
+        raise TypeError("q must be bf16")
+    n_qh = q.shape[0]
+    if out is None:
+        out = torch.empty((n_qh, q.shape[1]), dtype=torch.float32, device=q.device)
+    need = mxs_attn_decode_workspace_bytes(T, n_qh, n_kvh, q.shape[1])
+    ws = workspace if workspace is not None else _workspace(need, q.device)
+    _check(_lib.mxs_attn_decode(q.data_ptr(), n_qh, _rowmajor(q), ctypes.byref(K.c), ctypes.byref(V.c), T, n_kvh,
+                                float(sm_scale), out.data_ptr(), _rowmajor(out), _aligned_ptr(ws, 256), need,
+                                _stream(stream)), "mxs_attn_decode")
+    return out
 
 
 def mxs_sync(stream=None) -> None:

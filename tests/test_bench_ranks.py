@@ -7,10 +7,14 @@ throughput, every rank's work over that time.  Both are exercised here with
 ranks whose local times differ.
 """
 import datetime
+import json
 import os
 import socket
+import subprocess
+import sys
 
 import pytest
+import torch
 import torch.multiprocessing as mp
 
 import bench
@@ -60,3 +64,16 @@ def test_two_ranks_take_the_slowest_time_and_add_their_work():
         assert job == 0.75, rank
         # two replicas of 4 steps x 2 TFLOP each, over the slowest rank's 0.75 s
         assert tflops == pytest.approx(2 * 4 * 2.0 / 0.75)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="gloo ranks on CPU hosts; GPU hosts give each rank a GPU")
+def test_gpus_flag_launches_that_many_ranks():
+    """`bench.py --gpus 2` outside torchrun relaunches itself as two ranks
+    (here the launch check only: each rank joins the group and reports)."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--probe-ranks"],
+                         capture_output=True, text=True, timeout=180, cwd=root)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads([l for l in out.stdout.splitlines() if l.startswith("{")][-1])
+    assert line["n_gpus"] == 2 and line["ranks_seen"] == [0, 1] and line["backend"] == "gloo"
+    assert line["max_over_ranks"] == pytest.approx(0.2)

@@ -339,24 +339,63 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const __grid_c
   }
 }
 
-// One CTA per query head, one thread per head-dimension position: the
-// splits' weights 2^(m_j - M) rescale their sums and partial outputs.
-__global__ void __launch_bounds__(kAttnD) attn_combine_kernel(AttnArgs a) {
+// One CTA per query head.  The splits' weights 2^(m_j - M) rescale their
+// sums and partial outputs; thread (group r, position d) adds the splits
+// j = r, r + 4, ... for position d with several loads in flight, and the
+// four groups are added in group order (the result does not depend on the
+// launch).
+constexpr int kCombGroups = 4;
+constexpr int kCombThreads = kCombGroups * kAttnD;
+
+__global__ void __launch_bounds__(kCombThreads) attn_combine_kernel(AttnArgs a) {
   pdl_wait();
   pdl_trigger();
-  const int h = blockIdx.x, d = threadIdx.x;
+  __shared__ float red[kCombGroups][kAttnD];
+  __shared__ float wred[kCombThreads / 32];
+  const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t stride = static_cast<int64_t>(a.n_qh) * (kAttnD + 2);
   const float *p = a.part + static_cast<int64_t>(h) * (kAttnD + 2);
-  float M = -INFINITY;
-  for (int j = 0; j < a.splits; ++j) M = fmaxf(M, p[j * stride]);
-  float num = 0.f, den = 0.f;
-  for (int j = 0; j < a.splits; ++j) {
-    const float *pj = p + j * stride;
-    const float w = exp2f(pj[0] - M);
-    den = fmaf(w, pj[1], den);
-    num = fmaf(w, pj[2 + d], num);
+  // M = max_j m_j
+  float m = -INFINITY;
+  for (int j = tid; j < a.splits; j += kCombThreads) m = fmaxf(m, p[j * stride]);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) wred[warp] = m;
+  __syncthreads();
+  float M = wred[0];
+#pragma unroll
+  for (int w = 1; w < kCombThreads / 32; ++w) M = fmaxf(M, wred[w]);
+  __syncthreads();
+  // the denominator sum_j 2^(m_j - M) l_j, in split order (one warp)
+  if (warp == 0) {
+    float den = 0.f;
+    for (int j0 = 0; j0 < a.splits; j0 += 32) {
+      const int j = j0 + lane;
+      float v = j < a.splits ? exp2f(p[j * stride] - M) * p[j * stride + 1] : 0.f;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;                        // prefix sums: lane 31 holds the 32-split sum
+      }
+      den += __shfl_sync(0xffffffffu, v, 31);
+    }
+    if (lane == 0) wred[0] = den;
   }
-  a.out[static_cast<int64_t>(h) * a.ldo + d] = num / den;
+  const int r = tid / kAttnD, d = tid - r * kAttnD;
+  float num = 0.f;
+#pragma unroll 4
+  for (int j = r; j < a.splits; j += kCombGroups) {
+    const float *pj = p + j * stride;
+    num = fmaf(exp2f(pj[0] - M), pj[2 + d], num);
+  }
+  red[r][d] = num;
+  __syncthreads();
+  if (r == 0) {
+    float sum = red[0][d];
+#pragma unroll
+    for (int g = 1; g < kCombGroups; ++g) sum += red[g][d];
+    a.out[static_cast<int64_t>(h) * a.ldo + d] = sum / wred[0];
+  }
 }
 
 namespace {
@@ -467,7 +506,7 @@ extern "C" mxs_status mxs_attn_decode(const void *q, int64_t n_qh, int64_t ldq, 
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   launch_pdl(attn_split_kernel, dim3(static_cast<unsigned>(a.splits * n_kvh)), dim3(kAttnThreads),
              static_cast<size_t>(smem), cs, mKc, mKs, mVc, mVs, a, status);
-  launch_pdl(attn_combine_kernel, dim3(static_cast<unsigned>(n_qh)), dim3(kAttnD), 0, cs, a);
+  launch_pdl(attn_combine_kernel, dim3(static_cast<unsigned>(n_qh)), dim3(kCombThreads), 0, cs, a);
   count_launch(2);
   return cuda_status(cudaGetLastError());
 }

@@ -156,7 +156,8 @@ def rank_order(s) -> np.ndarray:
 
 def allocate(s_list, N_list, *, mode: str, budget=(9, 2), p8=(5, 100), p6=(15, 100),
              fixed8: int = 32, layer_w=None):
-    """Bit allocation over layers.  mode 'fractions' or 'budget'.
+    """Bit allocation over layers.  mode 'fractions', 'budget' or 'layer'
+    (the layer-score rule; layer_w holds the layer scores).
 
     Returns (perms, counts) with counts an (L, 3) int64 array of (n8, n6, n4).
     Raises ValueError if the fixed 8-bit blocks exceed the budget."""
@@ -171,7 +172,7 @@ def allocate(s_list, N_list, *, mode: str, budget=(9, 2), p8=(5, 100), p6=(15, 1
     w = None if layer_w is None else _f64(layer_w)
     rc = lib().orc_allocate(Lc, _ptr(K), _ptr(N), ctypes.cast(sp, ctypes.c_void_p),
                             None if w is None else _ptr(w),
-                            0 if mode == "fractions" else 1,
+                            {"fractions": 0, "budget": 1, "layer": 2}[mode],
                             int(budget[0]), int(budget[1]), int(p8[0]), int(p8[1]),
                             int(p6[0]), int(p6[1]), int(fixed8),
                             ctypes.cast(pp, ctypes.c_void_p), _ptr(counts))

@@ -236,6 +236,39 @@ static int64_t orc_round_frac(int64_t num, int64_t den, int64_t K)
     return (2 * num * K + den) / (2 * den);
 }
 
+/* The layer-score rule's steps.  Layer l with score w_l > 0 reaches its
+ * k-th 32-column 6-bit group when R * w_l >= 32 k, i.e. at R = 32 k / w_l.
+ * Steps are ordered by that R, compared exactly: k_a / w_a < k_b / w_b iff
+ * k_a * w_b < k_b * w_a, each product taken exactly as the pair (rounded
+ * product, its rounding error from fma), compared lexicographically. */
+typedef struct {
+    int layer;
+    int64_t k;        /* group index, 1-based */
+    int64_t cols;     /* 32, or fewer for the last group */
+} orc_rstep;
+
+static const double *g_rscore = NULL;
+
+static int orc_rstep_cmp_values(const orc_rstep *a, const orc_rstep *b)
+{
+    double ka = (double)a->k, kb = (double)b->k;
+    double wa = g_rscore[a->layer], wb = g_rscore[b->layer];
+    double p1 = ka * wb, e1 = fma(ka, wb, -p1);     /* k_a * w_b exactly = p1 + e1 */
+    double p2 = kb * wa, e2 = fma(kb, wa, -p2);     /* k_b * w_a exactly = p2 + e2 */
+    if (p1 != p2) return p1 < p2 ? -1 : 1;
+    if (e1 != e2) return e1 < e2 ? -1 : 1;
+    return 0;
+}
+
+static int orc_rstep_cmp(const void *pa, const void *pb)
+{
+    const orc_rstep *a = (const orc_rstep *)pa, *b = (const orc_rstep *)pb;
+    int c = orc_rstep_cmp_values(a, b);
+    if (c) return c;
+    if (a->layer != b->layer) return a->layer < b->layer ? -1 : 1;   /* fixes qsort's order only */
+    return a->k < b->k ? -1 : (a->k > b->k);
+}
+
 /* Bit allocation for n_layers linear layers.
  *   mode 0 (fractions): n8 = round(p8*K), n6 = round(p6*K) (half up, exact),
  *                       the rest 4-bit.
@@ -250,6 +283,17 @@ static int64_t orc_round_frac(int64_t num, int64_t den, int64_t K)
  *                       candidate that does not fit [TS §2.3: the 6-bit count
  *                       follows the layer's sensitivity, scaled to meet the
  *                       global average budget].
+ *   mode 2 (layer score): n8 as in mode 1; the 6-bit count of layer l is
+ *                       proportional to its layer score w_l = layer_w[l],
+ *                       scaled by one global R [TS §2.3 "Dynamische 6-bit
+ *                       Allocatie"], in whole 32-column groups:
+ *                         n6_l(R) = min(K_l - n8_l, 32 * floor(R * w_l / 32)),
+ *                       with R the largest value whose counts meet the
+ *                       budget.  n6_l(R) only changes at R = 32 k / w_l, so
+ *                       R is found by taking those steps in increasing R
+ *                       (all steps at one R value together) until the next
+ *                       value's steps no longer fit.  A layer with w_l = 0
+ *                       gets no 6-bit columns.
  *   Budget accounting: average mantissa bits over all weight elements, E8M0
  *   scales excluded; with B = num/den the test is
  *     sum_l N_l (4 K_l + 4 n8_l + 2 n6_l) * den <= num * sum_l N_l K_l.
@@ -266,6 +310,11 @@ int orc_allocate(int n_layers, const int64_t *K, const int64_t *N,
                  int64_t fixed8, int32_t *const *perm, int64_t *counts)
 {
     if (n_layers <= 0 || den <= 0) return 2;
+    if (mode == 2) {
+        if (!layer_w) return 2;
+        for (int l = 0; l < n_layers; ++l)
+            if (!(layer_w[l] >= 0.0) || !isfinite(layer_w[l])) return 2;
+    }
     int32_t **order = (int32_t **)calloc((size_t)n_layers, sizeof(int32_t *));
     for (int l = 0; l < n_layers; ++l) {
         order[l] = (int32_t *)malloc(sizeof(int32_t) * (size_t)(K[l] > 0 ? K[l] : 1));
@@ -290,6 +339,36 @@ int orc_allocate(int n_layers, const int64_t *K, const int64_t *N,
         }
         if (used > cap) {
             rc = 1;
+        } else if (mode == 2) {
+            int64_t nsteps = 0;
+            for (int l = 0; l < n_layers; ++l)
+                if (layer_w[l] > 0.0) nsteps += (K[l] - n8[l] + 31) / 32;
+            orc_rstep *st = (orc_rstep *)malloc(sizeof(orc_rstep) * (size_t)(nsteps + 1));
+            int64_t i = 0;
+            for (int l = 0; l < n_layers; ++l) {
+                if (!(layer_w[l] > 0.0)) continue;
+                int64_t avail = K[l] - n8[l];
+                for (int64_t k = 1; 32 * (k - 1) < avail; ++k) {
+                    st[i].layer = l;
+                    st[i].k = k;
+                    st[i].cols = avail - 32 * (k - 1) < 32 ? avail - 32 * (k - 1) : 32;
+                    ++i;
+                }
+            }
+            g_rscore = layer_w;
+            qsort(st, (size_t)nsteps, sizeof(orc_rstep), orc_rstep_cmp);
+            for (int64_t a = 0; a < nsteps;) {
+                int64_t b = a + 1;
+                while (b < nsteps && orc_rstep_cmp_values(&st[a], &st[b]) == 0) ++b;
+                __int128 add = 0;
+                for (int64_t j = a; j < b; ++j) add += (__int128)den * 2 * N[st[j].layer] * st[j].cols;
+                if (used + add > cap) break;          /* R stays below this step value */
+                used += add;
+                for (int64_t j = a; j < b; ++j) n6[st[j].layer] += st[j].cols;
+                a = b;
+            }
+            g_rscore = NULL;
+            free(st);
         } else {
             for (;;) {
                 int best = -1;

@@ -141,3 +141,76 @@ def test_layer_weight_steers_upgrades():
     assert list(c[:, 1]) == [0, 64]           # both go to the heavier layer
     _, c = oracle.allocate(s, [10, 10], mode="budget", budget=(93, 20), layer_w=[1.0, 1.0])
     assert list(c[:, 1]) == [64, 0]           # equal ratios: the lower layer wins each tie
+
+
+# ------------------------------------------------ layer-score rule (mode 2)
+def _r_rule_brute(K, N, scores, budget, fixed8=32):
+    """The layer-score rule from its definition, with exact fractions: every
+    R at which some layer's count changes (R = 32 k / w) is a candidate;
+    n6_l(R) = min(K_l - n8_l, 32 floor(R w_l / 32)); the answer is the counts
+    at the largest candidate R (or 0) whose counts meet the budget."""
+    n8 = [min(fixed8, k) for k in K]
+    cands = {Fraction(0)}
+    for k, w, e in zip(K, scores, n8):
+        if w > 0:
+            for j in range(1, (k - e + 31) // 32 + 1):
+                cands.add(Fraction(32 * j) / Fraction(w))
+    best = None
+    for R in sorted(cands):
+        n6 = [min(k - e, 32 * int((R * Fraction(w)) // 32)) if w > 0 else 0 for k, w, e in zip(K, scores, n8)]
+        used = sum(n * (4 * k + 4 * e + 2 * c) for k, n, e, c in zip(K, N, n8, n6))
+        if Fraction(used, sum(n * k for k, n in zip(K, N))) <= Fraction(*budget):
+            best = n6
+        else:
+            break
+    return [(e, c, k - e - c) for k, e, c in zip(K, n8, best)]
+
+
+def test_layer_rule_is_proportional_and_meets_the_budget():
+    s = [np.random.default_rng(i).random(4096) for i in range(2)]
+    _, counts = oracle.allocate(s, [4096, 4096], mode="layer", budget=(9, 2), layer_w=[2.0, 1.0])
+    assert [tuple(c) for c in counts] == [(32, 1280, 2784), (32, 640, 3424)]
+    assert Fraction(_used_bits([4096] * 2, [4096] * 2, counts), 2 * 4096 * 4096) == Fraction(9, 2)
+
+
+@pytest.mark.parametrize("K,N,budget,n6", [
+    (4096, 4096, (9, 2), 960), (14336, 4096, (9, 2), 3520), (8192, 8192, (17, 4), 960),
+    (28672, 8192, (17, 4), 3520), (4096, 4096, (129, 32), 0)])
+def test_layer_rule_single_layer_closed_form(K, N, budget, n6):
+    # one layer: R only scales that layer, so the rule fills the budget
+    s = np.random.default_rng(K).random(K)
+    _, counts = oracle.allocate([s], [N], mode="layer", budget=budget, layer_w=[0.37])
+    assert tuple(counts[0]) == (32, n6, K - 32 - n6)
+
+
+def test_layer_rule_zero_score_and_ties():
+    s = [np.random.default_rng(i).random(256) for i in range(3)]
+    # a zero score gets no 6-bit columns; the others share the budget
+    _, counts = oracle.allocate(s, [64, 64, 64], mode="layer", budget=(5, 1), layer_w=[1.0, 0.0, 1.0])
+    assert counts[1][1] == 0 and counts[0][1] == counts[2][1] > 0
+    # equal scores on equal layers step together: a budget with room for
+    # three 32-column groups takes two (one each), never three
+    K, N = [256, 256], [16, 16]
+    used0 = sum(n * (4 * k + 4 * 32) for k, n in zip(K, N))
+    room = used0 + 3 * 2 * 16 * 32
+    _, counts = oracle.allocate([s[0], s[1]], N, mode="layer", budget=(room, sum(n * k for k, n in zip(K, N))),
+                                layer_w=[0.5, 0.5])
+    assert [c[1] for c in counts] == [32, 32]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_layer_rule_matches_brute_force(seed):
+    rng = np.random.default_rng(100 + seed)
+    L = int(rng.integers(1, 5))
+    K = [int(rng.choice([40, 64, 100, 130, 200])) for _ in range(L)]
+    N = [int(rng.choice([8, 16, 24])) for _ in range(L)]
+    scores = [float(rng.choice([0.0, rng.random(), rng.random() * 10, 1.0])) for _ in range(L)]
+    budget = (int(rng.integers(41, 60)), 10)
+    s = [rng.random(k) for k in K]
+    try:
+        _, counts = oracle.allocate(s, N, mode="layer", budget=budget, layer_w=scores)
+    except ValueError:
+        used = sum(n * (4 * k + 4 * min(32, k)) for k, n in zip(K, N))
+        assert Fraction(used, sum(n * k for k, n in zip(K, N))) > Fraction(*budget)
+        return
+    assert [tuple(int(x) for x in c) for c in counts] == _r_rule_brute(K, N, scores, budget)

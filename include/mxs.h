@@ -95,7 +95,7 @@ typedef struct {
     int64_t scale_pitch[3];
 } mxs_mxtensor;
 
-enum { MXS_ALLOC_FRACTIONS = 0, MXS_ALLOC_BUDGET = 1 };
+enum { MXS_ALLOC_FRACTIONS = 0, MXS_ALLOC_BUDGET = 1, MXS_ALLOC_LAYER = 2 };
 
 /* Bit-allocation policy.
  *   MXS_ALLOC_FRACTIONS: n8 = round(p8*K), n6 = round(p6*K) (half up, exact
@@ -105,7 +105,17 @@ enum { MXS_ALLOC_FRACTIONS = 0, MXS_ALLOC_BUDGET = 1 };
  *     block]; then greedy 6-bit upgrades of 32-column groups under an average
  *     mantissa-bit budget num/den over all weight elements, E8M0 scales not
  *     counted [TS §2.3 dynamic 6-bit allocation; TS §4 hardware overhead:
- *     4 + 4*32/4096 = 4.03 bits for the fixed block alone]. */
+ *     4 + 4*32/4096 = 4.03 bits for the fixed block alone].
+ *   MXS_ALLOC_LAYER: n8 as in MXS_ALLOC_BUDGET; the 6-bit count of layer l
+ *     is proportional to its layer score w_l (mxs_allocate's layer_w, e.g.
+ *     from mxs_layer_scores), scaled by one global R that meets the budget
+ *     [TS §2.3 "Dynamische 6-bit Allocatie"], in whole 32-column groups:
+ *       n6_l(R) = min(K_l - n8_l, 32 * floor(R * w_l / 32)),
+ *     R the largest value whose counts fit.  The counts change only at
+ *     R = 32 k / w_l; those steps are taken in increasing R (ordered
+ *     exactly: k_a w_b against k_b w_a as exact products), all steps of one
+ *     R value together, until the next value's steps no longer fit.  No
+ *     device data is read, so the call never synchronises. */
 typedef struct {
     int32_t mode;
     int64_t num, den;
@@ -195,8 +205,9 @@ mxs_status mxs_sensitivity_noalloc(const void *X, mxs_dtype xt, int64_t T, int64
  *   fp64, ties to the lower layer) and stop at the first that does not fit
  *   sum_l N_l (4 K_l + 4 n8_l + 2 n6_l) * den <= num * sum_l N_l K_l.
  *   Inputs: K, N (host, n_layers each); s (host array of n_layers device
- *   pointers, K[l] doubles each, finite and >= 0); layer_w (host, n_layers,
- *   or NULL = all 1).
+ *   pointers, K[l] doubles each, finite and >= 0); layer_w (host, n_layers):
+ *   in MXS_ALLOC_BUDGET the greedy's gain weights (NULL = all 1), in
+ *   MXS_ALLOC_LAYER the layer scores (required, finite, >= 0).
  *   Outputs: perm (host array of device pointers, K[l] int32 each: the
  *   8-bit columns, then 6-bit, then 4-bit, ascending within each);
  *   counts (host, 3*n_layers: n8, n6, n4 per layer).

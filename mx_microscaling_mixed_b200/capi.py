@@ -20,7 +20,7 @@ if not os.path.exists(_LIB_PATH):
 _lib = ctypes.CDLL(_LIB_PATH)
 
 MXS_F32, MXS_BF16 = 0, 1
-MXS_ALLOC_FRACTIONS, MXS_ALLOC_BUDGET = 0, 1
+MXS_ALLOC_FRACTIONS, MXS_ALLOC_BUDGET, MXS_ALLOC_LAYER = 0, 1, 2
 SEG_BITS = (8, 6, 4)
 
 STATUS = {0: "MXS_OK", 1: "MXS_ERR_ARG", 2: "MXS_ERR_SHAPE", 3: "MXS_ERR_ALIGN", 4: "MXS_ERR_DTYPE",
@@ -248,7 +248,7 @@ def mxs_sensitivity_noalloc(X: torch.Tensor, W: torch.Tensor, out, stream=None):
 # --------------------------------------------------------------- allocation
 def make_budget(mode: str, budget=(9, 2), p8=(5, 100), p6=(15, 100), fixed8: int = 32) -> BudgetC:
     b = BudgetC()
-    b.mode = MXS_ALLOC_FRACTIONS if mode == "fractions" else MXS_ALLOC_BUDGET
+    b.mode = {"fractions": MXS_ALLOC_FRACTIONS, "budget": MXS_ALLOC_BUDGET, "layer": MXS_ALLOC_LAYER}[mode]
     b.num, b.den = int(budget[0]), int(budget[1])
     b.p8_num, b.p8_den = int(p8[0]), int(p8[1])
     b.p6_num, b.p6_den = int(p6[0]), int(p6[1])
@@ -260,6 +260,7 @@ def mxs_allocate(s_list: Sequence[torch.Tensor], N_list: Sequence[int], *, mode:
                  p8=(5, 100), p6=(15, 100), fixed8: int = 32, layer_w=None, stream=None,
                  perms: Optional[List[torch.Tensor]] = None, workspace: Optional[torch.Tensor] = None):
     """Returns (perms: list of device int32 tensors, counts: list of (n8, n6, n4)).
+    mode: "fractions", "budget" or "layer" (layer_w = the layer scores).
     Synchronises the stream only in multi-layer budget mode."""
     L = len(s_list)
     dev = s_list[0].device

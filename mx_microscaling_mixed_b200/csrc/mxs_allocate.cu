@@ -24,6 +24,7 @@
 // run on the host side of the call; only the multi-layer greedy needs device
 // data (the group gains) and so a stream synchronisation.
 #include <algorithm>
+#include <cmath>
 #include <vector>
 
 #include "mxs_internal.cuh"
@@ -223,6 +224,46 @@ static void budget_base(int32_t n_layers, const int64_t *K, const int64_t *N, co
   }
 }
 
+// The layer-score rule: layer l with score w_l > 0 reaches its k-th
+// 32-column 6-bit group at R = 32 k / w_l.  Steps are ordered by that R,
+// compared exactly (k_a w_b against k_b w_a, each product as the pair of its
+// rounded value and its fma rounding error, compared lexicographically), and
+// taken in increasing R, all steps of one R value together, while they fit.
+struct RStep {
+  int32_t layer;
+  int64_t k, cols;
+};
+
+static int rstep_cmp(const RStep &a, const RStep &b, const double *w) {
+  const double ka = static_cast<double>(a.k), kb = static_cast<double>(b.k);
+  const double p1 = ka * w[b.layer], e1 = std::fma(ka, w[b.layer], -p1);
+  const double p2 = kb * w[a.layer], e2 = std::fma(kb, w[a.layer], -p2);
+  if (p1 != p2) return p1 < p2 ? -1 : 1;
+  if (e1 != e2) return e1 < e2 ? -1 : 1;
+  return 0;
+}
+
+static void layer_rule(int32_t n_layers, const int64_t *K, const int64_t *N, const double *w, const mxs_budget &B,
+                       const std::vector<int64_t> &n8, __int128 cap, __int128 used, std::vector<int64_t> &n6) {
+  std::vector<RStep> st;
+  for (int l = 0; l < n_layers; ++l) {
+    if (!(w[l] > 0.0)) continue;
+    const int64_t avail = K[l] - n8[l];
+    for (int64_t k = 1; 32 * (k - 1) < avail; ++k) st.push_back(RStep{l, k, std::min<int64_t>(32, avail - 32 * (k - 1))});
+  }
+  std::sort(st.begin(), st.end(), [w](const RStep &a, const RStep &b) { return rstep_cmp(a, b, w) < 0; });
+  for (size_t a = 0; a < st.size();) {
+    size_t b = a + 1;
+    while (b < st.size() && rstep_cmp(st[a], st[b], w) == 0) ++b;
+    __int128 add = 0;
+    for (size_t j = a; j < b; ++j) add += static_cast<__int128>(B.den) * 2 * N[st[j].layer] * st[j].cols;
+    if (used + add > cap) break;                     // R stays below this step value
+    used += add;
+    for (size_t j = a; j < b; ++j) n6[st[j].layer] += st[j].cols;
+    a = b;
+  }
+}
+
 extern "C" mxs_status mxs_allocate(int32_t n_layers, const int64_t *K, const int64_t *N,
                                    const double *const *s, const double *layer_w,
                                    const mxs_budget *budget, int32_t *const *perm,
@@ -235,8 +276,13 @@ extern "C" mxs_status mxs_allocate(int32_t n_layers, const int64_t *K, const int
   const mxs_budget &B = *budget;
   if (B.mode == MXS_ALLOC_FRACTIONS) {
     if (B.p8_den <= 0 || B.p6_den <= 0 || B.p8_num < 0 || B.p6_num < 0) return MXS_ERR_ARG;
-  } else if (B.mode == MXS_ALLOC_BUDGET) {
+  } else if (B.mode == MXS_ALLOC_BUDGET || B.mode == MXS_ALLOC_LAYER) {
     if (B.den <= 0 || B.num < 0 || B.fixed8 < 0) return MXS_ERR_ARG;
+    if (B.mode == MXS_ALLOC_LAYER) {
+      if (!layer_w) return MXS_ERR_ARG;
+      for (int l = 0; l < n_layers; ++l)
+        if (!(layer_w[l] >= 0.0) || !std::isfinite(layer_w[l])) return MXS_ERR_ARG;
+    }
     __int128 cap, used;
     budget_base(n_layers, K, N, B, cap, used);
     if (used > cap) return MXS_ERR_BUDGET;           // before any launch
@@ -268,6 +314,11 @@ extern "C" mxs_status mxs_allocate(int32_t n_layers, const int64_t *K, const int
       n8[l] = std::min(round_half_up_frac(B.p8_num, B.p8_den, K[l]), K[l]);
       n6[l] = std::min(round_half_up_frac(B.p6_num, B.p6_den, K[l]), K[l] - n8[l]);
     }
+  } else if (B.mode == MXS_ALLOC_LAYER) {
+    __int128 cap, used;
+    budget_base(n_layers, K, N, B, cap, used);     // feasible: checked above
+    for (int l = 0; l < n_layers; ++l) n8[l] = std::min(B.fixed8, K[l]);
+    layer_rule(n_layers, K, N, layer_w, B, n8, cap, used, n6);
   } else {
     __int128 cap, used;
     budget_base(n_layers, K, N, B, cap, used);     // feasible: checked above

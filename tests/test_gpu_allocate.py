@@ -100,3 +100,25 @@ def test_llama3_8b_stack_global_budget(c):
     bits = sum(n * (8 * a + 6 * b + 4 * d) for n, (a, b, d) in zip(Ns, gc))
     elems = sum(n * k for n, k in shapes)
     assert bits <= 4.5 * elems                          # the budget holds across the stack
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_layer_score_rule(c, seed):
+    """MXS_ALLOC_LAYER: 6-bit counts proportional to the layer scores under one
+    global R; counts and permutations exact against the oracle, including
+    zero scores and repeated scores (steps taken together)."""
+    rng = np.random.default_rng(40 + seed)
+    L = 6
+    Ks = [int(k) for k in rng.integers(100, 5000, L)]
+    Ns = [int(n) for n in rng.integers(16, 1024, L)]
+    s_np = [rng.integers(0, 50, k).astype(np.float64) * 0.25 for k in Ks]
+    w = [float(x) for x in rng.choice([0.0, 0.5, 1.0, 1.0, 2.75, float(rng.random())], L)]
+    s_dev = [torch.from_numpy(x).cuda() for x in s_np]
+    n0 = c.mxs_launch_count()
+    gp, gc = c.mxs_allocate(s_dev, Ns, mode="layer", budget=(9, 2), layer_w=w)
+    op, oc = oracle.allocate(s_np, Ns, mode="layer", budget=(9, 2), layer_w=w)
+    _cmp(gp, gc, op, oc)
+    assert c.mxs_launch_count() - n0 == 2 * L             # rank + placement per layer, no gains pass
+    with pytest.raises(c.MxsError) as e:
+        c.mxs_allocate(s_dev, Ns, mode="layer", budget=(9, 2), layer_w=None)
+    assert e.value.status == 1

@@ -287,6 +287,48 @@ mxs_status mxs_attn_decode(const void *q, int64_t n_qh, int64_t ldq, const mxs_m
                            int64_t T, int64_t n_kvh, float sm_scale, float *out, int64_t ldo,
                            void *ws, size_t ws_bytes, void *stream);
 
+/* ---------------------------------------------------------------------------
+ * mxs_layer_scores -- layer-wise sensitivity of a decoder stack.
+ * [TS §2.1 "Laaggewijze Sensitiviteit": a layer's score is the L2 error at
+ * the model's final output when that layer alone is quantised; TS §2.3: the
+ * scores set each layer's 6-bit count, mxs_allocate's MXS_ALLOC_LAYER.]
+ * The pages name the measure, not the model code; the readings:
+ *   - the model is a Llama-architecture decoder stack without embedding
+ *     table or LM head: x (T synthetic hidden states) goes in, the final
+ *     RMSNorm of the last block's output comes out.  Block: RMSNorm (weight
+ *     1, eps rms_eps) -> q, k, v projections -> rotary embedding (pair
+ *     (i, i + d/2) of each head turned by t * rope_theta^(-2i/d) at token
+ *     t) -> causal softmax attention (scale 1/sqrt(d), query head h on kv
+ *     head h / (n_heads / n_kv_heads)) -> o projection + residual ->
+ *     RMSNorm -> silu(gate) * up -> down projection + residual;
+ *   - "quantised" is this library's W4A4 MXINT4 layer: the linear's fp32
+ *     input through mxs_quantize_act and its bf16 weight through
+ *     mxs_quantize_weight, both in the uniform 4-bit layout {0, 0, K}, then
+ *     mxs_gemm (bf16 output);
+ *   - score = Frobenius norm of (output with that layer quantised) minus
+ *     (output of the unquantised stack), in fp64.
+ * The unquantised stack runs in fp32 (bf16 weights widened exactly).
+ *   m: the stack; m->W (host array of 7 * n_blocks device pointers, bf16,
+ *   row-major out x in, 16-byte aligned) in the order q (n_heads*d x
+ *   hidden), k, v (n_kv_heads*d x hidden), o (hidden x n_heads*d), gate, up
+ *   (mlp x hidden), down (hidden x mlp) per block, d = hidden / n_heads.
+ *   x (device): T x hidden fp32, pitch ldx; 1 <= T <= 1024.
+ *   scores (host): 7 * n_blocks doubles, layer 7 b + j = linear j of block b.
+ *   hidden, mlp and n_heads*d multiples of 32; d even, <= 256; n_heads a
+ *   multiple of n_kv_heads.
+ *   ws (device, 256-byte aligned): mxs_layer_scores_workspace_bytes(m, T).
+ * A calibration routine, not a per-token one: it runs 1 + 7 * n_blocks
+ * partial forward passes and synchronises `stream` to return the scores. */
+typedef struct {
+    int32_t n_blocks;
+    int32_t hidden, n_heads, n_kv_heads, mlp;
+    float rms_eps, rope_theta;
+    const void *const *W;
+} mxs_stack;
+mxs_status mxs_layer_scores_workspace_bytes(const mxs_stack *m, int64_t T, size_t *bytes);
+mxs_status mxs_layer_scores(const mxs_stack *m, const float *x, int64_t T, int64_t ldx, double *scores,
+                            void *ws, size_t ws_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -50,6 +50,12 @@ class MXTensorC(ctypes.Structure):
                 ("scale_pitch", ctypes.c_int64 * 3)]
 
 
+class StackC(ctypes.Structure):
+    _fields_ = [("n_blocks", ctypes.c_int32), ("hidden", ctypes.c_int32), ("n_heads", ctypes.c_int32),
+                ("n_kv_heads", ctypes.c_int32), ("mlp", ctypes.c_int32), ("rms_eps", ctypes.c_float),
+                ("rope_theta", ctypes.c_float), ("W", ctypes.c_void_p)]
+
+
 class BudgetC(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("num", ctypes.c_int64), ("den", ctypes.c_int64),
                 ("p8_num", ctypes.c_int64), ("p8_den", ctypes.c_int64), ("p6_num", ctypes.c_int64),
@@ -84,6 +90,8 @@ _sig("mxs_quantize_act", [_P, _ST, _I64, _I64, ctypes.POINTER(MXTensorC), _P])
 _sig("mxs_dequantize", [ctypes.POINTER(MXTensorC), _P, _I64, _P])
 _sig("mxs_gemm_workspace_bytes", [ctypes.POINTER(MXTensorC), ctypes.POINTER(MXTensorC), ctypes.POINTER(_SZ)])
 _sig("mxs_gemm", [ctypes.POINTER(MXTensorC), ctypes.POINTER(MXTensorC), _P, _I64, _P, _SZ, _P])
+_sig("mxs_layer_scores_workspace_bytes", [ctypes.POINTER(StackC), _I64, ctypes.POINTER(_SZ)])
+_sig("mxs_layer_scores", [ctypes.POINTER(StackC), _P, _I64, _I64, _P, _P, _SZ, _P])
 _sig("mxs_attn_decode_workspace_bytes", [_I64, _I64, _I64, _I64, ctypes.POINTER(_SZ)])
 _sig("mxs_attn_decode", [_P, _I64, _I64, ctypes.POINTER(MXTensorC), ctypes.POINTER(MXTensorC), _I64, _I64,
                          ctypes.c_float, _P, _I64, _P, _SZ, _P])
@@ -92,7 +100,8 @@ EXPORTS = ["mxs_status_str", "mxs_launch_count", "mxs_sync", "mxs_layout_make", 
            "mxs_sensitivity_workspace_bytes", "mxs_sensitivity", "mxs_sensitivity_noalloc",
            "mxs_allocate_workspace_bytes",
            "mxs_allocate", "mxs_quantize_weight", "mxs_quantize_act", "mxs_dequantize",
-           "mxs_gemm_workspace_bytes", "mxs_gemm", "mxs_attn_decode_workspace_bytes", "mxs_attn_decode"]
+           "mxs_gemm_workspace_bytes", "mxs_gemm", "mxs_attn_decode_workspace_bytes", "mxs_attn_decode",
+           "mxs_layer_scores_workspace_bytes", "mxs_layer_scores"]
 
 
 def _check(st: int, where: str):
@@ -345,6 +354,53 @@ def mxs_attn_decode(q: torch.Tensor, K: MXTensor, V: MXTensor, T: int, n_kvh: in
     _check(_lib.mxs_attn_decode(q.data_ptr(), n_qh, _rowmajor(q), ctypes.byref(K.c), ctypes.byref(V.c), T, n_kvh,
                                 float(sm_scale), out.data_ptr(), _rowmajor(out), _aligned_ptr(ws, 256), need,
                                 _stream(stream)), "mxs_attn_decode")
+    return out
+
+
+# ---------------------------------------------------------- layer scores
+LINEARS = ("q", "k", "v", "o", "gate", "up", "down")
+
+
+def _stack_c(blocks, hidden, n_heads, n_kv_heads, mlp, rms_eps, rope_theta):
+    ptrs = (ctypes.c_void_p * (7 * len(blocks)))()
+    for b, Ws in enumerate(blocks):
+        for j, w in enumerate(Ws):
+            if w.dtype != torch.bfloat16 or not w.is_contiguous():
+                raise TypeError("stack weights must be contiguous bf16")
+            ptrs[7 * b + j] = w.data_ptr()
+    m = StackC(len(blocks), hidden, n_heads, n_kv_heads, mlp, rms_eps, rope_theta,
+               ctypes.cast(ptrs, ctypes.c_void_p))
+    return m, ptrs
+
+
+def mxs_layer_scores_workspace_bytes(n_blocks: int, hidden: int, n_heads: int, n_kv_heads: int, mlp: int,
+                                     T: int, rms_eps: float = 1e-5, rope_theta: float = 500000.0) -> int:
+    m = StackC(n_blocks, hidden, n_heads, n_kv_heads, mlp, rms_eps, rope_theta, ctypes.c_void_p(1 << 20))
+    need = _SZ(0)
+    _check(_lib.mxs_layer_scores_workspace_bytes(ctypes.byref(m), T, ctypes.byref(need)),
+           "mxs_layer_scores_workspace_bytes")
+    return need.value
+
+
+def mxs_layer_scores(x: torch.Tensor, blocks, *, n_heads: int, n_kv_heads: int, rms_eps: float = 1e-5,
+                     rope_theta: float = 500000.0, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Layer-wise sensitivity scores (7 per block: q, k, v, o, gate, up, down)
+    of the decoder stack `blocks` (a list of 7-tuples of bf16 weights) for the
+    fp32 hidden states x (T x hidden).  Synchronises the stream."""
+    import numpy as np
+    T, hidden = x.shape
+    mlp = blocks[0][4].shape[0]
+    m, ptrs = _stack_c(blocks, hidden, n_heads, n_kv_heads, mlp, rms_eps, rope_theta)
+    need = _SZ(0)
+    _check(_lib.mxs_layer_scores_workspace_bytes(ctypes.byref(m), T, ctypes.byref(need)),
+           "mxs_layer_scores_workspace_bytes")
+    ws = workspace if workspace is not None else _workspace(need.value, x.device)
+    out = np.zeros(7 * len(blocks))
+    if x.dtype != torch.float32:
+        raise TypeError("x must be fp32")
+    _check(_lib.mxs_layer_scores(ctypes.byref(m), x.data_ptr(), T, _rowmajor(x),
+                                 out.ctypes.data_as(ctypes.c_void_p), _aligned_ptr(ws, 256), need.value,
+                                 _stream(stream)), "mxs_layer_scores")
     return out
 
 

@@ -434,6 +434,11 @@ def run_gpu(args, rank, world, local_rank):
             "peak_basis": f"4-bit segment at 2x measured bf16 ({pk['fp8_tflops']:.0f} TFLOP/s, no measured fp8), "
                           f"6/8-bit at measured bf16 ({pk['bf16_tflops']:.0f}); of {pk['source']}"}
 
+    # HBM-bound calls with a working set below L2 also timed back to back on
+    # rotated input copies (more than twice the L2 between reuses)
+    for name, (us, frac) in run_stream(c, dev, path, torch, pk).items():
+        kernels[name]["us_stream"] = us
+        kernels[name]["frac_stream"] = frac
     e2e = run_e2e(path, args, dev, world)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -445,7 +450,10 @@ def run_gpu(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world} (no data-path collective)",
                    "timing": "step = one CUDA graph of all C-ABI calls, replayed per step between CUDA events; "
                              f"kernels{{}}: per call, (graph of {CALL_REPS} x [L2 flush, call]) - (graph of "
-                             f"{CALL_REPS} flushes), best of {CALL_TRIALS} replays each, / {CALL_REPS}; cold L2 per call",
+                             f"{CALL_REPS} flushes), best of {CALL_TRIALS} replays each, / {CALL_REPS}; cold L2 per call, "
+                             "launch gap included; us_stream/frac_stream (decode GEMMs, K/V quantiser, decode attention): "
+                             "a graph of back-to-back calls cycling through input copies with > 2x L2 read between "
+                             "reuses of a copy, best of 3 replays / calls",
                    "launches_per_step": launches_per_step},
         "roofline": roof, "kernels": kernels, "e2e": e2e, "gpu_launches": launches,
         "clocks": clocks.summary(), "wall_s_timed_region": wall,
@@ -454,6 +462,77 @@ def run_gpu(args, rank, world, local_rank):
         line["mixed_overhead"] = run_mixed_overhead(c, dev, path, torch)
         line["budget_sweep"] = run_budget_sweep(c, dev, path, torch, pk)
     return line
+
+
+L2_BYTES = 126 << 20
+
+
+def run_stream(c, dev, path, torch, pk, trials=3):
+    """Back-to-back time per call of the decode GEMMs, the K/V quantisers and
+    the decode attention: a CUDA graph of 2 x n calls cycling through n copies
+    of the call's large input, n chosen so more than twice the L2 of other
+    copies is read between two uses of one copy (every call reads its input
+    from HBM), replayed between CUDA events; best of `trials` / (2 n).  No L2
+    flush sits between the calls, so the launch gap the isolated per-call
+    timing pays is hidden by the programmatic launch chaining."""
+    out = {}
+
+    def measure(name, calls, unit_work, unit):
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        for fn in calls:
+            fn()
+        with torch.cuda.graph(g, stream=cap):
+            for _ in range(2):
+                for fn in calls:
+                    fn()
+        best = None
+        for _ in range(trials):
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record()
+            g.replay()
+            s1.record()
+            torch.cuda.synchronize()
+            t = s0.elapsed_time(s1) * 1e-3 / (2 * len(calls))
+            best = t if best is None else min(best, t)
+        return best
+
+    ncopy = lambda nbytes: max(2, -(-2 * L2_BYTES // max(nbytes, 1)) + 1)
+    for L in path.layers:
+        wbytes = layout_bytes(L.N, L.counts, 0)
+        copies = []
+        for _ in range(ncopy(wbytes)):
+            Wq = c.mxtensor_empty(L.N, L.lay, dev)
+            c.mxs_quantize_weight(L.W, Wq)
+            copies.append(Wq)
+        for M in L.Ms[1:]:                                   # the decode rows
+            calls = [lambda Wq=Wq, M=M: c.mxs_gemm(L.Aq[M], Wq, Y=L.Y[M], workspace=L.gemm_ws) for Wq in copies]
+            t = measure(f"{L.name}.mxs_gemm_M{M}", calls, None, None)
+            out[f"{L.name}.mxs_gemm_M{M}"] = (t * 1e6, gemm_roofline_s(M, L.N, L.counts, pk) / t)
+        del copies
+    T, H, D = KV_SHAPE
+    kv_bytes = path.KV[0].numel() * 2
+    srcs = [path.KV[0].clone() for _ in range(ncopy(kv_bytes))]
+    calls = [lambda x=x: c.mxs_quantize_act(x, path.KVq[0]) for x in srcs]
+    t = measure("kv.mxs_quantize_act_K", calls, None, None)
+    work = path.work["kv.mxs_quantize_act_K"][1]
+    out["kv.mxs_quantize_act_K"] = (t * 1e6, work / t / 1e9 / pk["hbm_gbs"])
+    del srcs
+    cache_bytes = 2 * layout_bytes(T * H, (0, 0, D), 0)
+    pairs = []
+    for _ in range(ncopy(cache_bytes)):
+        kq, vq = c.mxtensor_empty(T * H, path.kv_lay, dev), c.mxtensor_empty(T * H, path.kv_lay, dev)
+        c.mxs_quantize_act(path.KV[0], kq)
+        c.mxs_quantize_act(path.KV[1], vq)
+        pairs.append((kq, vq))
+    calls = [lambda kq=kq, vq=vq: c.mxs_attn_decode(path.q, kq, vq, T, H, path.sm_scale, out=path.attn_out,
+                                                    workspace=path.attn_ws) for kq, vq in pairs]
+    t = measure("kv.mxs_attn_decode", calls, None, None)
+    out["kv.mxs_attn_decode"] = (t * 1e6, path.work["kv.mxs_attn_decode"][1] / t / 1e9 / pk["hbm_gbs"])
+    del pairs
+    c.mxs_sync()
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_e2e(path, args, dev, world):

@@ -1046,6 +1046,54 @@ __global__ void __launch_bounds__(256) quant_contig_kernel(QuantArgs a) {
   }
 }
 
+// The K/V cache layout {0, 0, K} (one 4-bit segment, no permutation) on
+// bf16 rows of K % 32 == 0 values: one thread per 32-value block, its 64
+// source bytes read by two 32-byte loads, coded by encode_store_bf16's rule
+// and stored as one 16-byte code word and one scale byte.  Block i of the
+// tensor is row i / nb, block i % nb (a 32-bit multiply-high division); each
+// thread takes kKvU blocks, their loads issued together.
+constexpr int kKvU = 2;
+
+__device__ __forceinline__ void ld_stream_32B(const void *p, uint32_t (&w)[8]) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+               : "l"(p));
+}
+
+__global__ void __launch_bounds__(256) quant_kv4_kernel(QuantArgs a, uint32_t total) {
+  pdl_wait();
+  pdl_trigger();
+  const uint32_t nb = static_cast<uint32_t>(a.nb[2]);
+  const uint32_t stride = gridDim.x * blockDim.x;
+  const uint16_t *src = static_cast<const uint16_t *>(a.src);
+  for (uint32_t i0 = blockIdx.x * blockDim.x + threadIdx.x; i0 < total; i0 += kKvU * stride) {
+    uint32_t p[kKvU][16], row[kKvU], b[kKvU];
+#pragma unroll
+    for (int u = 0; u < kKvU; ++u) {
+      const uint32_t i = i0 + u * stride;
+      row[u] = nb > 1 ? __umulhi(i, a.nb_magic[2]) : i;
+      b[u] = i - row[u] * nb;
+      if (i < total) {
+        const uint16_t *blk = src + static_cast<int64_t>(row[u]) * a.ld + b[u] * kBlock;
+        uint32_t lo[8], hi[8];
+        ld_stream_32B(blk, lo);
+        ld_stream_32B(blk + 16, hi);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          p[u][t] = lo[t];
+          p[u][8 + t] = hi[t];
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kKvU; ++u) {
+      if (i0 + u * stride >= total) break;
+      encode_store_bf16<4>(p[u], a.codes[2] + static_cast<int64_t>(row[u]) * a.cpitch[2] + b[u] * 16,
+                           a.scales[2] + static_cast<int64_t>(row[u]) * a.spitch[2] + b[u]);
+    }
+  }
+}
+
 // One warp per (row, block), one lane per position.
 template <bool F32>
 __global__ void __launch_bounds__(256) quant_lane_kernel(QuantArgs a) {
@@ -1252,6 +1300,15 @@ static mxs_status quantize_impl(const void *src, mxs_dtype dt, int64_t rows, int
   const int nsm = sm_count();
   const int64_t warps = rows * a.nb_total;
   const bool tiny = warps <= 8192;                     // latency-bound: one warp per block
+  if (!tiny && !a.perm && !f32 && a.k_real[0] == 0 && a.k_real[1] == 0 && a.K % kBlock == 0 && aligned16(src) &&
+      (ld * 2) % 32 == 0 && (reinterpret_cast<uintptr_t>(src) & 31u) == 0 && warps < (1ll << 31) &&
+      (a.nb[2] <= 1 || warps * a.nb[2] < (1ll << 32))) {
+    // the K/V cache: one 4-bit segment, rows of whole blocks (32-byte aligned)
+    const int grid = static_cast<int>(std::min<int64_t>((warps + 256 * kKvU - 1) / (256 * kKvU), static_cast<int64_t>(nsm) * 8));
+    launch_pdl(quant_kv4_kernel, dim3(grid), dim3(256), 0, s, a, static_cast<uint32_t>(warps));
+    count_launch();
+    return cuda_status(cudaGetLastError());
+  }
   if (!tiny && !a.perm) {
     const int grid = static_cast<int>(std::min<int64_t>((warps + 255) / 256, static_cast<int64_t>(nsm) * 8));
     if (f32) launch_pdl(quant_contig_kernel<true>, dim3(grid), dim3(256), 0, s, a);

@@ -436,9 +436,10 @@ def run_gpu(args, rank, world, local_rank):
 
     # HBM-bound calls with a working set below L2 also timed back to back on
     # rotated input copies (more than twice the L2 between reuses)
-    for name, (us, frac) in run_stream(c, dev, path, torch, pk).items():
-        kernels[name]["us_stream"] = us
-        kernels[name]["frac_stream"] = frac
+    if not args.no_stream:
+        for name, (us, frac) in run_stream(c, dev, path, torch, pk).items():
+            kernels[name]["us_stream"] = us
+            kernels[name]["frac_stream"] = frac
     e2e = run_e2e(path, args, dev, world)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -451,7 +452,8 @@ def run_gpu(args, rank, world, local_rank):
                    "timing": "step = one CUDA graph of all C-ABI calls, replayed per step between CUDA events; "
                              f"kernels{{}}: per call, (graph of {CALL_REPS} x [L2 flush, call]) - (graph of "
                              f"{CALL_REPS} flushes), best of {CALL_TRIALS} replays each, / {CALL_REPS}; cold L2 per call, "
-                             "launch gap included; us_stream/frac_stream (decode GEMMs, K/V quantiser, decode attention): "
+                             "launch gap included; us_stream/frac_stream (decode GEMMs, quantisers, sensitivity, decode "
+                             "attention): "
                              "a graph of back-to-back calls cycling through input copies with > 2x L2 read between "
                              "reuses of a copy, best of 3 replays / calls",
                    "launches_per_step": launches_per_step},
@@ -468,8 +470,9 @@ L2_BYTES = 126 << 20
 
 
 def run_stream(c, dev, path, torch, pk, trials=3):
-    """Back-to-back time per call of the decode GEMMs, the K/V quantisers and
-    the decode attention: a CUDA graph of 2 x n calls cycling through n copies
+    """Back-to-back time per call of the HBM-bound calls (decode GEMMs, K/V
+    quantiser, decode attention, each layer's weight and prefill activation
+    quantisers and sensitivity): a CUDA graph of 2 x n calls cycling through n copies
     of the call's large input, n chosen so more than twice the L2 of other
     copies is read between two uses of one copy (every call reads its input
     from HBM), replayed between CUDA events; best of `trials` / (2 n).  No L2
@@ -530,6 +533,22 @@ def run_stream(c, dev, path, torch, pk, trials=3):
     t = measure("kv.mxs_attn_decode", calls, None, None)
     out["kv.mxs_attn_decode"] = (t * 1e6, path.work["kv.mxs_attn_decode"][1] / t / 1e9 / pk["hbm_gbs"])
     del pairs
+    # the per-layer quantisers and the sensitivity on rotated source copies
+    hbm = lambda name, t: (t * 1e6, path.work[name][1] / t / 1e9 / pk["hbm_gbs"])
+    for L in path.layers:
+        Wc = [L.W] + [L.W.clone() for _ in range(ncopy(L.W.numel() * 2) - 1)]
+        name = f"{L.name}.mxs_quantize_weight"
+        out[name] = hbm(name, measure(name, [lambda w=w: c.mxs_quantize_weight(w, L.Wq) for w in Wc], None, None))
+        M = L.Ms[0]
+        Ac = [L.A[M]] + [L.A[M].clone() for _ in range(ncopy(L.A[M].numel() * 2) - 1)]
+        name = f"{L.name}.mxs_quantize_act_M{M}"
+        out[name] = hbm(name, measure(name, [lambda x=x: c.mxs_quantize_act(x, L.Aq[M]) for x in Ac], None, None))
+        Xc = [L.X] + [L.X.clone() for _ in range(ncopy(L.X.numel() * 2 + L.W.numel() * 2) - 1)]
+        name = f"{L.name}.mxs_sensitivity"
+        calls = [lambda x=x, w=w: c.mxs_sensitivity(x, w, workspace=L.sens_ws, out=(L.H, L.E, L.s))
+                 for x, w in zip(Xc, (Wc * len(Xc))[:len(Xc)])]
+        out[name] = hbm(name, measure(name, calls, None, None))
+        del Wc, Ac, Xc
     c.mxs_sync()
     torch.cuda.empty_cache()
     return out
@@ -833,6 +852,7 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the mixed-overhead table and the budget sweep")
+    ap.add_argument("--no-stream", action="store_true", help="skip the back-to-back per-call timing")
     ap.add_argument("--probe-ranks", action="store_true", help="launch check: join the process group and exit")
     args = ap.parse_args()
     if args.warmup < 3:

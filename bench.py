@@ -295,16 +295,17 @@ def job_tflops(flops_per_rank_step: float, steps: int, world: int, job_s: float)
     return world * flops_per_rank_step * steps / job_s / 1e12
 
 
-def traffic_from_profile(pk_name: str, per_units: float = 1.0):
-    """dram bytes per launch recorded in profiles/, if the GEMM source is
-    unchanged since the capture; scaled by `per_units` (units of the bench
-    launch per unit of the captured one) when the capture was a smaller case."""
+def traffic_from_profile(pk_name: str, layer: str, per_units: float = 1.0):
+    """dram bytes of one call of `layer`'s GEMM recorded in profiles/ (a line
+    `dram_bytes_per_call[layer]: B`), if the GEMM source is unchanged since the
+    capture; scaled by `per_units` (units of the bench launch per unit of the
+    captured one) when the capture was a smaller case."""
     prof = os.path.join(ROOT, "profiles", pk_name)
     try:
         text = open(prof).read()
     except OSError:
         return None
-    m = re.search(r"dram_bytes_per_call:\s*([0-9.eE+]+)", text)
+    m = re.search(r"dram_bytes_per_call\[" + re.escape(layer) + r"\]:\s*([0-9.eE+]+)", text)
     h = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
     if not m or not h:
         return None
@@ -430,7 +431,7 @@ def run_gpu(args, rank, world, local_rank):
     roof = {"kernel": f"{dom} (one call: gemm_stage_kernel + gemm_tc2_kernel), M={M} N={N} K={K}",
             "bound": "tensor", "achieved": g["achieved"], "peak": 2 * M * N * K / rt / 1e12, "unit": "TFLOP/s",
             "frac": g["frac"],
-            "traffic": traffic_from_profile("gemm_mlp_prefill_M8192.md") if dom.startswith("mlp_up") else None,
+            "traffic": traffic_from_profile("gemm_mlp_prefill_M8192.md", dom.split(".")[0]) if dom.endswith("M8192") else None,
             "peak_basis": f"4-bit segment at 2x measured bf16 ({pk['fp8_tflops']:.0f} TFLOP/s, no measured fp8), "
                           f"6/8-bit at measured bf16 ({pk['bf16_tflops']:.0f}); of {pk['source']}"}
 

@@ -135,6 +135,17 @@ int64_t mxs_launch_count(void);
  * last call, MXS_ERR_CUDA if the stream reported an error, else MXS_OK. */
 mxs_status mxs_sync(void *stream);
 
+/* Diagnostic: sets, on the current device, how many SM clock cycles a
+ * pipeline wait of the prefill GEMM's tensor-core kernels (the mxs_gemm
+ * calls whose workspace size is non-zero) may spin before the kernel gives up: it records MXS_ERR_TIMEOUT
+ * in the status word, stops issuing, lets the copies and MMAs it already
+ * issued finish (waits bounded by the default limit), frees its tensor
+ * memory and returns; its output is then unspecified.  cycles <= 0 restores
+ * the default (4e9 cycles, about 2 s); larger values are clamped to it.
+ * Synchronous; applies to GEMM launches made after it returns.  Lets a test
+ * make a wait run out without a fault.  Errors: MXS_ERR_CUDA. */
+mxs_status mxs_set_wait_limit(int64_t cycles);
+
 /* Fills *out for K columns with counts = {n8, n6, n4} (host, summing to K)
  * and perm (device, K entries; NULL for the identity, e.g. the K/V cache
  * layout {0, 0, K}).  No device access; perm is stored, not read. */

@@ -78,6 +78,7 @@ def _sig(name, args, res=_ST):
 _sig("mxs_status_str", [_ST], ctypes.c_char_p)
 _sig("mxs_launch_count", [], _I64)
 _sig("mxs_sync", [_P])
+_sig("mxs_set_wait_limit", [_I64])
 _sig("mxs_layout_make", [_I64, _P, _P, ctypes.POINTER(LayoutC)])
 _sig("mxs_mxtensor_bytes", [_I64, ctypes.POINTER(LayoutC), _P, _P, _P, _P])
 _sig("mxs_sensitivity_workspace_bytes", [_I64, _I64, _I64, ctypes.POINTER(_SZ)])
@@ -96,7 +97,7 @@ _sig("mxs_attn_decode_workspace_bytes", [_I64, _I64, _I64, _I64, ctypes.POINTER(
 _sig("mxs_attn_decode", [_P, _I64, _I64, ctypes.POINTER(MXTensorC), ctypes.POINTER(MXTensorC), _I64, _I64,
                          ctypes.c_float, _P, _I64, _P, _SZ, _P])
 
-EXPORTS = ["mxs_status_str", "mxs_launch_count", "mxs_sync", "mxs_layout_make", "mxs_mxtensor_bytes",
+EXPORTS = ["mxs_status_str", "mxs_launch_count", "mxs_sync", "mxs_set_wait_limit", "mxs_layout_make", "mxs_mxtensor_bytes",
            "mxs_sensitivity_workspace_bytes", "mxs_sensitivity", "mxs_sensitivity_noalloc",
            "mxs_allocate_workspace_bytes",
            "mxs_allocate", "mxs_quantize_weight", "mxs_quantize_act", "mxs_dequantize",
@@ -406,6 +407,12 @@ def mxs_layer_scores(x: torch.Tensor, blocks, *, n_heads: int, n_kv_heads: int, 
 
 def mxs_sync(stream=None) -> None:
     _check(_lib.mxs_sync(_stream(stream)), "mxs_sync")
+
+
+def mxs_set_wait_limit(cycles: int) -> None:
+    """Diagnostic: the spin limit (SM cycles) of the prefill GEMM kernels'
+    pipeline waits on the current device; 0 restores the default."""
+    _check(_lib.mxs_set_wait_limit(int(cycles)), "mxs_set_wait_limit")
 
 
 def mxs_launch_count() -> int:

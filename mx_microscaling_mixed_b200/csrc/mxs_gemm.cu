@@ -62,6 +62,9 @@ constexpr int kSfSlots = 4;
 constexpr int kSfSlotCols = 12;
 constexpr int kGemmThreads = 192;
 constexpr long long kWaitLimit = 4000000000LL;   // cycles (~2 s): then give up
+// Limit of the pipeline waits of the two tensor-core kernels (mxs_set_wait_limit
+// lowers it for a diagnostic run).  The drains on the way out keep kWaitLimit.
+__device__ long long g_wait_limit = kWaitLimit;
 
 // kind::f16: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9 = 1), B bf16 (bits
 // 10-12 = 1), both K-major, N>>3 at bit 17, M>>4 at bit 24.
@@ -78,7 +81,8 @@ struct GemmSmem {
   static constexpr int sfa_off = b_off + kStages * kBBytes;
   static constexpr int sfb_off = sfa_off + kStages * kSfaBytes;
   static constexpr int bar_off = sfb_off + kStages * kSfbBytes;
-  static constexpr int bytes = bar_off + (2 * kStages + 1) * 8 + 16;
+  // full[S], empty[S], accum_full, drain; tmem slot, abort flag
+  static constexpr int bytes = bar_off + (2 * kStages + 2) * 8 + 16;
 };
 constexpr int kGemmSmemBytes = GemmSmem::bytes + 1024;   // + alignment slack
 
@@ -94,11 +98,11 @@ struct GemmArgs {
 
 __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
+  const long long t0 = clock64(), limit = g_wait_limit;
   for (;;) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitLimit) {
+    if (clock64() - t0 > limit) {
       *abort_flag = 1;
       atomicExch(&g_status, static_cast<int>(MXS_ERR_TIMEOUT));
       return false;
@@ -117,7 +121,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + GemmSmem::bar_off);
   uint64_t *empty = full + kStages;
   uint64_t *accum_full = empty + kStages;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum_full + 1);
+  uint64_t *drain = accum_full + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -130,6 +135,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       ptx::mbar_init(&empty[s], 1);
     }
     ptx::mbar_init(accum_full, 1);
+    ptx::mbar_init(drain, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -141,12 +147,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  int issued = 0;                                    // stages whose copies the producer issued
 
   if (warp == 0) {
     if (lane == 0) {
       for (int it = 0; it < n_iters; ++it) {
         const int s = it % kStages;
         if (it >= kStages && !wait_bounded(&empty[s], ((it / kStages) - 1) & 1, abort_flag)) break;
+        issued = it + 1;
         uint8_t *sa = smem + GemmSmem::a_off + s * kABytes;
         uint8_t *sb = smem + GemmSmem::b_off + s * kBBytes;
         if (it < g.n16_stages) {
@@ -233,6 +241,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   ptx::tc_fence_before();
   __syncthreads();
+  if (*abort_flag) {
+    // Given up: the copies already issued land and the MMAs already issued
+    // finish before the CTA frees its tensor memory and leaves (each wait
+    // bounded by the full limit).
+    if (warp == 0 && lane == 0)
+      for (int i = max(0, issued - kStages); i < issued; ++i)
+        ptx::mbar_wait_cycles(&full[i % kStages], (i / kStages) & 1, kWaitLimit);
+    if (warp == 1 && lane == 0) {
+      ptx::mma_commit(drain);
+      ptx::mbar_wait_cycles(drain, 0, kWaitLimit);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+  }
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
@@ -268,6 +290,16 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
+}
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+// lowers the barrier's pending transaction count by `bytes` without a copy
+__device__ __forceinline__ void mbar_complete_tx(uint64_t *b, uint32_t bytes) {
+  asm volatile("mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(b)), "r"(bytes)
+               : "memory");
 }
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
@@ -357,8 +389,9 @@ struct P2Smem {
   static constexpr int sfa_off = b_off + kP2Stages * kP2Sub * kP2TileBytes;
   static constexpr int sfb_off = sfa_off + kP2Stages * kP2Sub * kP2SfaBytes;
   static constexpr int bar_off = sfb_off + kP2Stages * kP2Sub * kP2SfbBytes;
-  // full[S], empty[S], acc_full[2], acc_empty[2], tmem slot, abort flag
-  static constexpr int bar_end = bar_off + (2 * kP2Stages + 4) * 8 + 16;
+  // full[S], empty[S], acc_full[2], acc_empty[2], drain; tmem slot, abort
+  // flag, issued-stage count
+  static constexpr int bar_end = bar_off + (2 * kP2Stages + 5) * 8 + 16;
   // per epilogue warp: a 32-row x 40-column bf16 piece of Y on its way out by TMA
   static constexpr int epi_off = (bar_end + 127) / 128 * 128;
   static constexpr int epi_bytes = 32 * kP2EpiCols * 2;
@@ -389,8 +422,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
   uint64_t *empty = full + kP2Stages;
   uint64_t *acc_full = empty + kP2Stages;             // [2]: one per accumulator buffer
   uint64_t *acc_empty = acc_full + 2;                 // [2]
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+  uint64_t *drain = acc_empty + 2;                    // the MMAs issued have finished
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  int *issued_slot = reinterpret_cast<int *>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = ptx::cluster_rank();
@@ -409,6 +444,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
       ptx::mbar_init(&acc_full[b], 1);
       ptx::mbar_init(&acc_empty[b], 2 * kP2EpiWarps);
     }
+    ptx::mbar_init(drain, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -426,12 +462,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
   const uint32_t tmem = *tmem_slot;
   // the staged operands and Y belong to earlier kernels in the stream
   pdl_wait();
+  // bytes of one K slice, both CTAs
+  constexpr uint32_t bytes16 = 2 * (kP2TileBytes + kP2BRows * kSliceBytes);
+  constexpr uint32_t bytes8 = 2 * (kP2TileBytes + kP2BRows * kSliceBytes + kP2SfaBytes + kP2SfbBytes);
+  int it = 0;                                         // producer: stages whose copies were issued
 
   if (warp == 0) {
     if (lane == 0) {
-      const uint32_t bytes16 = 2 * (kP2TileBytes + kP2BRows * kSliceBytes);           // per slice, both CTAs
-      const uint32_t bytes8 = 2 * (kP2TileBytes + kP2BRows * kSliceBytes + kP2SfaBytes + kP2SfbBytes);
-      int it = 0;
       for (int t = pair; t < n_tiles_total && !*abort_flag; t += npairs) {
         const int mt = t / g.n_tiles, nt = t - mt * g.n_tiles;
         const int am = mt * 256 + static_cast<int>(rank) * kP2Rows;      // this CTA's A rows
@@ -602,6 +639,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
 
   // the tensor stores of Y are complete before the CTA leaves
   if (warp >= 2 && lane == 0) ptx::bulk_wait_all();
+  if (warp == 0 && lane == 0) *issued_slot = it;
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();
+  // Neither CTA issues a copy or an MMA past this point.  Before either
+  // leaves, everything issued lands: the leader's commit arrives on both
+  // CTAs' drain barriers once every MMA (and scale copy) has finished, and
+  // the leader settles the pair's outstanding stages on its full barriers.
+  // Stage i was issued by both producers, by one, or by none; only the last
+  // kP2Stages stages can be outstanding (a producer issues stage i after the
+  // MMAs consumed stage i - kP2Stages, which needed both halves).  Where one
+  // half was never issued, the leader supplies its arrival and byte count
+  // itself, so the phase completes when the other half lands.  On a normal
+  // exit every stage is complete and each wait returns at once.
+  if (warp == 1 && lane == 0) {
+    if (leader) ptx::mma2_commit_both(drain);
+    ptx::mbar_wait_cycles(drain, 0, kWaitLimit);
+  }
+  if (leader && warp == 0 && lane == 0) {
+    const int L = it;
+    const int P = static_cast<int>(ptx::ld_cluster_u32(ptx::map_to_rank(ptx::smem_addr(issued_slot), 1)));
+    const int hi = max(L, P);
+    for (int i = max(0, hi - kP2Stages); i < hi; ++i) {
+      const int s = i % kP2Stages, k = i % n_iters;
+      const bool wide = k < n16s;
+      const int j0 = kP2Sub * (wide ? k : k - n16s);
+      const int nsub = min(kP2Sub, (wide ? g.n16_stages : g.n8_stages) - j0);
+      const uint32_t half = static_cast<uint32_t>(nsub) * ((wide ? bytes16 : bytes8) / 2);
+      if (i < L && i >= P) {
+        ptx::mbar_complete_tx(&full[s], half);
+      } else if (i >= L && i < P) {
+        ptx::mbar_arrive_expect_tx(&full[s], 2 * half);
+        ptx::mbar_complete_tx(&full[s], half);
+      }
+      ptx::mbar_wait_cycles(&full[s], (i / kP2Stages) & 1, kWaitLimit);
+    }
+  }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::cluster_sync();
@@ -988,6 +1062,11 @@ extern "C" mxs_status mxs_sync(void *stream) {
     return static_cast<mxs_status>(st);
   }
   return MXS_OK;
+}
+
+extern "C" mxs_status mxs_set_wait_limit(int64_t cycles) {
+  const long long v = cycles <= 0 ? kWaitLimit : std::min<long long>(cycles, kWaitLimit);
+  return cudaMemcpyToSymbol(g_wait_limit, &v, sizeof(v)) == cudaSuccess ? MXS_OK : MXS_ERR_CUDA;
 }
 
 extern "C" mxs_status mxs_gemm_workspace_bytes(const mxs_mxtensor *A, const mxs_mxtensor *W, size_t *bytes) {

@@ -11,6 +11,9 @@ import oracle
 
 GEMM_TOL = 2e-3          # relative error budget of mxs_gemm beyond the bf16 output rounding
 GEMM_FLOOR = 1e-2        # relative-error denominator floor, as a fraction of max|Yref|
+# normwise bound: the arithmetic budget plus the bf16 output rounding (8
+# significant bits: at most 2^-8 of the unrounded value's magnitude)
+GEMM_NORMWISE_TOL = GEMM_TOL + 2.0 ** -8 * (1.0 + GEMM_TOL)
 
 
 def need_gpu():
@@ -67,12 +70,12 @@ def gemm_rel_error(Y: np.ndarray, Yref: np.ndarray) -> float:
     return float(np.max(excess / den))
 
 
-def gemm_plain_rel_error(Y: np.ndarray, Yref: np.ndarray) -> float:
-    """max |Y - Yref| / max(|Yref|, 1% max|Yref|), output rounding included."""
+def gemm_normwise_error(Y: np.ndarray, Yref: np.ndarray) -> float:
+    """Normwise error max|Y - Yref| / max|Yref|, output rounding included
+    (0 when both are all zero)."""
     ymax = float(np.max(np.abs(Yref))) if Yref.size else 0.0
-    if ymax == 0.0:
-        return float(np.max(np.abs(Y))) if Y.size else 0.0
-    return float(np.max(np.abs(Y - Yref) / np.maximum(np.abs(Yref), GEMM_FLOOR * ymax)))
+    diff = float(np.max(np.abs(Y - Yref))) if Y.size else 0.0
+    return diff / ymax if ymax > 0.0 else diff
 
 
 def quantize_both(c, src: torch.Tensor, layout, perm_np, counts, weight: bool):

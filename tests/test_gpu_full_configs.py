@@ -64,8 +64,10 @@ def _gemm_sampled(c, A, W, counts, seed, rows, cols):
     wc, ws = _check_rows(Wq, W, cols, perm, counts, "weights")
     Yref = oracle.gemm(ac, as_, wc, ws, counts)
     Yg = Y[torch.from_numpy(rows).cuda()][:, torch.from_numpy(cols).cuda()].float().cpu().numpy().astype(np.float64)
-    err = parity.gemm_rel_error(Yg, Yref)
+    err, nw = parity.gemm_rel_error(Yg, Yref), parity.gemm_normwise_error(Yg, Yref)
+    print(f"sampled {len(rows)} x {len(cols)}: max rel err {err:.3e}, normwise {nw:.3e}")
     assert err <= parity.GEMM_TOL, f"max rel err {err:.3e}"
+    assert nw <= parity.GEMM_NORMWISE_TOL, f"normwise {nw:.3e}"
 
 
 def test_mlp_gate_up_prefill_M8192(c):
@@ -74,6 +76,14 @@ def test_mlp_gate_up_prefill_M8192(c):
     A = inputs.gaussian_acts("cuda", seed=5001, rows=8192, K=K)
     W = inputs.attn_weight("cuda", seed=5000, N=14336, K=K)
     _gemm_sampled(c, A, W, _counts(K, 4.5), seed=11, rows=_sample(8192, 40, 1), cols=_sample(14336, 40, 2))
+
+
+def test_mlp_down_prefill_M8192(c):
+    """Down projection W 4096 x 14336 at M = 8192: the longest call of the
+    layer step (2-CTA tcgen05 path, K = 14336)."""
+    d = inputs.mlp_down_layer("cuda", seed=3000, M=8192)
+    _gemm_sampled(c, d["A"], d["W"], _counts(14336, 4.5), seed=12, rows=_sample(8192, 40, 5),
+                  cols=_sample(4096, 40, 6))
 
 
 def test_mlp_down_prefill_M2048(c):

@@ -64,8 +64,10 @@ def test_gemm_matches_oracle(c, M, N, K, counts):
     A = inputs.random_matrix(M, K, device="cuda", seed=M + K, dtype=torch.bfloat16)
     W = inputs.random_matrix(N, K, device="cuda", seed=N + 2 * K, dtype=torch.bfloat16, std=0.02)
     Y, Yref = _run(c, A, W, counts, seed=K)
-    err = parity.gemm_rel_error(Y, Yref)
+    err, nw = parity.gemm_rel_error(Y, Yref), parity.gemm_normwise_error(Y, Yref)
+    print(f"M={M} N={N} K={K}: max rel err {err:.3e}, normwise {nw:.3e}")
     assert err <= parity.GEMM_TOL, f"max rel err {err:.3e}"
+    assert nw <= parity.GEMM_NORMWISE_TOL, f"normwise {nw:.3e}"
 
 
 def test_parity_layer_fp32_inputs(c):
@@ -159,8 +161,10 @@ def test_gemm_small_m_matches_oracle(c, M, N, K, counts):
     A = inputs.random_matrix(M, K, device="cuda", seed=3 * M + K, dtype=torch.bfloat16)
     W = inputs.random_matrix(N, K, device="cuda", seed=N + K, dtype=torch.bfloat16, std=0.02)
     Y, Yref = _run(c, A, W, counts, seed=M)
-    err = parity.gemm_rel_error(Y, Yref)
+    err, nw = parity.gemm_rel_error(Y, Yref), parity.gemm_normwise_error(Y, Yref)
+    print(f"M={M} N={N} K={K}: max rel err {err:.3e}, normwise {nw:.3e}")
     assert err <= parity.GEMM_TOL, f"max rel err {err:.3e}"
+    assert nw <= parity.GEMM_NORMWISE_TOL, f"normwise {nw:.3e}"
 
 
 def test_gemm_small_m_extreme_codes(c):
@@ -188,5 +192,7 @@ def test_gemm_pair_kernel_matches_oracle(c, M, N, K, counts):
     A = inputs.random_matrix(M, K, device="cuda", seed=M + 5 * K, dtype=torch.bfloat16)
     W = inputs.random_matrix(N, K, device="cuda", seed=N + 7 * K, dtype=torch.bfloat16, std=0.02)
     Y, Yref = _run(c, A, W, counts, seed=M + N)
-    err = parity.gemm_rel_error(Y, Yref)
+    err, nw = parity.gemm_rel_error(Y, Yref), parity.gemm_normwise_error(Y, Yref)
+    print(f"M={M} N={N} K={K}: max rel err {err:.3e}, normwise {nw:.3e}")
     assert err <= parity.GEMM_TOL, f"max rel err {err:.3e}"
+    assert nw <= parity.GEMM_NORMWISE_TOL, f"normwise {nw:.3e}"

@@ -143,3 +143,9 @@ def test_bf16_tolerance_metric():
     assert np.all(np.abs(rounded - x) <= hu)
     assert parity.gemm_rel_error(np.array([256.0]), np.array([257.0])) == 0.0
     assert parity.gemm_rel_error(np.array([254.0]), np.array([257.0])) > 0.0
+    # normwise: one element off by 1 against a max of 4 -> 1/4; rounding of
+    # the exact result alone stays within the normwise budget
+    assert parity.gemm_normwise_error(np.array([1.0, 4.0]), np.array([2.0, -4.0])) == 2.0
+    assert parity.gemm_normwise_error(np.array([1.0, 3.0]), np.array([2.0, 4.0])) == 0.25
+    assert parity.gemm_normwise_error(rounded, x) <= parity.GEMM_NORMWISE_TOL
+    assert parity.gemm_normwise_error(np.zeros(3), np.zeros(3)) == 0.0

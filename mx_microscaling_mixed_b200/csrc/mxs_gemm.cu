@@ -369,7 +369,7 @@ constexpr int kP2N = 240;                          // output columns per pair ti
 constexpr int kP2BRows = kP2N / 2;                 // rows of B per CTA per stage
 constexpr int kP2AccCols = kP2N;                   // one accumulator buffer; two buffers at columns 0 and 240
 constexpr int kP2SfCol = 2 * kP2AccCols;           // scale slots from column 480: 2 x 12 columns
-constexpr int kP2SfSlots = kP2Sub;                 // one scale slot per slice of a stage
+constexpr int kP2SfSlots = 2;                      // scale slots, taken by slices in turn
 static_assert(kP2SfCol + kP2SfSlots * kSfSlotCols <= kTmemCols, "accumulators and scale slots fit in TMEM");
 constexpr int kP2TileBytes = kP2Rows * kSliceBytes;
 constexpr int kP2SfaBytes = kSfChunk;              // own 128 A rows x 4 blocks
@@ -398,6 +398,20 @@ struct P2Smem {
   static constexpr int bytes = epi_off + kP2EpiWarps * epi_bytes;
 };
 constexpr int kP2SmemBytes = P2Smem::bytes + 1024;
+
+// Output tile t -> (mt, nt).  Tiles run through a group of kP2Raster
+// m-tiles for one n-tile before moving to the next n-tile, so the ~74 tiles
+// in flight at a time (one per pair) share about 8 m-tiles of A and 10
+// n-tiles of W, which stay in L2 while the group is worked on: A is read
+// from DRAM about once, W once per group.
+constexpr int kP2Raster = 8;
+__device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int &mt, int &nt) {
+  const int grp = t / (kP2Raster * n_tiles);
+  const int rem = t - grp * (kP2Raster * n_tiles);
+  const int gm = min(kP2Raster, m_tiles - grp * kP2Raster);     // m-tiles of this group
+  nt = rem / gm;
+  mt = grp * kP2Raster + (rem - nt * gm);
+}
 
 struct P2Args {
   int32_t M, N;
@@ -470,7 +484,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
   if (warp == 0) {
     if (lane == 0) {
       for (int t = pair; t < n_tiles_total && !*abort_flag; t += npairs) {
-        const int mt = t / g.n_tiles, nt = t - mt * g.n_tiles;
+        int mt, nt;
+        tile_coords(t, g.m_tiles, g.n_tiles, mt, nt);
         const int am = mt * 256 + static_cast<int>(rank) * kP2Rows;      // this CTA's A rows
         const int bn = nt * kP2N + static_cast<int>(rank) * kP2BRows;    // this CTA's B rows
         for (int k = 0; k < n_iters; ++k, ++it) {
@@ -521,14 +536,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
           const int j0 = kP2Sub * (wide ? k : k - n16s);
           const int nsub = min(kP2Sub, (wide ? g.n16_stages : g.n8_stages) - j0);
           if (!wide) {
-            // the stage's scale chunks first (one slot per slice), so the
-            // copies for a later slice are queued ahead of the earlier
-            // slice's MMAs; slots are reused only by later stages, behind
-            // these MMAs in the same issue order
+            // the stage's scale chunks first (slices take the slots in
+            // turn), so the copies for a later slice are queued ahead of
+            // the earlier slice's MMAs; a slot is reused only by a later
+            // slice, behind these MMAs in the same issue order
             for (int h = 0; h < nsub; ++h) {
               const uint32_t sfa_s = ptx::smem_addr(smem + P2Smem::sfa_off + (s * kP2Sub + h) * kP2SfaBytes);
               const uint32_t sfb_s = ptx::smem_addr(smem + P2Smem::sfb_off + (s * kP2Sub + h) * kP2SfbBytes);
-              const uint32_t slot = kSfSlotCols * static_cast<uint32_t>(h);
+              const uint32_t slot = kSfSlotCols * static_cast<uint32_t>((it * kP2Sub + h) % kP2SfSlots);
               ptx::copy_sf_to_tmem2(tsfa + slot, ptx::desc_sf(sfa_s));
               ptx::copy_sf_to_tmem2(tsfb + slot, ptx::desc_sf(sfb_s));
               ptx::copy_sf_to_tmem2(tsfb + slot + 4, ptx::desc_sf(sfb_s + kSfChunk));
@@ -543,7 +558,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
                 ptx::mma2_bf16(acc, ptx::desc_sw128(a_base + 32 * q), ptx::desc_sw128(b_base + 32 * q), kIdesc2Bf16,
                                (k > 0 || h > 0 || q > 0) ? 1u : 0u);
             } else {
-              const uint32_t slot = kSfSlotCols * static_cast<uint32_t>(h);
+              const uint32_t slot = kSfSlotCols * static_cast<uint32_t>((it * kP2Sub + h) % kP2SfSlots);
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 const uint32_t idesc = kIdesc2Mxf8 | (static_cast<uint32_t>(q) << 4) | (static_cast<uint32_t>(q) << 29);
@@ -577,7 +592,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&acc_empty[buf]), 0));
-      const int mt = t / g.n_tiles, nt = t - mt * g.n_tiles;
+      int mt, nt;
+      tile_coords(t, g.m_tiles, g.n_tiles, mt, nt);
       const int row0 = mt * 256 + static_cast<int>(rank) * kP2Rows + q * 32;
       if (g.y_tma) {
         // three 32 x 40 pieces per warp: bf16 rows into the warp's staging

@@ -484,7 +484,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quant_tile_kernel(QuantArgs 
                        &bar[st]);
     __syncwarp();
     if (lane == 0)
-      for (int st = 0; st < kQStages; ++st) issued[st] = st;
+      for (int st = 0; st < kQStages; ++st) issued[st] = st < nloc ? st : -1;   // -1: never copied into
   }
   // gather table: 8 permutation loads in flight per thread
   for (int g = 0; g < 3; ++g) {

@@ -58,6 +58,13 @@ WORKLOAD = ("llama3-8b layer: attention projection W 4096x4096 (M 2048/16/1), ML
             "down W 4096x14336 (M 8192/16/1), bf16, calib X 2048 rows, budget 4.5 bits each; K/V cache "
             "8192x8x128 bf16 x2 to MXINT4 + one decode-attention step (32 query heads)")
 SWEEP_BUDGETS = ((7, 2), (129, 32), (17, 4), (9, 2), (5, 1), (23, 4))     # 3.5 ... 5.75 average bits
+# Llama-2-70B-shaped stack: 80 layers of these linears (N, K), N(0, 0.015^2)
+# weights with 2% of the columns x20, 4.25 bits each, all quantised in place
+L70_SHAPES = (("q", 8192, 8192), ("k", 1024, 8192), ("v", 1024, 8192), ("o", 8192, 8192),
+              ("gate", 28672, 8192), ("up", 28672, 8192), ("down", 8192, 28672))
+L70_LAYERS = 80
+L70_BUDGET = (17, 4)
+L70_SEED = 5000                    # matrix j of layer l: seed L70_SEED + 16 l + j
 
 
 def peaks():
@@ -68,10 +75,38 @@ def peaks():
         p["source"] = "measured"
     except (OSError, KeyError, ValueError):
         pass
-    # No measured FP8 figure: the block-scaled E4M3 peak is taken as 2x bf16
-    # (the nominal dense ratio, 4.5 vs 2.25 PFLOP/s).
+    # Until measured on the device (measure_fp8_tflops), the E4M3 peak is
+    # taken as 2x bf16 (the nominal dense ratio, 4.5 vs 2.25 PFLOP/s).
     p["fp8_tflops"] = 2.0 * p["bf16_tflops"]
+    p["fp8_source"] = "2x measured bf16 (no fp8 measurement)"
     return p
+
+
+def measure_fp8_tflops(torch, dev, n=8192, reps=20):
+    """Dense E4M3 GEMM rate of this GPU, measured the way the bf16 peak was:
+    a library GEMM of two n x n E4M3 matrices (torch._scaled_mm, tensorwise
+    unit scales, bf16 out), median of `reps` back-to-back calls after
+    warm-up.  None if the library call is unavailable."""
+    try:
+        a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+        one = torch.ones((), device=dev)
+        f = lambda: torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        for _ in range(3):
+            f()
+        ev = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            ev.append((e0, e1))
+        torch.cuda.synchronize()
+        ms = statistics.median(x.elapsed_time(y) for x, y in ev)
+        del a, b
+        return 2.0 * n ** 3 / (ms * 1e-3) / 1e12
+    except (RuntimeError, AttributeError, TypeError):
+        return None
 
 
 def layout_bytes(rows, counts, in_bytes):
@@ -335,6 +370,10 @@ def run_gpu(args, rank, world, local_rank):
     from mx_microscaling_mixed_b200 import capi as c
     path = Path(dev, SEED + 97 * rank)
     pk = peaks()
+    fp8 = measure_fp8_tflops(torch, dev)
+    if fp8:
+        pk["fp8_tflops"] = fp8
+        pk["fp8_source"] = "measured on this GPU: torch._scaled_mm E4M3 8192^3, median of 20"
     for _ in range(args.warmup):
         path.flush.zero_()
         for _, fn in path.calls():
@@ -432,7 +471,7 @@ def run_gpu(args, rank, world, local_rank):
             "bound": "tensor", "achieved": g["achieved"], "peak": 2 * M * N * K / rt / 1e12, "unit": "TFLOP/s",
             "frac": g["frac"],
             "traffic": traffic_from_profile("gemm_mlp_prefill_M8192.md", dom.split(".")[0]) if dom.endswith("M8192") else None,
-            "peak_basis": f"4-bit segment at 2x measured bf16 ({pk['fp8_tflops']:.0f} TFLOP/s, no measured fp8), "
+            "peak_basis": f"4-bit segment at the E4M3 peak ({pk['fp8_tflops']:.0f} TFLOP/s, {pk['fp8_source']}), "
                           f"6/8-bit at measured bf16 ({pk['bf16_tflops']:.0f}); of {pk['source']}"}
 
     # HBM-bound calls with a working set below L2 also timed back to back on
@@ -464,6 +503,7 @@ def run_gpu(args, rank, world, local_rank):
     if not args.no_extras:
         line["mixed_overhead"] = run_mixed_overhead(c, dev, path, torch)
         line["budget_sweep"] = run_budget_sweep(c, dev, path, torch, pk)
+        line["stack70b_inplace"] = run_70b_inplace(c, dev, path, torch, pk)
     return line
 
 
@@ -637,6 +677,115 @@ def _time_call(torch, call, flush, reps):
         ev.append((e0, e1))
     torch.cuda.synchronize()
     return statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
+
+
+def l70_weight(inputs, torch, dev, layer, j):
+    _, N, K = L70_SHAPES[j]
+    return inputs.random_matrix(N, K, device=dev, seed=L70_SEED + 16 * layer + j, dtype=torch.bfloat16,
+                                std=0.015, outlier_frac=0.02, outlier_scale=20.0)
+
+
+def run_70b_inplace(c, dev, path, torch, pk, reps=5):
+    """The Llama-2-70B-shaped stack, all 80 layers' weights quantised in place:
+    each matrix is generated on the device in bf16, its sensitivity taken on
+    a 2048-row calibration X of its input width, its columns allocated at
+    4.25 bits and the weight quantised into storage that stays resident,
+    then the bf16 is freed.  Reports the per-call sensitivity and
+    quantisation times summed over the 560 matrices, the packed bytes held,
+    the prefill GEMM of layer 0's gate projection at M = 4096 (L2 flushed)
+    and one decode step over the whole stack: per matrix a one-row
+    activation quantisation and the M = 1 GEMM, 1120 launches in one CUDA
+    graph, reading every packed weight once."""
+    from mx_microscaling_mixed_b200 import inputs
+    X = {K: inputs.gaussian_acts(dev, L70_SEED - 1 - i, T_CAL, K) for i, K in enumerate((8192, 28672))}
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    store, marks = [], []
+    wbytes = sbytes = 0
+    for layer in range(L70_LAYERS):
+        for j, (name, N, K) in enumerate(L70_SHAPES):
+            W = l70_weight(inputs, torch, dev, layer, j)
+            e = [ev() for _ in range(3)]
+            e[0].record()
+            _, _, s = c.mxs_sensitivity(X[K], W)
+            e[1].record()
+            perms, counts = c.mxs_allocate([s], [N], mode="budget", budget=L70_BUDGET)
+            lay = c.mxs_layout_make(K, counts[0], perms[0])
+            Wq = c.mxtensor_empty(N, lay, dev)
+            e2 = ev()
+            e2.record()
+            c.mxs_quantize_weight(W, Wq)
+            e[2].record()
+            marks.append((e[0], e[1], e2, e[2], N, K, tuple(counts[0])))
+            store.append((name, N, K, lay, Wq, tuple(counts[0])))
+            wbytes += layout_bytes(N, counts[0], 0)
+            del W, s
+    torch.cuda.synchronize()
+    sens_ms = sum(a.elapsed_time(b) for a, b, _, _, _, _, _ in marks)
+    quant_ms = sum(x.elapsed_time(y) for _, _, x, y, _, _, _ in marks)
+    q_bytes = sum(layout_bytes(N, cnt, 2) for _, _, _, _, N, _, cnt in marks)
+    s_bytes = sum(T_CAL * K * 2 + N * K * 2 for _, _, _, _, N, K, _ in marks)
+    del X
+    out = {"layers": L70_LAYERS, "matrices": len(store), "budget_bits": L70_BUDGET[0] / L70_BUDGET[1],
+           "counts_n8_n6_n4": {f"K={K}": list(cnt) for _, _, K, _, _, cnt in store[:7]},
+           "weights": sum(N * K for _, N, K, _, _, _ in store), "packed_bytes": wbytes,
+           "device_bytes_peak": torch.cuda.max_memory_allocated(dev),
+           "sensitivity_ms_total": sens_ms, "sensitivity_gbs": s_bytes / (sens_ms * 1e-3) / 1e9,
+           "quantize_weight_ms_total": quant_ms, "quantize_weight_gbs": q_bytes / (quant_ms * 1e-3) / 1e9,
+           "quantize_weight_frac_hbm": q_bytes / (quant_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+           "timing": "calls in stream order with CUDA events around each, summed over the 560 matrices"}
+    per = {}
+    for (x0, x1, y0, y1, N, K, cnt), (name, *_rest) in zip(marks, store):
+        d = per.setdefault(name, [0.0, 0.0, 0])
+        d[0] += y0.elapsed_time(y1)
+        d[1] += layout_bytes(N, cnt, 2)
+        d[2] += 1
+    out["quantize_weight_by_matrix"] = {n: {"ms": ms, "gbs": b / (ms * 1e-3) / 1e9,
+                                            "frac_hbm": b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+                                        for n, (ms, b, _) in per.items()}
+    # prefill: layer 0's gate projection at M = 4096
+    _, N, K, lay, Wq, cnt = store[4]
+    M = 4096
+    Aq = c.mxtensor_empty(M, lay, dev)
+    c.mxs_quantize_act(inputs.gaussian_acts(dev, L70_SEED - 3, M, K), Aq)
+    ws = torch.empty(c.mxs_gemm_workspace_bytes(Aq, Wq) + 1024, dtype=torch.uint8, device=dev)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    us = _time_call(torch, lambda: c.mxs_gemm(Aq, Wq, Y=Y, workspace=ws), path.flush, reps)
+    out["gemm_gate_M4096"] = {"us": us, "tflops": 2 * M * N * K / us / 1e6,
+                              "frac": gemm_roofline_s(M, N, cnt, pk) / (us * 1e-6)}
+    del Aq, ws, Y
+    # decode: every matrix once, one activation row each
+    a1 = {K: inputs.gaussian_acts(dev, L70_SEED - 5 - i, 1, K) for i, K in enumerate((8192, 28672))}
+    calls = []
+    for _, N, K, lay, Wq, _ in store:
+        Aq = c.mxtensor_empty(1, lay, dev)
+        Y = torch.empty(1, N, dtype=torch.bfloat16, device=dev)
+        calls.append((a1[K], Aq, Wq, Y))
+
+    def step():
+        for x, Aq, Wq, Y in calls:
+            c.mxs_quantize_act(x, Aq)
+            c.mxs_gemm(Aq, Wq, Y=Y)
+    step()
+    c.mxs_sync()
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    with torch.cuda.graph(g, stream=cap):
+        step()
+    times = []
+    for _ in range(reps):
+        e0, e1 = ev(), ev()
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    out["decode_step_M1"] = {"ms": ms, "launches": 2 * len(calls), "w_bytes": wbytes,
+                             "gbs": wbytes / (ms * 1e-3) / 1e9, "frac_hbm": wbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+    del g, calls, store
+    c.mxs_sync()
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_mixed_overhead(c, dev, path, torch, reps=30):

@@ -394,17 +394,47 @@ __device__ __forceinline__ void issue_batch(const QuantArgs &a, int64_t batch, u
   for (int rr = lane; rr < nr; rr += 32) ptx::bulk_load(buf + rr * srow_bytes, src + rr * a.ld * ES, row_bytes, bar);
 }
 
+// Byte offsets in a staged row of positions 4j .. 4j+3 of block b of segment
+// g: from the gather table in shared memory (TAB), else from the permutation
+// itself (rows too wide for the table beside the staging buffers; the
+// permutation stays in L2).  Positions past the segment's real columns read
+// the zero slot at column K.
+template <bool TAB, int ES>
+__device__ __forceinline__ uint4 gather4(const QuantArgs &a, int g, int b, const uint32_t *tab, int j) {
+  if constexpr (TAB) {
+    return reinterpret_cast<const uint4 *>(tab + (a.boff[g] + b) * kTabWordsPerBlock)[j];
+  } else {
+    const int p0 = kBlock * b + 4 * j;
+    if (a.perm && p0 + 3 < a.k_real[g]) {
+      const int32_t *src = a.perm + a.real_off[g] + p0;
+      if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
+        const int4 v = __ldg(reinterpret_cast<const int4 *>(src));    // four real columns, one load
+        return make_uint4(static_cast<uint32_t>(v.x * ES), static_cast<uint32_t>(v.y * ES),
+                          static_cast<uint32_t>(v.z * ES), static_cast<uint32_t>(v.w * ES));
+      }
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int p = p0 + u;
+      const int col = p < a.k_real[g] ? (a.perm ? __ldg(a.perm + a.real_off[g] + p) : a.real_off[g] + p) : a.K;
+      o[u] = static_cast<uint32_t>(col * ES);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
 // One lane's item of a work unit: gathers block b of segment g (width M) of
-// staged row `srow` through the table and codes it into row `row`.
-template <int M, bool F32>
+// staged row `srow` and codes it into row `row`.
+template <int M, bool F32, bool TAB>
 __device__ __forceinline__ void code_item(const QuantArgs &a, int g, int b, const uint32_t *tab, const uint8_t *srow,
                                           int64_t row) {
-  const uint4 *tw = reinterpret_cast<const uint4 *>(tab + (a.boff[g] + b) * kTabWordsPerBlock);
+  constexpr int ES = F32 ? 4 : 2;
   if constexpr (!F32 && M != 8) {
     uint32_t p[kBlock / 2];
 #pragma unroll
     for (int j = 0; j < kBlock / 4; ++j) {
-      const uint4 w = tw[j];
+      const uint4 w = gather4<TAB, ES>(a, g, b, tab, j);
       p[2 * j] = static_cast<uint32_t>(*reinterpret_cast<const unsigned short *>(srow + w.x)) |
                  (static_cast<uint32_t>(*reinterpret_cast<const unsigned short *>(srow + w.y)) << 16);
       p[2 * j + 1] = static_cast<uint32_t>(*reinterpret_cast<const unsigned short *>(srow + w.z)) |
@@ -415,7 +445,7 @@ __device__ __forceinline__ void code_item(const QuantArgs &a, int g, int b, cons
     float v[kBlock];
 #pragma unroll
     for (int j = 0; j < kBlock / 4; ++j) {
-      const uint4 w = tw[j];
+      const uint4 w = gather4<TAB, ES>(a, g, b, tab, j);
       v[4 * j] = staged_elem<F32>(srow, w.x);
       v[4 * j + 1] = staged_elem<F32>(srow, w.y);
       v[4 * j + 2] = staged_elem<F32>(srow, w.z);
@@ -447,15 +477,16 @@ __device__ __forceinline__ bool spin_until_equal(volatile int *p, int want, long
 // the zero slots.  Loop (per warp): take the next unit, wait until its batch
 // has been issued and has landed, code it, and count it done; the warp that
 // completes a batch refills that buffer with the batch kQStages ahead.
-template <bool F32>
+template <bool F32, bool TAB>
 __global__ void __launch_bounds__(kQuantThreads, 1) quant_tile_kernel(QuantArgs a, int *status) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int ES = F32 ? 4 : 2;
   uint32_t *tab = reinterpret_cast<uint32_t *>(smem);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + quant_table_bytes(a.nb_total));
-  uint8_t *bufs = smem + quant_table_bytes(a.nb_total) + 128;
+  const int64_t tab_bytes = TAB ? quant_table_bytes(a.nb_total) : 0;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + tab_bytes);
+  uint8_t *bufs = smem + tab_bytes + 128;
   __shared__ int next_unit, abort_flag;
   __shared__ int done_cnt[kQStages];
   __shared__ int issued[kQStages];
@@ -487,7 +518,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quant_tile_kernel(QuantArgs 
       for (int st = 0; st < kQStages; ++st) issued[st] = st < nloc ? st : -1;   // -1: never copied into
   }
   // gather table: 8 permutation loads in flight per thread
-  for (int g = 0; g < 3; ++g) {
+  for (int g = 0; TAB && g < 3; ++g) {
     const int n = a.nb[g] * kBlock;
     for (int p0 = threadIdx.x; p0 < n; p0 += 8 * kQuantThreads) {
       int col[8];
@@ -546,9 +577,9 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quant_tile_kernel(QuantArgs 
     const int b = q * (32 >> a.lg) + (lane >> a.lg);
     if (r0 + rl < a.rows && b < a.nb[g]) {
       const uint8_t *srow = bufs + st * buf_bytes + rl * srow_bytes;
-      if (g == 0) code_item<8, F32>(a, 0, b, tab, srow, r0 + rl);
-      else if (g == 1) code_item<6, F32>(a, 1, b, tab, srow, r0 + rl);
-      else code_item<4, F32>(a, 2, b, tab, srow, r0 + rl);
+      if (g == 0) code_item<8, F32, TAB>(a, 0, b, tab, srow, r0 + rl);
+      else if (g == 1) code_item<6, F32, TAB>(a, 1, b, tab, srow, r0 + rl);
+      else code_item<4, F32, TAB>(a, 2, b, tab, srow, r0 + rl);
     }
     __syncwarp();
     int last = 0;
@@ -1352,14 +1383,22 @@ static mxs_status quantize_impl(const void *src, mxs_dtype dt, int64_t rows, int
     }
   }
   bool tiled = !tiny && vec_rows;
+  bool tab = true;            // gather table in shared memory, else offsets from the permutation
   int64_t smem = 0;
   int grid = 0;
   if (tiled) {
     // pitch: room for the zero slot, 16 bytes mod 128
     const int64_t pitch = round_up((a.K + 1) * es, 128) + 16;
     a.row_stride = static_cast<int32_t>(pitch / es);
-    const int64_t fixed = quant_table_bytes(a.nb_total) + 128;
-    const int64_t rows_fit = std::min<int64_t>(256, (kQuantSmemBudget - fixed) / kQStages / pitch);
+    int64_t fixed = quant_table_bytes(a.nb_total) + 128;
+    int64_t rows_fit = std::min<int64_t>(256, (kQuantSmemBudget - fixed) / kQStages / pitch);
+    if (rows_fit < 1) {
+      // rows too wide for the table beside three row buffers (K above about
+      // 20 K for bf16): stage the rows alone and read the permutation from L2
+      tab = false;
+      fixed = 128;
+      rows_fit = std::min<int64_t>(256, (kQuantSmemBudget - fixed) / kQStages / pitch);
+    }
     tiled = rows_fit >= 1;
     if (tiled) {
       a.lg = rows_fit >= 8 ? 3 : rows_fit >= 4 ? 2 : rows_fit >= 2 ? 1 : 0;
@@ -1382,13 +1421,14 @@ static mxs_status quantize_impl(const void *src, mxs_dtype dt, int64_t rows, int
   if (tiled) {
     int *status = device_status_word();
     if (!status) return MXS_ERR_CUDA;
-    if (f32) {
-      if (!ensure_smem(quant_tile_kernel<true>, static_cast<int>(smem))) return MXS_ERR_CUDA;
-      launch_pdl(quant_tile_kernel<true>, dim3(grid), dim3(kQuantThreads), smem, s, a, status);
-    } else {
-      if (!ensure_smem(quant_tile_kernel<false>, static_cast<int>(smem))) return MXS_ERR_CUDA;
-      launch_pdl(quant_tile_kernel<false>, dim3(grid), dim3(kQuantThreads), smem, s, a, status);
-    }
+    auto go = [&](auto kernel) -> mxs_status {
+      if (!ensure_smem(kernel, static_cast<int>(smem))) return MXS_ERR_CUDA;
+      launch_pdl(kernel, dim3(grid), dim3(kQuantThreads), smem, s, a, status);
+      return MXS_OK;
+    };
+    const mxs_status st = f32 ? (tab ? go(quant_tile_kernel<true, true>) : go(quant_tile_kernel<true, false>))
+                              : (tab ? go(quant_tile_kernel<false, true>) : go(quant_tile_kernel<false, false>));
+    if (st != MXS_OK) return st;
   } else {
     const int lgrid = static_cast<int>(std::min<int64_t>((warps + 7) / 8, static_cast<int64_t>(nsm) * 16));
     if (f32) launch_pdl(quant_lane_kernel<true>, dim3(lgrid), dim3(256), 0, s, a);

@@ -104,6 +104,18 @@ def test_strided_rows_staged(c):
     parity.assert_codes_equal(t, oc, os_, "strided staged")
 
 
+@pytest.mark.parametrize("rows,K,counts,weight", [
+    (300, 24008, (32, 5000, 18976), True),      # bf16 rows too wide for the gather table: offsets from the permutation
+    (37, 28672, (32, 3520, 25120), False),      # the 70B down-projection width, a ragged row count
+    (64, 24008, (7, 1001, 23000), True),        # segment starts off the 16-byte grid: single-entry loads
+])
+def test_wide_rows_table_free(c, rows, K, counts, weight):
+    src = inputs.random_matrix(rows, K, device="cuda", seed=K + rows, dtype=torch.bfloat16)
+    lay, perm, counts = _random_layout(c, K, seed=rows, counts=counts)
+    t, oc, os_ = parity.quantize_both(c, src, lay, perm, counts, weight=weight)
+    parity.assert_codes_equal(t, oc, os_, f"{rows} x {K} bf16")
+
+
 def test_strided_rows(c):
     wide = inputs.random_matrix(20, 300, device="cuda", seed=3, dtype=torch.bfloat16)
     src = wide[:, :257]                      # pitch 300 elements, K = 257

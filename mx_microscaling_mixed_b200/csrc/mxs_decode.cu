@@ -526,10 +526,17 @@ mxs_status gemm_small(const mxs_mxtensor *A, const mxs_mxtensor *W, void *Y, int
       int dev = 0, nsm = 148;
       cudaGetDevice(&dev);
       cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+      if (!ensure_smem(gemm_gemv_kernel, static_cast<int>(std::max<int64_t>(gsmem, 16)))) return MXS_ERR_CUDA;
+      // one resident wave: every CTA widens the activations once, then its
+      // warps take W rows until none are left
+      int occ = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gemm_gemv_kernel, kGvThreads,
+                                                        static_cast<size_t>(std::max<int64_t>(gsmem, 16))) != cudaSuccess ||
+          occ < 1)
+        occ = 1;
       const int rows_per_cta = kGvThreads / 32;
       const int grid = static_cast<int>(std::min<int64_t>((a.N + rows_per_cta - 1) / rows_per_cta,
-                                                          static_cast<int64_t>(nsm) * 64));
-      if (!ensure_smem(gemm_gemv_kernel, static_cast<int>(std::max<int64_t>(gsmem, 16)))) return MXS_ERR_CUDA;
+                                                          static_cast<int64_t>(nsm) * occ));
       launch_pdl(gemm_gemv_kernel, dim3(grid), dim3(kGvThreads), static_cast<size_t>(std::max<int64_t>(gsmem, 16)), cs, a);
       count_launch();
       return cuda_status(cudaGetLastError());

@@ -52,7 +52,7 @@ constexpr int kAttnD = 128;               // head dimension served
 constexpr int kAttnWarps = 8;
 constexpr int kAttnThreads = kAttnWarps * 32;
 constexpr int kAttnMaxRep = 8;            // query heads per kv head: one n-tile of 8
-constexpr int kAttnTargetCtas = 296;      // two CTAs per SM of a 148-SM part
+constexpr int kAttnTargetCtas = 256;      // splits of 256 tokens: 16 token tiles, 2 per warp
 constexpr int kAttnMinChunk = 64;
 constexpr int kAttnMaxChunk = 256;        // a TMA box holds at most 256 rows
 constexpr int kRowBytes = kAttnD / 2;     // packed codes of one cache row

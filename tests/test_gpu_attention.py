@@ -11,7 +11,7 @@ products in fp32 (|error| <= 128 * 2^-24 * sum|q k| * sm_scale, about
 6e-5 at the workload's scale, which moves a weight by that relative amount);
 exp2 is within 2^-22; the weights enter the output product with 16
 significant bits (2^-17); the output sums at most 256 tokens per split and
-37 splits in fp32 (< 2e-5).  Together below 1.5e-4 of max|V|; the test
+32 splits in fp32 (< 2e-5).  Together below 1.5e-4 of max|V|; the test
 allows 5e-4 (1e-3 for the sharpened softmax, whose scores are 4x larger).
 """
 import math

@@ -65,6 +65,12 @@ L70_SHAPES = (("q", 8192, 8192), ("k", 1024, 8192), ("v", 1024, 8192), ("o", 819
 L70_LAYERS = 80
 L70_BUDGET = (17, 4)
 L70_SEED = 5000                    # matrix j of layer l: seed L70_SEED + 16 l + j
+# Llama-3-8B-shaped stack: 32 layers of these linears, the attention weight
+# recipe, one 4.5-bit budget over all 224 matrices
+L8_SHAPES = (("q", 4096, 4096), ("k", 1024, 4096), ("v", 1024, 4096), ("o", 4096, 4096),
+             ("gate", 14336, 4096), ("up", 14336, 4096), ("down", 4096, 14336))
+L8_LAYERS = 32
+L8_SEED = 4000
 
 
 def peaks():
@@ -504,6 +510,7 @@ def run_gpu(args, rank, world, local_rank):
         line["mixed_overhead"] = run_mixed_overhead(c, dev, path, torch)
         line["budget_sweep"] = run_budget_sweep(c, dev, path, torch, pk)
         line["stack70b_inplace"] = run_70b_inplace(c, dev, path, torch, pk)
+        line["stack8b_global"] = run_8b_stack(c, dev, torch, pk)
     return line
 
 
@@ -683,6 +690,66 @@ def l70_weight(inputs, torch, dev, layer, j):
     _, N, K = L70_SHAPES[j]
     return inputs.random_matrix(N, K, device=dev, seed=L70_SEED + 16 * layer + j, dtype=torch.bfloat16,
                                 std=0.015, outlier_frac=0.02, outlier_scale=20.0)
+
+
+def run_8b_stack(c, dev, torch, pk):
+    """The Llama-3-8B-shaped stack under one budget: the sensitivities of all
+    224 matrices (each generated on the device, scored on a 2048-row X of its
+    input width, freed), one mxs_allocate call whose greedy spans the whole
+    stack at 4.5 bits, then every matrix generated again from its seed and
+    quantised into resident storage.  Reports the three phases' times (CUDA
+    events around each call, summed; the allocation's host arithmetic and its
+    one synchronisation included), the bits achieved and the bytes held."""
+    from mx_microscaling_mixed_b200 import inputs
+    X = {K: inputs.gaussian_acts(dev, L8_SEED - 1 - i, T_CAL, K) for i, K in enumerate((4096, 14336))}
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    mats = [(l, j, N, K) for l in range(L8_LAYERS) for j, (_, N, K) in enumerate(L8_SHAPES)]
+    gen = lambda l, j, N, K: inputs.attn_weight(dev, L8_SEED + 16 * l + j, N, K)
+    ss, marks = [], []
+    for l, j, N, K in mats:
+        W = gen(l, j, N, K)
+        e0, e1 = ev(), ev()
+        e0.record()
+        _, _, s = c.mxs_sensitivity(X[K], W)
+        e1.record()
+        ss.append(s)
+        marks.append((e0, e1))
+        del W
+    torch.cuda.synchronize()
+    sens_ms = sum(a.elapsed_time(b) for a, b in marks)
+    t0 = time.perf_counter()
+    perms, counts = c.mxs_allocate(ss, [N for _, _, N, _ in mats], mode="budget", budget=BUDGET)
+    torch.cuda.synchronize()
+    alloc_ms = (time.perf_counter() - t0) * 1e3
+    del ss
+    store, qmarks = [], []
+    for (l, j, N, K), perm, cnt in zip(mats, perms, counts):
+        W = gen(l, j, N, K)
+        Wq = c.mxtensor_empty(N, c.mxs_layout_make(K, cnt, perm), dev)
+        e0, e1 = ev(), ev()
+        e0.record()
+        c.mxs_quantize_weight(W, Wq)
+        e1.record()
+        store.append(Wq)
+        qmarks.append((e0, e1, N, tuple(cnt)))
+        del W
+    torch.cuda.synchronize()
+    quant_ms = sum(a.elapsed_time(b) for a, b, _, _ in qmarks)
+    q_bytes = sum(layout_bytes(N, cnt, 2) for _, _, N, cnt in qmarks)
+    bits = sum(N * (8 * n8 + 6 * n6 + 4 * n4) for (_, _, N, _), (n8, n6, n4) in zip(mats, counts))
+    elems = sum(N * K for _, _, N, K in mats)
+    out = {"layers": L8_LAYERS, "matrices": len(mats), "weights": elems,
+           "budget_bits": BUDGET[0] / BUDGET[1], "achieved_bits": bits / elems,
+           "packed_bytes": sum(layout_bytes(N, cnt, 0) for _, _, N, cnt in qmarks),
+           "sensitivity_ms_total": sens_ms,
+           "sensitivity_gbs": sum(T_CAL * K * 2 + N * K * 2 for _, _, N, K in mats) / (sens_ms * 1e-3) / 1e9,
+           "allocate_ms": alloc_ms, "quantize_weight_ms_total": quant_ms,
+           "quantize_weight_gbs": q_bytes / (quant_ms * 1e-3) / 1e9,
+           "quantize_weight_frac_hbm": q_bytes / (quant_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+           "counts_layer0_n8_n6_n4": {name: list(counts[j]) for j, (name, _, _) in enumerate(L8_SHAPES)}}
+    del store, X
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_70b_inplace(c, dev, path, torch, pk, reps=5):

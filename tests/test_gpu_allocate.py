@@ -76,6 +76,27 @@ def test_large_k(c):
     _cmp(gp, gc, op, oc)
 
 
+def test_large_k_ties(c):
+    """Long rows with heavy ties: four distinct values, -0.0 among the zeros
+    (equal to +0.0, so the two must tie and fall back to the column index),
+    the 8/6/4 boundaries inside tie groups; one layer in fractions mode and two
+    in the multi-layer budget greedy (whose group gains follow the rank
+    order)."""
+    rng = np.random.default_rng(21)
+    s_np = rng.integers(0, 4, 16384).astype(np.float64)
+    s_np[rng.random(16384) < 0.1] = -0.0
+    s_np[s_np == 0] = np.where(rng.random(int((s_np == 0).sum())) < 0.5, 0.0, -0.0)
+    s = torch.from_numpy(s_np).cuda()
+    gp, gc = c.mxs_allocate([s], [100], mode="fractions", p8=(7, 100), p6=(31, 100))
+    op, oc = oracle.allocate([s_np], [100], mode="fractions", p8=(7, 100), p6=(31, 100))
+    _cmp(gp, gc, op, oc)
+    t_np = np.round(rng.random(9000) * 50) / 8                       # 401 distinct values
+    s2 = [s, torch.from_numpy(t_np).cuda()]
+    gp, gc = c.mxs_allocate(s2, [300, 500], mode="budget", budget=(19, 4))
+    op, oc = oracle.allocate([s_np, t_np], [300, 500], mode="budget", budget=(19, 4))
+    _cmp(gp, gc, op, oc)
+
+
 def test_infeasible_budget(c):
     s = torch.ones(64, dtype=torch.float64, device="cuda")
     with pytest.raises(c.MxsError) as e:

@@ -152,6 +152,10 @@ SMALL_M = [
     (8, 130, 1000, (40, 200, 760)),
     (11, 64, 14336, (32, 3520, 10784)),
     (16, 96, 14336, (32, 3520, 10784)),
+    # K = 14336 with 9 activation rows: CTA pairs share the activation rows
+    # (rank 1 holds one), 7 W-row tiles so the pair grid has one CTA past N
+    (9, 100, 14336, (32, 3520, 10784)),
+    (16, 40, 28672, (32, 3520, 25120)),    # the 70B down projection's width
     (17, 300, 640, (32, 96, 512)),
 ]
 

@@ -34,8 +34,8 @@ namespace mxs {
 // needs is in flight at once; every lane then builds, per block, its A and
 // B fragments from the shared copies, widening only the two 4-code groups a
 // fragment holds.  When the W rows do not fit beside the activations, their
-// codes stream from global memory instead (no L1 allocation, several blocks
-// in flight).  The warps' partial sums are added in shared memory in warp
+// codes stream from global memory instead (through L1, several blocks in
+// flight).  The warps' partial sums are added in shared memory in warp
 // order.  Calls whose packed activation rows do not fit in shared memory
 // take the tensor-core path.
 struct SmallArgs {
@@ -84,14 +84,12 @@ __device__ __forceinline__ void mma_s8_16x8x32(const uint4 &a, uint32_t b0, uint
       : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1), "r"(0), "r"(0), "r"(0), "r"(0));
 }
 
-__device__ __forceinline__ uint32_t ld_stream_u16(const uint8_t *p) {
-  unsigned short v;
-  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
-  return v;
-}
+// A W word read from global memory through L1: the four lanes of a block
+// row and the warps on neighbouring blocks share its 32-byte sectors, which
+// L1 then serves once instead of L2 four times.
 __device__ __forceinline__ uint32_t ld_stream_u32(const uint8_t *p) {
   uint32_t v;
-  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
   return v;
 }
 
@@ -99,46 +97,47 @@ __device__ __forceinline__ uint32_t ld_stream_u32(const uint8_t *p) {
 // and how many blocks a warp keeps in flight.
 template <int G> struct DecSeg;
 template <> struct DecSeg<0> { static constexpr int kRaw = 2, kU = 4; };   // 8-bit: words t, 4+t
-template <> struct DecSeg<1> { static constexpr int kRaw = 4, kU = 4; };   // 6-bit: two word pairs
-template <> struct DecSeg<2> { static constexpr int kRaw = 2, kU = 8; };   // 4-bit: two 16-bit groups
+template <> struct DecSeg<1> { static constexpr int kRaw = 2, kU = 4; };   // 6-bit: one word pair, codes 8t..8t+7
+template <> struct DecSeg<2> { static constexpr int kRaw = 1, kU = 8; };   // 4-bit: one word, codes 8t..8t+7
 
-__device__ __forceinline__ uint32_t lds_u16(const uint8_t *p) { return *reinterpret_cast<const unsigned short *>(p); }
 __device__ __forceinline__ uint32_t lds_u32(const uint8_t *p) { return *reinterpret_cast<const uint32_t *>(p); }
 
 // The words of block c (packed, m-bit) that lane-in-group t needs for its
-// fragment: code groups t and 4+t (codes 4t..4t+3 and 16+4t..16+4t+3).
+// fragment: code groups t and 4+t (codes 4t..4t+3 and 16+4t..16+4t+3) for
+// 8-bit blocks; for 6- and 4-bit blocks, codes 8t..8t+7 (one word pair, one
+// word), which fill the same fragment slots in another order.  A and W take
+// the same order, so every code still meets its partner and the integer dot
+// product is unchanged.
 // SMEM: c points into shared memory (activations), else into global memory
 // (W, streaming loads).
 template <int G, bool SMEM>
 __device__ __forceinline__ void load_frag_raw(const uint8_t *c, int t, uint32_t (&r)[DecSeg<G>::kRaw]) {
   if constexpr (G == 2) {
-    r[0] = SMEM ? lds_u16(c + 2 * t) : ld_stream_u16(c + 2 * t);
-    r[1] = SMEM ? lds_u16(c + 8 + 2 * t) : ld_stream_u16(c + 8 + 2 * t);
+    r[0] = SMEM ? lds_u32(c + 4 * t) : ld_stream_u32(c + 4 * t);
   } else if constexpr (G == 0) {
     r[0] = SMEM ? lds_u32(c + 4 * t) : ld_stream_u32(c + 4 * t);
     r[1] = SMEM ? lds_u32(c + 16 + 4 * t) : ld_stream_u32(c + 16 + 4 * t);
   } else {
-    // group t: bytes 3t..3t+2, inside words (3t)/4 and (3t+2)/4
-    const int w0 = 4 * ((3 * t) >> 2), w1 = 4 * ((3 * t + 2) >> 2);
+    // codes 8t..8t+7: bytes 6t..6t+5, inside the two words from 4 floor(6t/4)
+    const int w0 = (6 * t) & ~3;
     r[0] = SMEM ? lds_u32(c + w0) : ld_stream_u32(c + w0);
-    r[1] = SMEM ? lds_u32(c + w1) : ld_stream_u32(c + w1);
-    r[2] = SMEM ? lds_u32(c + 12 + w0) : ld_stream_u32(c + 12 + w0);
-    r[3] = SMEM ? lds_u32(c + 12 + w1) : ld_stream_u32(c + 12 + w1);
+    r[1] = SMEM ? lds_u32(c + w0 + 4) : ld_stream_u32(c + w0 + 4);
   }
 }
 
 template <int G>
 __device__ __forceinline__ void widen_frag(const uint32_t (&r)[DecSeg<G>::kRaw], int t, uint32_t &b0, uint32_t &b1) {
   if constexpr (G == 2) {
-    b0 = widen4(r[0]);
-    b1 = widen4(r[1]);
+    b0 = widen4(r[0] & 0xFFFFu);            // slots 4t..4t+3: codes 8t..8t+3
+    b1 = widen4(r[0] >> 16);                // slots 16+4t..16+4t+3: codes 8t+4..8t+7
   } else if constexpr (G == 0) {
     b0 = r[0];
     b1 = r[1];
   } else {
-    const int sh = (3 * t & 3) * 8;
-    b0 = widen6(__funnelshift_r(r[0], r[1], sh));
-    b1 = widen6(__funnelshift_r(r[2], r[3], sh));
+    // the 48 bits of codes 8t..8t+7 start 0 or 16 bits into the pair
+    const uint64_t v = ((static_cast<uint64_t>(r[1]) << 32) | r[0]) >> ((6 * t & 3) * 8);
+    b0 = widen6(static_cast<uint32_t>(v));          // slots 4t..: codes 8t..8t+3 (low 24 bits)
+    b1 = widen6(static_cast<uint32_t>(v >> 24));    // slots 16+4t..: codes 8t+4..8t+7
   }
 }
 

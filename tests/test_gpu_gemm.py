@@ -150,10 +150,11 @@ SMALL_M = [
     (3, 37, 96, (0, 32, 64)),
     (5, 260, 512, (32, 96, 384)),
     (8, 130, 1000, (40, 200, 760)),
+    (12, 300, 4096, (32, 960, 3104)),      # the attention layer's width, W staged beside A
     (11, 64, 14336, (32, 3520, 10784)),
     (16, 96, 14336, (32, 3520, 10784)),
-    # K = 14336 with 9 activation rows: CTA pairs share the activation rows
-    # (rank 1 holds one), 7 W-row tiles so the pair grid has one CTA past N
+    # K = 14336 with 9 activation rows over 7 W-row tiles (the last ragged):
+    # W streams from global memory beside the staged activations
     (9, 100, 14336, (32, 3520, 10784)),
     (16, 40, 28672, (32, 3520, 25120)),    # the 70B down projection's width
     (17, 300, 640, (32, 96, 512)),
@@ -171,10 +172,12 @@ def test_gemm_small_m_matches_oracle(c, M, N, K, counts):
     assert nw <= parity.GEMM_NORMWISE_TOL, f"normwise {nw:.3e}"
 
 
-def test_gemm_small_m_extreme_codes(c):
-    # blocks at the clamp (all codes +-(2^(m-1)-1)) in every segment
+@pytest.mark.parametrize("M", [4, 16])
+def test_gemm_small_m_extreme_codes(c, M):
+    # blocks at the clamp (all codes +-(2^(m-1)-1)) in every segment, through
+    # the GEMV (M = 4) and the integer-MMA kernel (M = 16)
     K = 256
-    A = torch.full((4, K), 1.96875, dtype=torch.bfloat16, device="cuda")
+    A = torch.full((M, K), 1.96875, dtype=torch.bfloat16, device="cuda")
     A[:, 1::2] = -1.96875
     W = torch.full((40, K), -1.96875, dtype=torch.bfloat16, device="cuda")
     Y, Yref = _run(c, A, W, (64, 64, 128), seed=9)

@@ -1084,6 +1084,7 @@ __global__ void __launch_bounds__(256) quant_contig_kernel(QuantArgs a) {
 // tensor is row i / nb, block i % nb (a 32-bit multiply-high division); each
 // thread takes kKvU blocks, their loads issued together.
 constexpr int kKvU = 2;
+constexpr int kKvThreads = 128;
 
 __device__ __forceinline__ void ld_stream_32B(const void *p, uint32_t (&w)[8]) {
   asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
@@ -1091,7 +1092,7 @@ __device__ __forceinline__ void ld_stream_32B(const void *p, uint32_t (&w)[8]) {
                : "l"(p));
 }
 
-__global__ void __launch_bounds__(256) quant_kv4_kernel(QuantArgs a, uint32_t total) {
+__global__ void __launch_bounds__(kKvThreads) quant_kv4_kernel(QuantArgs a, uint32_t total) {
   pdl_wait();
   pdl_trigger();
   const uint32_t nb = static_cast<uint32_t>(a.nb[2]);
@@ -1334,9 +1335,12 @@ static mxs_status quantize_impl(const void *src, mxs_dtype dt, int64_t rows, int
   if (!tiny && !a.perm && !f32 && a.k_real[0] == 0 && a.k_real[1] == 0 && a.K % kBlock == 0 && aligned16(src) &&
       (ld * 2) % 32 == 0 && (reinterpret_cast<uintptr_t>(src) & 31u) == 0 && warps < (1ll << 31) &&
       (a.nb[2] <= 1 || warps * a.nb[2] < (1ll << 32))) {
-    // the K/V cache: one 4-bit segment, rows of whole blocks (32-byte aligned)
-    const int grid = static_cast<int>(std::min<int64_t>((warps + 256 * kKvU - 1) / (256 * kKvU), static_cast<int64_t>(nsm) * 8));
-    launch_pdl(quant_kv4_kernel, dim3(grid), dim3(256), 0, s, a, static_cast<uint32_t>(warps));
+    // the K/V cache: one 4-bit segment, rows of whole blocks (32-byte
+    // aligned); 128-thread CTAs, so that the SMs' shares differ by at most
+    // one small CTA
+    const int grid = static_cast<int>(std::min<int64_t>((warps + kKvThreads * kKvU - 1) / (kKvThreads * kKvU),
+                                                        static_cast<int64_t>(nsm) * 16));
+    launch_pdl(quant_kv4_kernel, dim3(grid), dim3(kKvThreads), 0, s, a, static_cast<uint32_t>(warps));
     count_launch();
     return cuda_status(cudaGetLastError());
   }
